@@ -1,0 +1,413 @@
+#!/usr/bin/env python
+"""Benchmark of the routed-expert MoE layer (512 experts, top-10, hidden
+3072, expert FFN 1024, SB3 up/gate + NL4 down) on B200.
+
+A step is one whole decode layer -- router + top-k, grouping, expert FFN
+with in-kernel dequantisation, combine -- for T tokens (default 3: one token
+plus two MTP drafts), through the C ABI (moe_layer_forward).  Steps rotate
+over `--layers` distinct layers whose experts are all resident in HBM
+(2.19 GB each), so no step finds its expert bytes in L2 (126 MB).
+
+Prints one JSON line (rank 0).  `--impl reference` times the fp64 CPU oracle
+on the same workload instead (a bounded sample per step).
+Multi-GPU (torchrun): independent replicas, one per GPU ("replicas only":
+the decode layer does not shard); max-over-ranks device time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = ("MoE-layer tokens/s (decode GB/s vs HBM peak; prefill TFLOP/s vs "
+          "bf16 peak)")
+UP_BYTES = 2 * synth.BIG.up_bytes          # up + gate of one expert
+DOWN_BYTES = synth.BIG.down_bytes
+BLOB = synth.BIG.blob_bytes
+WR_BYTES = synth.BIG.E * synth.BIG.H * 2   # bf16 router of one layer
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d["hbm_gbs"], d["bf16_tflops"], "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+# ------------------------------------------------------------ clocks ----
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str | None):
+        self.uuid = uuid
+        self.p = None
+
+    def start(self):
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}",
+               "--format=csv,noheader,nounits", "-lms", "200"]
+        if self.uuid:
+            cmd += ["-i", self.uuid]
+        try:
+            self.p = subprocess.Popen(cmd, stdout=subprocess.PIPE,
+                                      stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return None
+        self.p.terminate()
+        try:
+            out, _ = self.p.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.p.kill()
+            out, _ = self.p.communicate()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                 "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 8:
+                continue
+            try:
+                sm.append(float(f[0]))
+                mx.append(float(f[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------- oracle ----
+def oracle_step(layer: int, step: int, T: int, tokens, n_experts=None):
+    """The oracle on one decode step: routing of all T tokens, then the
+    expert FFNs and combine of `tokens` (all k experts each, or only the
+    first n_experts of one token).  Returns the number of tokens computed
+    (fractional when a token is sampled)."""
+    import oracle as o
+    shp = synth.BIG
+    x = o.bf16_to_f64(synth.gen_x(0, T, shp.H, step))
+    wr = o.bf16_to_f64(synth.gen_router(0, layer, shp.E, shp.H))
+    src = o.ExpertSource(shp.H, shp.F, shp.fmt_up_gate, shp.fmt_down,
+                         lambda e: synth.gen_expert_blob(shp, 0, layer, e))
+    logits = o.router_logits(x, wr, None)
+    idx, w = o.route(logits, shp.k)
+    done = 0.0
+    for t in tokens:
+        js = range(shp.k if n_experts is None else n_experts)
+        out = np.zeros(shp.H)
+        for j in js:
+            wu, wg, wd = src.weights(int(idx[t, j]))
+            _, y = o.expert_ffn(x[t:t + 1], wu, wg, wd)
+            out += w[t, j] * y[0]
+        done += len(js) / shp.k
+    return done
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info()
+             if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(T: int) -> dict:
+    t0 = time.perf_counter()
+    done = oracle_step(layer=0, step=0, T=T, tokens=range(T))
+    dt = time.perf_counter() - t0
+    return {"value": done / dt, "unit": "tokens/s", "cores": blas_threads(),
+            "kind": "oracle",
+            "sample": (f"one {T}-token decode step of layer 0: fp64 routing of "
+                       f"all {T} tokens, then dequantisation and fp64 SwiGLU "
+                       f"FFN of every chosen expert and the combine "
+                       f"({dt:.1f} s)")}
+
+
+def run_reference(args) -> None:
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    # bounded sample per step: one token's first n experts, n sized so
+    # that warm-up + steps stay within ~3 minutes
+    t0 = time.perf_counter()
+    oracle_step(0, 0, args.T, tokens=[0], n_experts=1)
+    per_expert = time.perf_counter() - t0
+    budget = 180.0 / max(1, args.steps + args.warmup)
+    n = int(max(1, min(synth.BIG.k, budget // max(per_expert, 1e-3))))
+    for i in range(args.warmup):
+        oracle_step(i % args.layers, i, args.T, tokens=[i % args.T],
+                    n_experts=n)
+    t0 = time.perf_counter()
+    done = 0.0
+    for i in range(args.steps):
+        s = args.warmup + i
+        done += oracle_step(s % args.layers, s, args.T, tokens=[s % args.T],
+                            n_experts=n)
+    dt = time.perf_counter() - t0
+    v = done / dt
+    line = {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * dt / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": workload_config(args),
+        "cpu_baseline": {"value": v, "unit": "tokens/s",
+                         "cores": blas_threads(), "kind": "oracle",
+                         "sample": (f"per step: routing of a {args.T}-token "
+                                    f"decode step, then {n} of the k=10 "
+                                    f"experts of one token (fp64 dequant + "
+                                    f"SwiGLU FFN); counted as {n}/10 token")},
+        "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(args) -> dict:
+    return {"workload": (f"decode, one MoE layer: {args.T} tokens, hidden "
+                         f"3072, expert FFN 1024, 512 experts, top-10, SB3 "
+                         f"up/gate + NL4 down"),
+            "T": args.T, "H": 3072, "F": 1024, "E": 512, "k": 10,
+            "layers_rotated": args.layers,
+            "l2": (f"inputs larger than L2: steps rotate over {args.layers} "
+                   f"resident layers x {synth.BIG.E * synth.BIG.blob_stride / 1e9:.2f}"
+                   f" GB of experts"),
+            "parallelism": f"replicas x{args.gpus}"}
+
+
+# ---------------------------------------------------------------- GPU ----
+class Layers:
+    """Resident layers: packed expert pools, router weights, inputs."""
+
+    def __init__(self, L: int, T: int, n_x: int = 64):
+        import torch
+        from synth.pools import build_pool, dev, layer_desc
+        import quantized_moe_expert_02_b200 as moe
+        self.moe = moe
+        shp = synth.BIG
+        self.L, self.T = L, T
+        self.pools = [build_pool(shp, 0, l) for l in range(L)]
+        self.descs = [layer_desc(shp, p) for p in self.pools]
+        self.wr = [dev(synth.gen_router(0, l, shp.E, shp.H)) for l in range(L)]
+        self.xs = [dev(synth.gen_x(0, T, shp.H, s)) for s in range(n_x)]
+        self.ws_bytes = moe.moe_layer_workspace_bytes(T, shp.k, shp.E, shp.H,
+                                                      shp.F)
+        self.ws = torch.zeros(self.ws_bytes, dtype=torch.uint8, device="cuda")
+        self.idx = torch.empty((T, shp.k), dtype=torch.int32, device="cuda")
+        self.w = torch.empty((T, shp.k), device="cuda")
+        self.out = torch.empty((T, shp.H), device="cuda")
+        # separate-call buffers (kernel timing pass)
+        self.ffn_ws_bytes = moe.moe_ffn_workspace_bytes(T, shp.k, shp.H, shp.F)
+        self.ffn_ws = torch.zeros(self.ffn_ws_bytes, dtype=torch.uint8,
+                                  device="cuda")
+        self.gws_bytes = moe.moe_group_workspace_bytes(T, shp.k, shp.E)
+        self.gws = torch.zeros(self.gws_bytes, dtype=torch.uint8,
+                               device="cuda")
+        self.lg = torch.empty((T, shp.E), device="cuda")
+        self.off = torch.empty(shp.E + 1, dtype=torch.int32, device="cuda")
+        self.pairs = torch.empty(T * shp.k, dtype=torch.int32, device="cuda")
+        self.act = torch.empty(shp.E, dtype=torch.int32, device="cuda")
+        self.na = torch.zeros(1, dtype=torch.int32, device="cuda")
+
+    def step(self, i: int, x=None):
+        shp = synth.BIG
+        l = i % self.L
+        xx = self.xs[i % len(self.xs)] if x is None else x
+        self.moe.moe_layer_forward(self.descs[l], xx, self.T, shp.k,
+                                   self.wr[l], None, None, None, self.out,
+                                   None, self.idx, self.w, None, self.ws,
+                                   self.ws_bytes)
+
+    def unique_experts(self, i: int) -> int:
+        """Distinct experts of step i (untimed: routing only)."""
+        import torch
+        shp = synth.BIG
+        l = i % self.L
+        self.moe.moe_route_topk(self.xs[i % len(self.xs)], self.T, shp.H,
+                                self.wr[l], shp.E, None, shp.k, self.idx,
+                                self.w, self.lg)
+        return int(torch.unique(self.idx).numel())
+
+
+def time_steps(layers, steps, warmup, fn):
+    import torch
+    for i in range(warmup):
+        fn(i)
+    torch.cuda.synchronize()
+    s = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(
+        enable_timing=True)
+    e0.record(s)
+    for i in range(steps):
+        fn(warmup + i)
+    e1.record(s)
+    e1.synchronize()
+    return e0.elapsed_time(e1)
+
+
+def kernel_timing(lay, steps, warmup):
+    """Average device time of the up/gate and down kernels, each timed with
+    CUDA events around its own C-ABI call (route and grouping untimed)."""
+    import torch
+    moe, shp, T = lay.moe, synth.BIG, lay.T
+    s = torch.cuda.current_stream()
+    t_up = t_dn = 0.0
+    u_sum = 0
+    for i in range(warmup + steps):
+        l = i % lay.L
+        x = lay.xs[i % len(lay.xs)]
+        moe.moe_route_topk(x, T, shp.H, lay.wr[l], shp.E, None, shp.k, lay.idx,
+                           lay.w, lay.lg)
+        moe.moe_group_tokens(lay.idx, T, shp.k, shp.E, lay.off, lay.pairs,
+                             lay.act, lay.na, lay.gws, lay.gws_bytes)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        ev[0].record(s)
+        moe.moe_expert_up_q(lay.descs[l], x, T, shp.k, lay.off, lay.pairs,
+                            lay.act, lay.na, None, lay.ffn_ws,
+                            lay.ffn_ws_bytes)
+        ev[1].record(s)
+        moe.moe_expert_down_q(lay.descs[l], T, shp.k, lay.off, lay.pairs,
+                              lay.act, lay.na, None, None, lay.w, None,
+                              lay.out, None, lay.ffn_ws, lay.ffn_ws_bytes)
+        ev[2].record(s)
+        ev[2].synchronize()
+        if i >= warmup:
+            t_up += ev[0].elapsed_time(ev[1])
+            t_dn += ev[1].elapsed_time(ev[2])
+            u_sum += int(lay.na.item())
+    return t_up / steps, t_dn / steps, u_sum / steps
+
+
+def run_ours(args) -> None:
+    import torch
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    lay = Layers(args.layers, args.T)
+    T, K, W = args.T, args.steps, args.warmup
+
+    # algorithmic bytes of the timed steps (routing replayed untimed)
+    uniq = [lay.unique_experts(W + i) for i in range(K)]
+    bytes_steps = sum(WR_BYTES + u * BLOB + T * 3072 * 6 for u in uniq)
+    torch.cuda.synchronize()
+
+    props = torch.cuda.get_device_properties(local)
+    uuid = getattr(props, "uuid", None)
+    clk = ClockSampler(f"GPU-{uuid}" if uuid else None)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clk.start()
+    ms = time_steps(lay, K, W, lay.step)
+    clocks = clk.stop()
+    if dist:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    tok_s = T * K * world / (ms / 1e3)
+
+    line = None
+    if rank == 0:
+        hbm, tf, src = peaks()
+        # dominant kernel: up/gate + SwiGLU, timed on its own
+        kt_up, kt_dn, u_avg = kernel_timing(lay, min(K, 50), 3)
+        up_bytes = u_avg * UP_BYTES + T * 3072 * 2 + u_avg * 32 * 512
+        dn_bytes = u_avg * DOWN_BYTES + u_avg * 32 * 512 + T * 3072 * 4
+        up_gbs = up_bytes / (kt_up * 1e-3) / 1e9
+        dn_gbs = dn_bytes / (kt_dn * 1e-3) / 1e9
+        # end to end: host x in, host out back, through the C ABI
+        xh = [torch.from_numpy(synth.gen_x(0, T, 3072, s).view(np.int16))
+              .pin_memory() for s in range(8)]
+        xd = torch.empty((T, 3072), dtype=torch.int16, device="cuda")
+        oh = torch.empty((T, 3072), dtype=torch.float32).pin_memory()
+
+        def e2e_step(i):
+            xd.copy_(xh[i % len(xh)], non_blocking=True)
+            lay.step(i, x=xd)
+            oh.copy_(lay.out, non_blocking=True)
+        ms_e2e = time_steps(lay, K, W, e2e_step)
+        line = {
+            "metric": METRIC, "value": tok_s, "unit": "tokens/s",
+            "n_gpus": world, "steps": K, "warmup": W,
+            "ms_per_step": ms / K, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": "int8 mma (s32 accumulate) + f32",
+            "data": "synthetic",
+            "config": workload_config(args),
+            "layer_gbs": bytes_steps / (ms / K * K * 1e-3) / 1e9,
+            "roofline": {
+                "bound": "hbm", "kernel": "ffn_up_decode (up/gate + SwiGLU)",
+                "achieved": up_gbs, "peak": hbm, "unit": "GB/s",
+                "frac": up_gbs / hbm, "peak_source": src,
+                "traffic": None,
+                "algorithmic_bytes_per_launch": up_bytes,
+                "avg_launch_ms": kt_up},
+            "kernels": {"ffn_up_decode_ms": kt_up, "ffn_down_decode_ms": kt_dn,
+                        "ffn_down_gbs": dn_gbs,
+                        "unique_experts_per_step": u_avg},
+            "e2e": {"value": T * K / (ms_e2e / 1e3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": T * 3072 * 2,
+                    "d2h_bytes_per_step": T * 3072 * 4},
+            "gpu_launches": 5 * K,
+            "clocks": clocks,
+        }
+        if not args.no_cpu_baseline and world == 1:
+            line["cpu_baseline"] = cpu_baseline(T)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    if line is not None:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--layers", type=int, default=16)
+    ap.add_argument("--T", type=int, default=3)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,270 @@
+/*
+ * moe.h -- C ABI of the routed Mixture-of-Experts FFN layer with low-bit
+ * block-quantised experts, for NVIDIA B200 (sm_100a).
+ *
+ * The layer is the one described by the "Avalon" README and its GGUF model
+ * card: 512 routed experts, 10 active per token, 48 layers; expert up/gate
+ * tensors in a 3.25-bpw super-block format (one scale per 256 weights, 4-bit
+ * sub-scales per 32 weights), down in a 4-bit non-uniform-codebook format,
+ * and each expert stored packed as up | gate | down (model card, "Files").
+ * The device-side expert-slot lookup follows the "Betelgeuse" post (VRAM
+ * slot pool with per-layer capacities, hits resolved on the device, only
+ * misses reported).
+ *
+ * Conventions (every entry point):
+ *   - Pointers are DEVICE pointers unless the comment says "host".
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy stream).
+ *   - The library never allocates memory, never synchronises the stream
+ *     (except moe_get_device_status) and never prints.  Memory is owned by
+ *     the caller; workspaces are sized with the *_workspace_bytes queries.
+ *   - Argument errors are returned synchronously (MOE_ERR_INVALID /
+ *     MOE_ERR_SHAPE / MOE_ERR_WORKSPACE) before anything is launched.  A
+ *     failed launch returns MOE_ERR_CUDA.  Bad data seen on the device (an
+ *     expert id out of range, a missing slot) never traps: the kernel sets
+ *     the workspace's device error word and skips the access; read it with
+ *     moe_get_device_status.
+ *   - Calls on different streams must use different workspaces.
+ *   - bf16 and fp16 values are passed as uint16_t bit patterns.
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID = 1,     /* null pointer, unknown enum, bad argument   */
+  MOE_ERR_SHAPE = 2,       /* a size the format or the kernels reject   */
+  MOE_ERR_UNSUPPORTED = 3, /* valid but not implemented                 */
+  MOE_ERR_CUDA = 4,        /* a CUDA launch or runtime call failed      */
+  MOE_ERR_DEVICE = 5,      /* the device error word was set             */
+  MOE_ERR_CAPACITY = 6,    /* slot pool: more misses than free slots    */
+  MOE_ERR_TIMEOUT = 7,     /* a bounded device wait gave up             */
+  MOE_ERR_WORKSPACE = 8    /* workspace missing or too small            */
+} moe_status;
+
+/* Expert weight formats (model card, "Files"; value semantics below).
+ *  MOE_Q4_B32 : 32 weights per block, fp16 scale d, 4-bit codes q,
+ *               w = d * (q - 8).
+ *  MOE_SB3_256: 256-weight super-block, fp16 scale d, eight 4-bit
+ *               sub-scales s_j (one per 32 weights), 3-bit codes q,
+ *               w = d * (2*s_j + 1) * (2*q - 7) / 8.   (3.1875 bpw)
+ *  MOE_NL4_B32: 32 weights per block, fp16 scale d, 4-bit codes q into the
+ *               int8 codebook {-127,-104,-83,-65,-49,-35,-22,-10,1,13,25,
+ *               38,53,69,89,113}, w = d * cb[q].             (4.5 bpw)
+ * Natural byte layout of a [rows x cols] tensor (rows of blocks along the
+ * columns, planar): codes plane, then (SB3 only) sub-scale plane, then the
+ * fp16 d plane.  SB3 codes: 96 bytes per super-block, a little-endian bit
+ * stream with code i at bit 3i; sub-scale j at bit 4j of a little-endian
+ * 32-bit word.  Q4/NL4 codes: weight i of a row in byte i/2, low nibble for
+ * even i.  The *packed* layout (same byte count) is the GPU tile layout
+ * that moe_pack_tensor produces and every compute entry point reads. */
+typedef enum { MOE_Q4_B32 = 1, MOE_SB3_256 = 2, MOE_NL4_B32 = 3 } moe_qfmt;
+
+/* One MoE layer's experts as the FFN sees them.
+ * Expert e's blob starts at pool + blob_index[e] * blob_stride and holds the
+ * packed tensors up [F x H] | gate [F x H] | down [H x F] back to back
+ * (model card: "Experts packed per layer (up | gate | down contiguous), so a
+ * GPU cache fill is one copy per expert").  blob_stride must be a multiple
+ * of 16 bytes and at least moe_blob_bytes(...). */
+typedef struct {
+  int H;            /* hidden size                      */
+  int F;            /* expert FFN width                 */
+  int E;            /* number of routed experts         */
+  int fmt_up_gate;  /* moe_qfmt of up and gate          */
+  int fmt_down;     /* moe_qfmt of down                 */
+  const uint8_t* pool;   /* device, packed expert blobs */
+  int64_t blob_stride;   /* bytes between blobs         */
+} moe_layer_desc;
+
+/* ---------------------------------------------------------- formats ---- */
+
+/* Bytes of one [rows x cols] tensor in format fmt (natural and packed
+ * layouts have the same size); 0 if fmt or the shape is invalid. */
+size_t moe_tensor_bytes(int fmt, int rows, int cols);
+
+/* Bytes of one expert blob (up | gate | down, unpadded). */
+size_t moe_blob_bytes(int fmt_up_gate, int fmt_down, int H, int F);
+
+/* Natural layout -> packed GPU tile layout (model card, "Files": the expert
+ * quant types; the packed layout is this library's own).  `natural` and
+ * `packed` are distinct device buffers of moe_tensor_bytes() bytes.
+ * Needs rows % 16 == 0, cols % 256 == 0 (SB3) or cols % 64 == 0 (Q4/NL4). */
+moe_status moe_pack_tensor(int fmt, const uint8_t* natural, int rows,
+                           int cols, uint8_t* packed, void* stream);
+
+/* Packed tensor -> fp32 [rows x cols] row-major.  The closed forms above
+ * are exact in fp32, so the result is bit-exact. */
+moe_status moe_dequant(int fmt, const uint8_t* packed, int rows, int cols,
+                       float* out, void* stream);
+
+/* ---------------------------------------------------------- routing ---- */
+
+/* Router and top-k ("Avalon": 512 experts, 10 active; softmax over all E,
+ * top-k by probability with ties to the lower index, renormalised).
+ *   x        bf16 [T x H] row-major        w_router bf16 [E x H] row-major
+ *   bias     fp32 [E] added to the logits, or NULL
+ *   topk_idx int32 [T x k]: experts by descending weight
+ *   topk_w   fp32 [T x k]: renormalised softmax weights (sum to 1)
+ *   logits_out fp32 [T x E] (the fp32 logits the selection used), or NULL
+ * Needs 1 <= k <= min(E, 32), E <= 4096, H % 8 == 0. */
+moe_status moe_route_topk(const uint16_t* x, int T, int H,
+                          const uint16_t* w_router, int E, const float* bias,
+                          int k, int32_t* topk_idx, float* topk_w,
+                          float* logits_out, void* stream);
+
+/* Workspace of moe_group_tokens. */
+size_t moe_group_workspace_bytes(int T, int k, int E);
+
+/* Token-to-expert grouping: the pairs p = t*k + j sorted by expert, stable
+ * in p ("MoE GEMM" grouping of the hybrid-placement post).
+ *   expert_offsets int32 [E+1]: pairs of expert e are
+ *                  pair_ids[expert_offsets[e] .. expert_offsets[e+1]-1]
+ *   pair_ids       int32 [T*k]
+ *   active         int32 [E]: experts with at least one pair, ascending;
+ *                  the first *n_active entries are valid
+ *   n_active       int32 [1] (device)
+ * An expert id outside [0, E) sets the device error word and is dropped. */
+moe_status moe_group_tokens(const int32_t* topk_idx, int T, int k, int E,
+                            int32_t* expert_offsets, int32_t* pair_ids,
+                            int32_t* active, int32_t* n_active, void* ws,
+                            size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------ slot cache ---- */
+
+/* Resolve one layer's chosen experts against its slot partition
+ * ("Betelgeuse": VRAM slot pool, per-layer capacities, an in-stream kernel
+ * resolves hits and reports only the misses).  One call per (step, layer).
+ *   slot_table  int32 [E]      local slot of expert e or -1   (updated)
+ *   slot_owner  int32 [n_slots] expert in each slot or -1     (updated)
+ *   last_use    uint32 [n_slots] stamp of each slot's last use (updated)
+ *   stamp       the stamp written to every slot this call uses or fills
+ *   blob_index  int32 [E]: for each chosen expert, slot_base + its slot
+ *   miss_expert int32 [T*k]: missed experts, ascending id
+ *   miss_slot   int32 [T*k]: the slot each miss was given (its victim)
+ *   n_miss      int32 [1] (device)
+ *   err         int32 [1] device error word (MOE_ERR_CAPACITY when the
+ *               misses outnumber the slots not used by this call; then
+ *               nothing is updated)
+ * Victim rule: the slot with the smallest last_use among the slots this
+ * call has not used or filled, ties to the lowest slot; the evicted
+ * expert's table entry becomes -1.  After the call the caller copies each
+ * missed expert's blob into pool + blob_index[e] * stride (one copy per
+ * expert) before the FFN runs on the same stream.  Needs T*k <= 1024,
+ * E <= 8192, n_slots <= 8192. */
+moe_status moe_slot_resolve(const int32_t* topk_idx, int T, int k, int E,
+                            int32_t* slot_table, int32_t* slot_owner,
+                            uint32_t* last_use, int n_slots, int slot_base,
+                            uint32_t stamp, int32_t* blob_index,
+                            int32_t* miss_expert, int32_t* miss_slot,
+                            int32_t* n_miss, int32_t* err, void* stream);
+
+/* ------------------------------------------------------- expert FFN ---- */
+
+/* Workspace of the FFN entry points (decode and prefill paths). */
+size_t moe_ffn_workspace_bytes(int T, int k, int H, int F);
+
+/* Zero a workspace before its first use (the kernels leave their counters
+ * at zero when they finish, so this is needed once). */
+moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream);
+
+/* Expert FFN on the grouped pairs: for every pair p of expert e,
+ *   h = silu(Wg_e x_t) * (Wu_e x_t),  y_pairs[p] = Wd_e h
+ * with the weights dequantised inside the kernel.
+ *   x          bf16 [T x H];  y_pairs fp32 [T*k x H] (row p = pair p)
+ *   expert_offsets/pair_ids/active/n_active: moe_group_tokens' outputs
+ *   blob_index int32 [E] or NULL (NULL: expert e's blob is blob e)
+ * Needs H, F multiples of 256 (SB3) or 64 (Q4/NL4) and of 16. */
+moe_status moe_expert_ffn_q(const moe_layer_desc* desc, const uint16_t* x,
+                            int T, int k, const int32_t* expert_offsets,
+                            const int32_t* pair_ids, const int32_t* active,
+                            const int32_t* n_active,
+                            const int32_t* blob_index, float* y_pairs,
+                            void* ws, size_t ws_bytes, void* stream);
+
+/* The two halves of moe_expert_ffn_q, callable on their own (same
+ * arguments and workspace; call up, then down, on the same stream).
+ *   moe_expert_up_q:   h = silu(Wg x) * (Wu x) for every pair, kept in the
+ *                      workspace (decode path: as int8 operands of the down
+ *                      projection with one scale per pair and 32 values).
+ *   moe_expert_down_q: y_pairs[p] = Wd h_p; y_pairs may be NULL when out is
+ *                      given; with out != NULL the weighted combine of
+ *                      moe_combine follows (topk_w, residual, out_bf16 as
+ *                      there). */
+moe_status moe_expert_up_q(const moe_layer_desc* desc, const uint16_t* x,
+                           int T, int k, const int32_t* expert_offsets,
+                           const int32_t* pair_ids, const int32_t* active,
+                           const int32_t* n_active, const int32_t* blob_index,
+                           void* ws, size_t ws_bytes, void* stream);
+moe_status moe_expert_down_q(const moe_layer_desc* desc, int T, int k,
+                             const int32_t* expert_offsets,
+                             const int32_t* pair_ids, const int32_t* active,
+                             const int32_t* n_active,
+                             const int32_t* blob_index, float* y_pairs,
+                             const float* topk_w, const float* residual,
+                             float* out, uint16_t* out_bf16, void* ws,
+                             size_t ws_bytes, void* stream);
+
+/* Weighted combine: out[t] = sum_j topk_w[t,j] * y_pairs[t*k+j]
+ * (+ residual[t]), summed in j order.  out fp32 [T x H]; out_bf16 bf16
+ * [T x H] or NULL; residual fp32 [T x H] or NULL (may alias out). */
+moe_status moe_combine(const float* y_pairs, const float* topk_w, int T,
+                       int k, int H, const float* residual, float* out,
+                       uint16_t* out_bf16, void* stream);
+
+/* Fused expert FFN + combine (the decode fast path): the same result as
+ * moe_expert_ffn_q followed by moe_combine, without the caller's y_pairs. */
+moe_status moe_expert_ffn_combine_q(const moe_layer_desc* desc,
+                                    const uint16_t* x, int T, int k,
+                                    const int32_t* expert_offsets,
+                                    const int32_t* pair_ids,
+                                    const int32_t* active,
+                                    const int32_t* n_active,
+                                    const int32_t* blob_index,
+                                    const float* topk_w,
+                                    const float* residual, float* out,
+                                    uint16_t* out_bf16, void* ws,
+                                    size_t ws_bytes, void* stream);
+
+/* x_out = bf16(r / sqrt(mean(r^2) + 1e-6)) per row: the input of the next
+ * layer of a pre-norm residual stack.  r fp32 [T x H]. */
+moe_status moe_rmsnorm_bf16(const float* r, int T, int H, uint16_t* x_out,
+                            void* stream);
+
+/* Workspace of moe_layer_forward. */
+size_t moe_layer_workspace_bytes(int T, int k, int E, int H, int F);
+
+/* One whole MoE layer: moe_route_topk, moe_group_tokens, then the fused
+ * expert FFN + combine, on one stream (the decode kernels when T <= 8 and
+ * T*k is at most the SM count, the general path otherwise).  The grouping
+ * lives in the workspace.  w_router bf16 [E x H]; bias fp32 [E] or NULL;
+ * blob_index as in moe_expert_ffn_q; residual/out/out_bf16 as in
+ * moe_combine; topk_idx int32 [T x k], topk_w fp32 [T x k] and logits_out
+ * fp32 [T x E] (or NULL) receive the routing.  The decode kernels are
+ * chained with programmatic dependent launch. */
+moe_status moe_layer_forward(const moe_layer_desc* desc, const uint16_t* x,
+                             int T, int k, const uint16_t* w_router,
+                             const float* bias, const int32_t* blob_index,
+                             const float* residual, float* out,
+                             uint16_t* out_bf16, int32_t* topk_idx,
+                             float* topk_w, float* logits_out, void* ws,
+                             size_t ws_bytes, void* stream);
+
+/* Synchronise `stream`, read the FFN/grouping workspace's device error word
+ * into *host_err (host pointer, may be NULL) and clear it.  Returns
+ * MOE_ERR_DEVICE if it was set, MOE_OK otherwise. */
+moe_status moe_get_device_status(void* ws, int32_t* host_err, void* stream);
+
+/* Human-readable name of a status code (static string). */
+const char* moe_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H_ */

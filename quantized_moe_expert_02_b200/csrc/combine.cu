@@ -1,0 +1,75 @@
+// Weighted combine of the k expert outputs of each token, and the
+// row-wise RMS normalisation used between the layers of a stack.
+#include "moe_internal.cuh"
+
+namespace moe {
+
+// out[t,h] = sum_j w[t,j] * y[t*k+j, h]  (j ascending)  + residual[t,h]
+__global__ void combine_kernel(const float* __restrict__ y,
+                               const float* __restrict__ w, int T, int k,
+                               int H, const float* residual, float* out,
+                               uint16_t* __restrict__ out_bf16) {
+  const int64_t n = (int64_t)T * H;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int t = (int)(i / H), h = (int)(i % H);
+    float acc = 0.f;
+    for (int j = 0; j < k; ++j)
+      acc = fmaf(w[(int64_t)t * k + j], y[((int64_t)t * k + j) * H + h], acc);
+    if (residual) acc += residual[i];
+    out[i] = acc;
+    if (out_bf16) out_bf16[i] = f32_to_bf16_rne(acc);
+  }
+}
+
+// x = bf16(r / sqrt(mean(r^2) + eps)), one block per row.
+__global__ void __launch_bounds__(256)
+    rmsnorm_bf16_kernel(const float* __restrict__ r, int H,
+                        uint16_t* __restrict__ x) {
+  __shared__ float red[8];
+  const float* row = r + (int64_t)blockIdx.x * H;
+  float s = 0.f;
+  for (int h = threadIdx.x; h < H; h += blockDim.x) s = fmaf(row[h], row[h], s);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = s;
+  __syncthreads();
+  float tot = 0.f;
+  for (int i = 0; i < (int)(blockDim.x >> 5); ++i) tot += red[i];
+  const float inv = 1.0f / sqrtf(tot / (float)H + 1e-6f);
+  for (int h = threadIdx.x; h < H; h += blockDim.x)
+    x[(int64_t)blockIdx.x * H + h] = f32_to_bf16_rne(row[h] * inv);
+}
+
+moe_status launch_combine(const float* y, const float* w, int T, int k,
+                          int H, const float* residual, float* out,
+                          uint16_t* out_bf16, cudaStream_t s) {
+  const int64_t n = (int64_t)T * H;
+  int64_t g = (n + 255) / 256;
+  if (g > (int64_t)num_sms() * 16) g = (int64_t)num_sms() * 16;
+  combine_kernel<<<(int)g, 256, 0, s>>>(y, w, T, k, H, residual, out,
+                                        out_bf16);
+  return launch_status();
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" moe_status moe_combine(const float* y_pairs, const float* topk_w,
+                                  int T, int k, int H, const float* residual,
+                                  float* out, uint16_t* out_bf16,
+                                  void* stream) {
+  if (!y_pairs || !topk_w || !out) return MOE_ERR_INVALID;
+  if (T <= 0 || k <= 0 || H <= 0) return MOE_ERR_SHAPE;
+  return launch_combine(y_pairs, topk_w, T, k, H, residual, out, out_bf16,
+                        (cudaStream_t)stream);
+}
+
+extern "C" moe_status moe_rmsnorm_bf16(const float* r, int T, int H,
+                                       uint16_t* x_out, void* stream) {
+  if (!r || !x_out) return MOE_ERR_INVALID;
+  if (T <= 0 || H <= 0) return MOE_ERR_SHAPE;
+  rmsnorm_bf16_kernel<<<T, 256, 0, (cudaStream_t)stream>>>(r, H, x_out);
+  return launch_status();
+}

@@ -1,0 +1,658 @@
+// Expert FFN, decode path (T <= 8 tokens): fused dequant-GEMV on the int8
+// tensor-core path.  HBM-bound: every expert byte is read once.
+//
+// Structure (both kernels): a persistent grid of one block per SM; warp 8
+// is a producer that streams packed expert tiles global -> shared memory
+// with 1-D bulk copies (cp.async.bulk) into a ring of stages guarded by
+// mbarriers; warps 0..7 are two consumer groups of four warps that take
+// alternate units.  A consumer turns the codes of its tile into the int8
+// A fragment of mma.m16n8k32 with byte-table lookups (prmt), and the
+// activations enter as the B fragment split into two int8 halves
+// (v = 256*hi + lo, v = round(a * 2^sigma), |v| < 2^14), so the products
+// and their sums over a 32-block are exact integers.  Scales are applied
+// in fp32 per block (per super-block for SB3, whose sub-scales multiply
+// the integer partials).
+//
+// Up/gate kernel: unit = (expert, 32 rows of F, quarter of H).  Its four
+// chunks (up/gate x two 16-row tiles) go to the four warps of a group.  The
+// partials of the quarters are summed in fixed order by whichever block
+// finishes a 32-row tile last (arrival counter), which applies SwiGLU and
+// writes h of each of the expert's tokens as the int8 B fragments of the
+// down projection (one scale per token and 32-block).
+//
+// Down kernel: unit = (expert, 16 rows of H), all of F; the four warps of
+// a group split F.  y of each pair is written per row tile; with the fused
+// combine, the block that finishes a row tile last (over all experts) sums
+// the k expert outputs of each token in j order.
+#include "moe_internal.cuh"
+
+namespace moe {
+
+constexpr int NGRP = 2;                    // consumer groups
+constexpr int GRP_WARPS = 4;               // warps per group
+constexpr int DEC_THREADS = (NGRP * GRP_WARPS + 1) * 32;
+constexpr int PROD_WARP = NGRP * GRP_WARPS;
+constexpr int UP_STAGES = 4;
+constexpr int DN_STAGES = 8;
+
+struct DecParams {
+  const uint8_t* pool;
+  int64_t stride;
+  const int32_t* blob_index;
+  int E, H, F, T, k;
+  int64_t gate_off, down_off;
+  const uint16_t* x;
+  const int32_t* offsets;
+  const int32_t* pair_ids;
+  const int32_t* active;
+  const int32_t* n_active;
+  int32_t* err;
+  int32_t* up_cnt;
+  int32_t* dn_cnt;
+  float* up_part;
+  uint32_t* bfrag;
+  float* bscale;
+  float* y;               // y of each pair [T*k][H]
+  const float* topk_w;    // fused combine (out != nullptr)
+  const float* residual;
+  float* out;
+  uint16_t* out_bf16;
+};
+
+__device__ __forceinline__ const uint8_t* blob_of(const DecParams& p, int e) {
+  if (e < 0 || e >= p.E) { set_err(p.err, MOE_ERR_DEVICE); return nullptr; }
+  const int64_t b = p.blob_index ? (int64_t)__ldcg(p.blob_index + e) : e;
+  if (b < 0) { set_err(p.err, MOE_ERR_DEVICE); return nullptr; }
+  return p.pool + b * p.stride;
+}
+
+// ---- tile decoders ----------------------------------------------------
+// SB3 tile (16 x 256): acc[nt][0/1] += rows g / g+8 for column token
+// (lane&3) + 4nt.  xfb = B fragments of the tile's first 32-block,
+// [blk][BF_NT][32][2] words; xs[nt] = 2^-sigma_t / 8 of the lane's token.
+__device__ __forceinline__ void piece_sb3(const uint8_t* tp,
+                                          const uint32_t* xfb, int NT,
+                                          const float (&xs)[2],
+                                          float (&acc)[2][2], int lane) {
+  const int g = lane >> 2;
+  const uint4 L0 = *reinterpret_cast<const uint4*>(tp + 16 * lane);
+  const uint4 L1 = *reinterpret_cast<const uint4*>(tp + 512 + 16 * lane);
+  const uint4 HV = *reinterpret_cast<const uint4*>(tp + 1024 + 16 * lane);
+  const uint2 SC = *reinterpret_cast<const uint2*>(tp + 1536 + 8 * g);
+  const uint32_t DD = *reinterpret_cast<const uint32_t*>(tp + 1600 + 4 * g);
+  const uint32_t lo[8] = {L0.x, L0.y, L0.z, L0.w, L1.x, L1.y, L1.z, L1.w};
+  const uint32_t hi[4] = {HV.x, HV.y, HV.z, HV.w};
+  int32_t S[2][2] = {{0, 0}, {0, 0}};
+  const int32_t zero[4] = {0, 0, 0, 0};
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const uint32_t LO = lo[j], HH = hi[j >> 1];
+    const uint32_t ha = (j & 1) ? HH : (HH << 2);
+    const uint32_t hb = (j & 1) ? (HH >> 1) : (HH << 1);
+    const uint32_t sa = (LO & 0x33333333u) | (ha & 0x44444444u);
+    const uint32_t sb = ((LO >> 2) & 0x33333333u) | (hb & 0x44444444u);
+    uint32_t a[4];
+    a[0] = prmt(SB3_TAB0, SB3_TAB1, sa);
+    a[1] = prmt(SB3_TAB0, SB3_TAB1, sa >> 16);
+    a[2] = prmt(SB3_TAB0, SB3_TAB1, sb);
+    a[3] = prmt(SB3_TAB0, SB3_TAB1, sb >> 16);
+    const int mg = (int)((SC.x >> (4 * j)) & 15u) * 2 + 1;
+    const int mg8 = (int)((SC.y >> (4 * j)) & 15u) * 2 + 1;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      if (nt < NT) {
+        const uint2 b = *reinterpret_cast<const uint2*>(
+            xfb + (j * BF_NT + nt) * 64 + 2 * lane);
+        int32_t d[4];
+        mma_s8(d, a, b.x, b.y, zero);
+        S[nt][0] += (d[0] * 256 + d[1]) * mg;
+        S[nt][1] += (d[2] * 256 + d[3]) * mg8;
+      }
+    }
+  }
+  const float2 dv = __half22float2(*reinterpret_cast<const __half2*>(&DD));
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt) {
+    if (nt < NT) {
+      acc[nt][0] = fmaf((float)S[nt][0], dv.x * xs[nt], acc[nt][0]);
+      acc[nt][1] = fmaf((float)S[nt][1], dv.y * xs[nt], acc[nt][1]);
+    }
+  }
+}
+
+// Q4 / NL4 tile (16 x 64, two 32-blocks).  cs = column scales of the
+// lane's columns: value for (local block bl, nt) at cs[bl*cs_stride + 4nt].
+template <int FMT>
+__device__ __forceinline__ void piece_b32(const uint8_t* tp,
+                                          const uint32_t* bfb, int NT,
+                                          const float* cs, int cs_stride,
+                                          float (&acc)[2][2], int lane) {
+  constexpr uint32_t TA0 = FMT == MOE_NL4_B32 ? NL4_TA0 : Q4_TA0;
+  constexpr uint32_t TA1 = FMT == MOE_NL4_B32 ? NL4_TA1 : Q4_TA1;
+  constexpr uint32_t TB0 = FMT == MOE_NL4_B32 ? NL4_TB0 : Q4_TB0;
+  constexpr uint32_t TB1 = FMT == MOE_NL4_B32 ? NL4_TB1 : Q4_TB1;
+  const int g = lane >> 2;
+  const uint4 W = *reinterpret_cast<const uint4*>(tp + 16 * lane);
+  const uint2 DV = *reinterpret_cast<const uint2*>(tp + 512 + 8 * g);
+  const float2 dg = __half22float2(*reinterpret_cast<const __half2*>(&DV.x));
+  const float2 dg8 = __half22float2(*reinterpret_cast<const __half2*>(&DV.y));
+  const uint32_t w[4] = {W.x, W.y, W.z, W.w};
+  const int32_t zero[4] = {0, 0, 0, 0};
+#pragma unroll
+  for (int bl = 0; bl < 2; ++bl) {
+    const uint32_t w0 = w[2 * bl], w1 = w[2 * bl + 1];
+    const uint32_t x0 = w0 ^ 0x88888888u, x1 = w1 ^ 0x88888888u;
+    uint32_t a1[4], a2[4];
+    a1[0] = prmt(TA0, TA1, w0);
+    a1[1] = prmt(TA0, TA1, w0 >> 16);
+    a1[2] = prmt(TA0, TA1, w1);
+    a1[3] = prmt(TA0, TA1, w1 >> 16);
+    a2[0] = prmt(TB0, TB1, x0);
+    a2[1] = prmt(TB0, TB1, x0 >> 16);
+    a2[2] = prmt(TB0, TB1, x1);
+    a2[3] = prmt(TB0, TB1, x1 >> 16);
+    const float d0 = bl ? dg.y : dg.x, d8 = bl ? dg8.y : dg8.x;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      if (nt < NT) {
+        const uint2 b = *reinterpret_cast<const uint2*>(
+            bfb + (bl * BF_NT + nt) * 64 + 2 * lane);
+        int32_t d[4];
+        mma_s8(d, a1, b.x, b.y, zero);
+        mma_s8(d, a2, b.x, b.y, d);
+        const float c = cs[bl * cs_stride + 4 * nt];
+        acc[nt][0] = fmaf((float)(d[0] * 256 + d[1]), d0 * c, acc[nt][0]);
+        acc[nt][1] = fmaf((float)(d[2] * 256 + d[3]), d8 * c, acc[nt][1]);
+      }
+    }
+  }
+}
+
+// 2^sigma with sigma chosen so that max|v| * 2^sigma < 2^14.
+__device__ __forceinline__ int pow2_sigma(float m) {
+  if (!(m > 0.f) || !isfinite(m)) return 0;
+  const int e = (int)((__float_as_uint(m) >> 23) & 255u) - 126;  // m < 2^e
+  int s = 14 - e;
+  if (s > 100) s = 100;
+  if (s < -100) s = -100;
+  return s;
+}
+__device__ __forceinline__ float exp2i(int s) {
+  return __uint_as_float((uint32_t)(127 + s) << 23);
+}
+
+// ---------------------------------------------------------------- up ---
+template <int FMT>
+__global__ void __launch_bounds__(DEC_THREADS, 1)
+    ffn_up_decode_kernel(DecParams p) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  constexpr int TB = FMT == MOE_SB3_256 ? SB3_TILE_BYTES : B32_TILE_BYTES;
+  constexpr int TC = FMT == MOE_SB3_256 ? SB3_TILE_COLS : B32_TILE_COLS;
+  const int nk = p.H / TC;
+  const int nsplit = nk < NSPLIT_MAX ? nk : NSPLIT_MAX;
+  const int kmax = (nk + nsplit - 1) / nsplit;
+  const int chunk_bytes = kmax * TB;
+  const int stage_bytes = 4 * chunk_bytes;
+  const int NT = (p.T + 3) / 4;
+  const int nblk = p.H / 32;
+  const int nrt = p.F / 32;
+  uint8_t* stages = smem;
+  uint32_t* xf = reinterpret_cast<uint32_t*>(smem + UP_STAGES * stage_bytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(xf + nblk * BF_NT * 64);
+  uint64_t* empty = full + UP_STAGES;
+  float* xsc = reinterpret_cast<float*>(empty + UP_STAGES);  // [8]
+  int* xsig = reinterpret_cast<int*>(xsc + DEC_TMAX);        // [8]
+  int* flag = xsig + DEC_TMAX;                               // [NGRP]
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {
+    for (int s = 0; s < UP_STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], GRP_WARPS);
+    }
+    fence_mbar_init();
+  }
+  // per-token scale of the activations (x is an input of this layer)
+  for (int t = warp; t < p.T; t += DEC_THREADS / 32) {
+    float m = 0.f;
+    for (int h = lane; h < p.H; h += 32)
+      m = fmaxf(m, fabsf(bf16_to_f32(p.x[(int64_t)t * p.H + h])));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (lane == 0) {
+      const int s = pow2_sigma(m);
+      xsig[t] = s;
+      xsc[t] = exp2i(-s) * (FMT == MOE_SB3_256 ? 0.125f : 1.0f);
+    }
+  }
+  __syncthreads();
+  // B fragments of x: [blk][nt][lane][reg], 4 int8 of column n = g:
+  // token 4nt + n/2, n even = high half, odd = low half of v.
+  for (int i = tid; i < nblk * BF_NT * 64; i += DEC_THREADS) {
+    const int reg = i & 1, L = (i >> 1) & 31, nt = (i >> 6) % BF_NT;
+    const int blk = i / (64 * BF_NT);
+    const int n = L >> 2, c = L & 3;
+    const int t = 4 * nt + (n >> 1);
+    uint32_t word = 0;
+    if (t < p.T) {
+      const float sc = exp2i(xsig[t]);
+      const uint16_t* xr = p.x + (int64_t)t * p.H + 32 * blk + 16 * reg + 4 * c;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int v = __float2int_rn(bf16_to_f32(xr[q]) * sc);
+        const int hi = (v + 128) >> 8, lo = v - hi * 256;
+        word |= (uint32_t)((n & 1) ? lo : hi) << (8 * q) & (0xFFu << (8 * q));
+      }
+    }
+    xf[i] = word;
+  }
+  __syncthreads();
+  grid_dep_wait();      // routing of this layer is complete and visible
+  grid_dep_launch();
+
+  const int n_act = *p.n_active;
+  const int64_t n_units = (int64_t)n_act * nrt * nsplit;
+  const int64_t v0 = n_units * blockIdx.x / gridDim.x;
+  const int64_t v1 = n_units * (blockIdx.x + 1) / gridDim.x;
+  const int nu = (int)(v1 - v0);
+
+  if (warp == PROD_WARP) {
+    if (lane == 0) {
+      for (int i = 0; i < nu; ++i) {
+        const int s = i % UP_STAGES;
+        if (i >= UP_STAGES)
+          mbar_wait(&empty[s], ((i / UP_STAGES) - 1) & 1, p.err);
+        const int64_t v = v0 + i;
+        const int u = (int)(v / (nrt * nsplit));
+        const int rt = (int)((v / nsplit) % nrt), kq = (int)(v % nsplit);
+        const int k0 = kq * nk / nsplit, k1 = (kq + 1) * nk / nsplit;
+        const uint32_t nbytes = (uint32_t)((k1 - k0) * TB);
+        const uint8_t* blob = blob_of(p, p.active[u]);
+        if (!blob) { mbar_arrive_expect_tx(&full[s], 0); continue; }
+        mbar_arrive_expect_tx(&full[s], 4 * nbytes);
+        for (int w = 0; w < 4; ++w) {
+          const int tz = w >> 1, rg = w & 1;
+          const uint8_t* src = blob + tz * p.gate_off +
+                               ((int64_t)(2 * rt + rg) * nk + k0) * TB;
+          bulk_g2s(stages + s * stage_bytes + w * chunk_bytes, src, nbytes,
+                   &full[s]);
+        }
+      }
+    }
+    return;
+  }
+
+  const int grp = warp / GRP_WARPS, wg = warp % GRP_WARPS;
+  const int gtid = tid - grp * GRP_WARPS * 32;   // 0..127 within the group
+  const int tz = wg >> 1, rg = wg & 1;
+  const int g = lane >> 2, c = lane & 3;
+  float xs[2];
+  xs[0] = xsc[c];
+  xs[1] = xsc[4 + c];
+  for (int i = grp; i < nu; i += NGRP) {
+    const int s = i % UP_STAGES;
+    mbar_wait(&full[s], (i / UP_STAGES) & 1, p.err);
+    const int64_t v = v0 + i;
+    const int u = (int)(v / (nrt * nsplit));
+    const int rt = (int)((v / nsplit) % nrt), kq = (int)(v % nsplit);
+    const int k0 = kq * nk / nsplit, k1 = (kq + 1) * nk / nsplit;
+    float acc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+    const uint8_t* chunk = stages + s * stage_bytes + wg * chunk_bytes;
+    for (int kt = 0; kt < k1 - k0; ++kt) {
+      const int blk0 = (k0 + kt) * (TC / 32);
+      if (FMT == MOE_SB3_256)
+        piece_sb3(chunk + kt * TB, xf + blk0 * BF_NT * 64, NT, xs, acc, lane);
+      else
+        piece_b32<FMT>(chunk + kt * TB, xf + blk0 * BF_NT * 64, NT, xsc + c,
+                       0, acc, lane);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
+    // split-K partial of this quarter
+    float* part = p.up_part +
+                  ((((int64_t)u * nrt + rt) * NSPLIT_MAX + kq) * 2 + tz) * 256;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      const int t = 4 * nt + c;
+      if (t < p.T) {
+        part[(rg * 16 + g) * 8 + t] = acc[nt][0];
+        part[(rg * 16 + g + 8) * 8 + t] = acc[nt][1];
+      }
+    }
+    __threadfence();
+    named_bar_sync(1 + grp, GRP_WARPS * 32);
+    if (gtid == 0) {
+      const int old = atomicAdd(&p.up_cnt[u * nrt + rt], 1);
+      flag[grp] = (old == nsplit - 1);
+    }
+    named_bar_sync(1 + grp, GRP_WARPS * 32);
+    if (flag[grp]) {
+      __threadfence();
+      // finalize the 32-row tile: SwiGLU, then the down B fragments
+      const int e = p.active[u];
+      const int off = p.offsets[e], Tu = p.offsets[e + 1] - off;
+      const int slot = gtid >> 4, r0 = (gtid & 15) * 2;
+      float hv[2] = {0.f, 0.f};
+      if (slot < Tu) {
+        const int pp = p.pair_ids[off + slot];
+        const int t = pp / p.k;
+        const float* pb = p.up_part +
+                          (((int64_t)u * nrt + rt) * NSPLIT_MAX) * 2 * 256;
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          const int r = r0 + q;
+          float su = 0.f, sg = 0.f;
+          for (int kk = 0; kk < nsplit; ++kk) {
+            su += __ldcg(pb + (kk * 2 + 0) * 256 + r * 8 + t);
+            sg += __ldcg(pb + (kk * 2 + 1) * 256 + r * 8 + t);
+          }
+          hv[q] = sg / (1.0f + expf(-sg)) * su;
+        }
+      }
+      float m = fmaxf(fabsf(hv[0]), fabsf(hv[1]));
+#pragma unroll
+      for (int o = 8; o > 0; o >>= 1)
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      const int sig = pow2_sigma(m);
+      const float sc = exp2i(sig);
+      uint8_t* bf8 = reinterpret_cast<uint8_t*>(p.bfrag);
+      const int nt = slot >> 2, nhi = 2 * (slot & 3);
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        const int r = r0 + q;
+        const int vq = slot < Tu ? __float2int_rn(hv[q] * sc) : 0;
+        const int hi = (vq + 128) >> 8, lo = vq - hi * 256;
+        const int cc = (r & 15) >> 2, reg = r >> 4, byte = r & 3;
+        const int64_t base =
+            (((int64_t)u * nrt + rt) * BF_NT + nt) * 32 * 8 + reg * 4 + byte;
+        bf8[base + (4 * nhi + cc) * 8] = (uint8_t)hi;
+        bf8[base + (4 * (nhi + 1) + cc) * 8] = (uint8_t)lo;
+      }
+      if ((gtid & 15) == 0)
+        p.bscale[((int64_t)u * nrt + rt) * 8 + slot] = exp2i(-sig);
+      if (gtid == 0) p.up_cnt[u * nrt + rt] = 0;
+    }
+  }
+}
+
+// -------------------------------------------------------------- down ---
+template <int FMT>
+__global__ void __launch_bounds__(DEC_THREADS, 1)
+    ffn_down_decode_kernel(DecParams p) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int nk = p.F / B32_TILE_COLS;
+  const int nrt = p.H / TILE_ROWS;
+  const int nblk = p.F / 32;
+  const int stage_bytes = nk * B32_TILE_BYTES;
+  const int NT = (p.T + 3) / 4;
+  const int bwords = nblk * BF_NT * 64;
+  uint8_t* stages = smem;
+  uint32_t* bbuf = reinterpret_cast<uint32_t*>(smem + DN_STAGES * stage_bytes);
+  float* bsc = reinterpret_cast<float*>(bbuf + 2 * bwords);     // [2][nblk*8]
+  float* red = bsc + 2 * nblk * 8;                 // [NGRP][4][2][2][32]
+  uint64_t* full = reinterpret_cast<uint64_t*>(red + NGRP * 4 * 2 * 2 * 32);
+  uint64_t* empty = full + DN_STAGES;
+  uint64_t* bfull = empty + DN_STAGES;
+  int* flag = reinterpret_cast<int*>(bfull + 1);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {
+    for (int s = 0; s < DN_STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], GRP_WARPS);
+    }
+    mbar_init(bfull, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  // The routing (two launches back) is complete: the up kernel waited for
+  // it before it allowed this grid to start.  Read it through L2.
+  const int n_act = __ldcg(p.n_active);
+  const int64_t n_units = (int64_t)n_act * nrt;
+  const int64_t v0 = n_units * blockIdx.x / gridDim.x;
+  const int64_t v1 = n_units * (blockIdx.x + 1) / gridDim.x;
+  const int nu = (int)(v1 - v0);
+  const int u_first = nu > 0 ? (int)(v0 / nrt) : 0;
+  const int u_last = nu > 0 ? (int)((v1 - 1) / nrt) : -1;
+
+  if (warp == PROD_WARP) {
+    if (lane == 0) {
+      auto issue = [&](int i) {
+        const int s = i % DN_STAGES;
+        const int64_t v = v0 + i;
+        const int u = (int)(v / nrt), rt = (int)(v % nrt);
+        const uint8_t* blob = blob_of(p, __ldcg(p.active + u));
+        if (!blob) { mbar_arrive_expect_tx(&full[s], 0); return; }
+        mbar_arrive_expect_tx(&full[s], (uint32_t)stage_bytes);
+        bulk_g2s(stages + s * stage_bytes,
+                 blob + p.down_off + (int64_t)rt * stage_bytes,
+                 (uint32_t)stage_bytes, &full[s]);
+      };
+      const int pre = nu < DN_STAGES ? nu : DN_STAGES;
+      for (int i = 0; i < pre; ++i) issue(i);
+      grid_dep_wait();    // the up kernel's B fragments are complete
+      grid_dep_launch();
+      if (u_last >= u_first && u_last - u_first <= 1) {
+        const uint32_t nb = (uint32_t)(bwords * 4 + nblk * 8 * 4);
+        mbar_arrive_expect_tx(bfull, (u_last - u_first + 1) * nb);
+        for (int u = u_first; u <= u_last; ++u) {
+          const int bi = u - u_first;
+          bulk_g2s(bbuf + bi * bwords, p.bfrag + (int64_t)u * bwords,
+                   (uint32_t)(bwords * 4), bfull);
+          bulk_g2s(bsc + bi * nblk * 8, p.bscale + (int64_t)u * nblk * 8,
+                   (uint32_t)(nblk * 8 * 4), bfull);
+        }
+      } else {
+        if (u_last - u_first > 1) set_err(p.err, MOE_ERR_DEVICE);
+        mbar_arrive_expect_tx(bfull, 0);
+      }
+      for (int i = pre; i < nu; ++i) {
+        const int s = i % DN_STAGES;
+        mbar_wait(&empty[s], ((i / DN_STAGES) - 1) & 1, p.err);
+        issue(i);
+      }
+    }
+    return;
+  }
+
+  grid_dep_wait();
+  const int grp = warp / GRP_WARPS, wg = warp % GRP_WARPS;
+  const int gtid = tid - grp * GRP_WARPS * 32;
+  const int c = lane & 3;
+  mbar_wait(bfull, 0, p.err);
+  const int kt0 = wg * nk / GRP_WARPS, kt1 = (wg + 1) * nk / GRP_WARPS;
+  float* myred = red + grp * (4 * 2 * 2 * 32);
+  for (int i = grp; i < nu; i += NGRP) {
+    const int s = i % DN_STAGES;
+    mbar_wait(&full[s], (i / DN_STAGES) & 1, p.err);
+    const int64_t v = v0 + i;
+    const int u = (int)(v / nrt), rt = (int)(v % nrt);
+    const int bi = u - u_first;
+    const bool bok = bi >= 0 && bi <= 1;
+    float acc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+    if (bok) {
+      const uint32_t* bb = bbuf + bi * bwords;
+      const float* bs = bsc + bi * nblk * 8;
+      for (int kt = kt0; kt < kt1; ++kt)
+        piece_b32<FMT>(stages + s * stage_bytes + kt * B32_TILE_BYTES,
+                       bb + (2 * kt) * BF_NT * 64, NT, bs + (2 * kt) * 8 + c,
+                       8, acc, lane);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+        myred[((wg * 2 + nt) * 2 + h) * 32 + lane] = acc[nt][h];
+    named_bar_sync(1 + grp, GRP_WARPS * 32);
+    {
+      const int rho = gtid >> 3, slot = gtid & 7;
+      const int L = 4 * (rho & 7) + (slot & 3), nt = slot >> 2, h = rho >> 3;
+      float yv = 0.f;
+#pragma unroll
+      for (int w = 0; w < GRP_WARPS; ++w)
+        yv += myred[((w * 2 + nt) * 2 + h) * 32 + L];
+      const int e = __ldcg(p.active + u);
+      const int off = __ldcg(p.offsets + e);
+      const int Tu = __ldcg(p.offsets + e + 1) - off;
+      if (slot < Tu && bok) {
+        const int pp = __ldcg(p.pair_ids + off + slot);
+        p.y[(int64_t)pp * p.H + 16 * rt + rho] = yv;
+      }
+    }
+    if (p.out) {
+      __threadfence();
+      named_bar_sync(1 + grp, GRP_WARPS * 32);
+      if (gtid == 0) {
+        const int old = atomicAdd(&p.dn_cnt[rt], 1);
+        flag[grp] = (old == n_act - 1);
+      }
+      named_bar_sync(1 + grp, GRP_WARPS * 32);
+      if (flag[grp]) {
+        __threadfence();
+        const int t = gtid >> 4, rho = gtid & 15;
+        if (t < p.T) {
+          const int64_t col = 16 * rt + rho;
+          float a = 0.f;
+          for (int j = 0; j < p.k; ++j) {
+            const int64_t pp = (int64_t)t * p.k + j;
+            a = fmaf(p.topk_w[pp], __ldcg(p.y + pp * p.H + col), a);
+          }
+          if (p.residual) a += p.residual[(int64_t)t * p.H + col];
+          p.out[(int64_t)t * p.H + col] = a;
+          if (p.out_bf16) p.out_bf16[(int64_t)t * p.H + col] = f32_to_bf16_rne(a);
+        }
+        if (gtid == 0) p.dn_cnt[rt] = 0;
+      }
+    }
+    named_bar_sync(1 + grp, GRP_WARPS * 32);
+  }
+}
+
+// ------------------------------------------------------------ launch ---
+static size_t up_smem_bytes(int fmt, int H) {
+  const int TB = tile_bytes(fmt), TC = tile_cols(fmt);
+  const int nk = H / TC;
+  const int nsplit = nk < NSPLIT_MAX ? nk : NSPLIT_MAX;
+  const int kmax = (nk + nsplit - 1) / nsplit;
+  return (size_t)UP_STAGES * 4 * kmax * TB + (size_t)(H / 32) * BF_NT * 64 * 4 +
+         2 * UP_STAGES * 8 + 2 * DEC_TMAX * 4 + 64;
+}
+static size_t dn_smem_bytes(int F) {
+  const int nk = F / B32_TILE_COLS, nblk = F / 32;
+  return (size_t)DN_STAGES * nk * B32_TILE_BYTES +
+         (size_t)2 * nblk * BF_NT * 64 * 4 + (size_t)2 * nblk * 8 * 4 +
+         (size_t)NGRP * 4 * 2 * 2 * 32 * 4 + (2 * DN_STAGES + 1) * 8 + 64;
+}
+
+bool ffn_decode_supported(const moe_layer_desc& d, int T, int k) {
+  if (T < 1 || T > DEC_TMAX) return false;
+  if (d.fmt_down != MOE_NL4_B32 && d.fmt_down != MOE_Q4_B32) return false;
+  if (d.F % 32 != 0 || d.H % 16 != 0) return false;
+  if ((int64_t)T * k > num_sms()) return false;
+  if (up_smem_bytes(d.fmt_up_gate, d.H) > 220 * 1024) return false;
+  if (dn_smem_bytes(d.F) > 220 * 1024) return false;
+  return true;
+}
+
+template <typename K>
+static moe_status launch_pdl(K kernel, int grid, size_t smem, cudaStream_t s,
+                             bool pdl, const DecParams& prm) {
+  MOE_CUDA_TRY(cudaFuncSetAttribute(
+      kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(DEC_THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  MOE_CUDA_TRY(cudaLaunchKernelEx(&cfg, kernel, prm));
+  return MOE_OK;
+}
+
+static DecParams make_params(const moe_layer_desc& d, const uint16_t* x,
+                             int T, int k, const int32_t* offsets,
+                             const int32_t* pair_ids, const int32_t* active,
+                             const int32_t* n_active,
+                             const int32_t* blob_index, const FfnWs& ws,
+                             float* y, const float* topk_w,
+                             const float* residual, float* out,
+                             uint16_t* out_bf16) {
+  DecParams prm;
+  prm.pool = d.pool;
+  prm.stride = d.blob_stride;
+  prm.blob_index = blob_index;
+  prm.E = d.E;
+  prm.H = d.H;
+  prm.F = d.F;
+  prm.T = T;
+  prm.k = k;
+  prm.gate_off = tensor_bytes_of(d.fmt_up_gate, d.F, d.H);
+  prm.down_off = 2 * prm.gate_off;
+  prm.x = x;
+  prm.offsets = offsets;
+  prm.pair_ids = pair_ids;
+  prm.active = active;
+  prm.n_active = n_active;
+  prm.err = ws.err;
+  prm.up_cnt = ws.up_cnt;
+  prm.dn_cnt = ws.dn_cnt;
+  prm.up_part = ws.up_part;
+  prm.bfrag = ws.bfrag;
+  prm.bscale = ws.bscale;
+  prm.y = y;
+  prm.topk_w = topk_w;
+  prm.residual = residual;
+  prm.out = out;
+  prm.out_bf16 = out_bf16;
+  return prm;
+}
+
+moe_status launch_up_decode(const moe_layer_desc& d, const uint16_t* x,
+                            int T, int k, const int32_t* offsets,
+                            const int32_t* pair_ids, const int32_t* active,
+                            const int32_t* n_active, const int32_t* blob_index,
+                            const FfnWs& ws, cudaStream_t s, bool pdl) {
+  const DecParams prm =
+      make_params(d, x, T, k, offsets, pair_ids, active, n_active, blob_index,
+                  ws, nullptr, nullptr, nullptr, nullptr, nullptr);
+  const int grid = num_sms();
+  const size_t su = up_smem_bytes(d.fmt_up_gate, d.H);
+  switch (d.fmt_up_gate) {
+    case MOE_SB3_256:
+      return launch_pdl(ffn_up_decode_kernel<MOE_SB3_256>, grid, su, s, pdl,
+                        prm);
+    case MOE_NL4_B32:
+      return launch_pdl(ffn_up_decode_kernel<MOE_NL4_B32>, grid, su, s, pdl,
+                        prm);
+    default:
+      return launch_pdl(ffn_up_decode_kernel<MOE_Q4_B32>, grid, su, s, pdl,
+                        prm);
+  }
+}
+
+moe_status launch_down_decode(const moe_layer_desc& d, int T, int k,
+                              const int32_t* offsets, const int32_t* pair_ids,
+                              const int32_t* active, const int32_t* n_active,
+                              const int32_t* blob_index, const FfnWs& ws,
+                              float* y, const float* topk_w,
+                              const float* residual, float* out,
+                              uint16_t* out_bf16, cudaStream_t s, bool pdl) {
+  const DecParams prm =
+      make_params(d, nullptr, T, k, offsets, pair_ids, active, n_active,
+                  blob_index, ws, y, topk_w, residual, out, out_bf16);
+  const int grid = num_sms();
+  const size_t sd = dn_smem_bytes(d.F);
+  if (d.fmt_down == MOE_NL4_B32)
+    return launch_pdl(ffn_down_decode_kernel<MOE_NL4_B32>, grid, sd, s, pdl,
+                      prm);
+  return launch_pdl(ffn_down_decode_kernel<MOE_Q4_B32>, grid, sd, s, pdl, prm);
+}
+
+}  // namespace moe

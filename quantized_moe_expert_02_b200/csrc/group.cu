@@ -1,0 +1,205 @@
+// Token-to-expert grouping: the (token, slot) pairs p = t*k + j sorted by
+// expert, stable in p -- the per-expert token lists that the expert GEMMs
+// of the "llama-halo-hybrid" post's MoE path consume.
+#include "moe_internal.cuh"
+
+namespace moe {
+
+constexpr int GROUP_CHUNK = 2048;   // pairs per block of the large path
+constexpr int GROUP_SMALL_MAX = 16384;
+
+// Exclusive scan of v[0..n) in place by one block of 1024 threads;
+// returns the total.  n <= 8 * 1024.
+__device__ int block_exclusive_scan(int32_t* v, int n, int32_t* tmp) {
+  const int tid = threadIdx.x, per = (n + 1023) / 1024;
+  int local = 0;
+  for (int i = 0; i < per; ++i) {
+    const int idx = tid * per + i;
+    if (idx < n) local += v[idx];
+  }
+  // warp inclusive scan
+  const int lane = tid & 31, warp = tid >> 5;
+  int x = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) tmp[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int w = tmp[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    tmp[lane] = w;  // inclusive over warps
+  }
+  __syncthreads();
+  int run = x - local + (warp ? tmp[warp - 1] : 0);
+  const int total = tmp[31];
+  __syncthreads();
+  for (int i = 0; i < per; ++i) {
+    const int idx = tid * per + i;
+    if (idx < n) {
+      const int c = v[idx];
+      v[idx] = run;
+      run += c;
+    }
+  }
+  __syncthreads();
+  return total;
+}
+
+// Whole grouping in one block (P = T*k <= GROUP_SMALL_MAX, E <= EMAX).
+__global__ void __launch_bounds__(1024)
+    group_small_kernel(const int32_t* __restrict__ idx, int P, int E,
+                       int32_t* __restrict__ offsets,
+                       int32_t* __restrict__ pair_ids,
+                       int32_t* __restrict__ active,
+                       int32_t* __restrict__ n_active, int32_t* err) {
+  __shared__ int32_t cnt[EMAX + 1];
+  __shared__ int32_t flag[EMAX + 1];
+  __shared__ int32_t tmp[32];
+  for (int e = threadIdx.x; e <= E; e += blockDim.x) { cnt[e] = 0; flag[e] = 0; }
+  __syncthreads();
+  for (int p = threadIdx.x; p < P; p += blockDim.x) {
+    const int e = idx[p];
+    if (e < 0 || e >= E) { set_err(err, MOE_ERR_DEVICE); continue; }
+    atomicAdd(&cnt[e], 1);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) flag[e] = cnt[e] > 0;
+  __syncthreads();
+  block_exclusive_scan(cnt, E + 1, tmp);   // cnt[E] (=0) becomes the total
+  const int na = block_exclusive_scan(flag, E + 1, tmp);
+  for (int e = threadIdx.x; e <= E; e += blockDim.x) {
+    offsets[e] = cnt[e];
+    if (e < E && ((e + 1 <= E ? flag[e + 1] : na) != flag[e]))
+      active[flag[e]] = e;
+  }
+  if (threadIdx.x == 0) *n_active = na;
+  __syncthreads();
+  // stable scatter by warp 0: 32 pairs per step, ranks by __match_any_sync
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    for (int base = 0; base < P; base += 32) {
+      const int p = base + lane;
+      const int e = (p < P) ? idx[p] : -1;
+      const bool ok = (p < P) && e >= 0 && e < E;
+      const unsigned m = __match_any_sync(0xffffffffu, ok ? e : -1 - lane);
+      const int rank = __popc(m & ((1u << lane) - 1u));
+      if (ok) pair_ids[cnt[e] + rank] = p;
+      __syncwarp();
+      if (ok && rank == 0) cnt[e] += __popc(m);
+      __syncwarp();
+    }
+  }
+}
+
+// Large path, step 1: per-chunk histograms hist[blk][E].
+__global__ void __launch_bounds__(256)
+    group_hist_kernel(const int32_t* __restrict__ idx, int P, int E,
+                      int32_t* __restrict__ hist, int32_t* err) {
+  __shared__ int32_t cnt[EMAX];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
+  __syncthreads();
+  const int p0 = blockIdx.x * GROUP_CHUNK;
+  for (int i = threadIdx.x; i < GROUP_CHUNK; i += blockDim.x) {
+    const int p = p0 + i;
+    if (p >= P) break;
+    const int e = idx[p];
+    if (e < 0 || e >= E) { set_err(err, MOE_ERR_DEVICE); continue; }
+    atomicAdd(&cnt[e], 1);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x)
+    hist[(int64_t)blockIdx.x * E + e] = cnt[e];
+}
+
+// Step 2 (one block): offsets, active list, per-chunk bases (in place).
+__global__ void __launch_bounds__(1024)
+    group_scan_kernel(int32_t* __restrict__ hist, int nblk, int E,
+                      int32_t* __restrict__ offsets,
+                      int32_t* __restrict__ active,
+                      int32_t* __restrict__ n_active) {
+  __shared__ int32_t tot[EMAX + 1];
+  __shared__ int32_t flag[EMAX + 1];
+  __shared__ int32_t tmp[32];
+  for (int e = threadIdx.x; e <= E; e += blockDim.x) {
+    int s = 0;
+    if (e < E)
+      for (int b = 0; b < nblk; ++b) s += hist[(int64_t)b * E + e];
+    tot[e] = s;
+    flag[e] = (e < E) && s > 0;
+  }
+  __syncthreads();
+  block_exclusive_scan(tot, E + 1, tmp);
+  const int na = block_exclusive_scan(flag, E + 1, tmp);
+  for (int e = threadIdx.x; e <= E; e += blockDim.x) {
+    offsets[e] = tot[e];
+    if (e < E && ((e + 1 <= E ? flag[e + 1] : na) != flag[e]))
+      active[flag[e]] = e;
+  }
+  if (threadIdx.x == 0) *n_active = na;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int run = tot[e];
+    for (int b = 0; b < nblk; ++b) {
+      const int c = hist[(int64_t)b * E + e];
+      hist[(int64_t)b * E + e] = run;
+      run += c;
+    }
+  }
+}
+
+// Step 3: stable scatter, one warp per chunk.
+__global__ void __launch_bounds__(32)
+    group_scatter_kernel(const int32_t* __restrict__ idx, int P, int E,
+                         const int32_t* __restrict__ base,
+                         int32_t* __restrict__ pair_ids) {
+  __shared__ int32_t cur[EMAX];
+  const int lane = threadIdx.x;
+  for (int e = lane; e < E; e += 32)
+    cur[e] = base[(int64_t)blockIdx.x * E + e];
+  __syncwarp();
+  const int p0 = blockIdx.x * GROUP_CHUNK;
+  for (int b = 0; b < GROUP_CHUNK; b += 32) {
+    const int p = p0 + b + lane;
+    const int e = (p < P) ? idx[p] : -1;
+    const bool ok = (p < P) && e >= 0 && e < E;
+    const unsigned m = __match_any_sync(0xffffffffu, ok ? e : -1 - lane);
+    const int rank = __popc(m & ((1u << lane) - 1u));
+    if (ok) pair_ids[cur[e] + rank] = p;
+    __syncwarp();
+    if (ok && rank == 0) cur[e] += __popc(m);
+    __syncwarp();
+  }
+}
+
+size_t group_ws_bytes(int T, int k, int E) {
+  const int64_t P = (int64_t)T * k;
+  if (P <= GROUP_SMALL_MAX) return 256;
+  const int64_t nblk = (P + GROUP_CHUNK - 1) / GROUP_CHUNK;
+  return (size_t)(nblk * E * 4 + 256);
+}
+
+moe_status launch_group(const int32_t* idx, int T, int k, int E,
+                        int32_t* offsets, int32_t* pair_ids, int32_t* active,
+                        int32_t* n_active, int32_t* scratch, int32_t* err,
+                        cudaStream_t s) {
+  const int P = T * k;
+  if (P <= GROUP_SMALL_MAX) {
+    group_small_kernel<<<1, 1024, 0, s>>>(idx, P, E, offsets, pair_ids,
+                                          active, n_active, err);
+    return launch_status();
+  }
+  const int nblk = (P + GROUP_CHUNK - 1) / GROUP_CHUNK;
+  group_hist_kernel<<<nblk, 256, 0, s>>>(idx, P, E, scratch, err);
+  group_scan_kernel<<<1, 1024, 0, s>>>(scratch, nblk, E, offsets, active,
+                                       n_active);
+  group_scatter_kernel<<<nblk, 32, 0, s>>>(idx, P, E, scratch, pair_ids);
+  return launch_status();
+}
+
+}  // namespace moe
