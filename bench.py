@@ -36,6 +36,7 @@ UP_BYTES = 2 * synth.BIG.up_bytes          # up + gate of one expert
 DOWN_BYTES = synth.BIG.down_bytes
 BLOB = synth.BIG.blob_bytes
 WR_BYTES = synth.BIG.E * synth.BIG.H * 2   # bf16 router of one layer
+LAUNCHES_PER_STEP = 1                      # the one-kernel decode layer
 
 
 def peaks():
@@ -202,105 +203,140 @@ def workload_config(args) -> dict:
 
 # ---------------------------------------------------------------- GPU ----
 class Layers:
-    """Resident layers: packed expert pools, router weights, inputs."""
+    """Resident layers (packed expert pools, router weights) and the
+    per-T step buffers."""
 
-    def __init__(self, L: int, T: int, n_x: int = 64):
+    def __init__(self, L: int, n_x: int = 64):
         import torch
         from synth.pools import build_pool, dev, layer_desc
         import quantized_moe_expert_02_b200 as moe
-        self.moe = moe
+        self.moe, self.torch, self.dev = moe, torch, dev
         shp = synth.BIG
-        self.L, self.T = L, T
+        self.L, self.n_x = L, n_x
         self.pools = [build_pool(shp, 0, l) for l in range(L)]
         self.descs = [layer_desc(shp, p) for p in self.pools]
         self.wr = [dev(synth.gen_router(0, l, shp.E, shp.H)) for l in range(L)]
-        self.xs = [dev(synth.gen_x(0, T, shp.H, s)) for s in range(n_x)]
-        self.ws_bytes = moe.moe_layer_workspace_bytes(T, shp.k, shp.E, shp.H,
+        self.bufs = {}
+
+    def buffers(self, T: int):
+        if T in self.bufs:
+            return self.bufs[T]
+        torch, moe, shp = self.torch, self.moe, synth.BIG
+        b = {}
+        b["xs"] = [self.dev(synth.gen_x(0, T, shp.H, s)) for s in range(self.n_x)]
+        b["ws_bytes"] = moe.moe_layer_workspace_bytes(T, shp.k, shp.E, shp.H,
                                                       shp.F)
-        self.ws = torch.zeros(self.ws_bytes, dtype=torch.uint8, device="cuda")
-        self.idx = torch.empty((T, shp.k), dtype=torch.int32, device="cuda")
-        self.w = torch.empty((T, shp.k), device="cuda")
-        self.out = torch.empty((T, shp.H), device="cuda")
-        # separate-call buffers (kernel timing pass)
-        self.ffn_ws_bytes = moe.moe_ffn_workspace_bytes(T, shp.k, shp.H, shp.F)
-        self.ffn_ws = torch.zeros(self.ffn_ws_bytes, dtype=torch.uint8,
+        b["ws"] = torch.zeros(b["ws_bytes"], dtype=torch.uint8, device="cuda")
+        b["idx"] = torch.empty((T, shp.k), dtype=torch.int32, device="cuda")
+        b["w"] = torch.empty((T, shp.k), device="cuda")
+        b["out"] = torch.empty((T, shp.H), device="cuda")
+        b["ffn_ws_bytes"] = moe.moe_ffn_workspace_bytes(T, shp.k, shp.H, shp.F)
+        b["ffn_ws"] = torch.zeros(b["ffn_ws_bytes"], dtype=torch.uint8,
                                   device="cuda")
-        self.gws_bytes = moe.moe_group_workspace_bytes(T, shp.k, shp.E)
-        self.gws = torch.zeros(self.gws_bytes, dtype=torch.uint8,
+        b["gws_bytes"] = moe.moe_group_workspace_bytes(T, shp.k, shp.E)
+        b["gws"] = torch.zeros(b["gws_bytes"], dtype=torch.uint8,
                                device="cuda")
-        self.lg = torch.empty((T, shp.E), device="cuda")
-        self.off = torch.empty(shp.E + 1, dtype=torch.int32, device="cuda")
-        self.pairs = torch.empty(T * shp.k, dtype=torch.int32, device="cuda")
-        self.act = torch.empty(shp.E, dtype=torch.int32, device="cuda")
-        self.na = torch.zeros(1, dtype=torch.int32, device="cuda")
+        b["lg"] = torch.empty((T, shp.E), device="cuda")
+        b["off"] = torch.empty(shp.E + 1, dtype=torch.int32, device="cuda")
+        b["pairs"] = torch.empty(T * shp.k, dtype=torch.int32, device="cuda")
+        b["act"] = torch.empty(shp.E, dtype=torch.int32, device="cuda")
+        b["na"] = torch.zeros(1, dtype=torch.int32, device="cuda")
+        self.bufs[T] = b
+        return b
 
-    def step(self, i: int, x=None):
-        shp = synth.BIG
+    def step(self, T: int, i: int, x=None):
+        """One decode layer through the C ABI (5 kernels)."""
+        b, shp = self.buffers(T), synth.BIG
         l = i % self.L
-        xx = self.xs[i % len(self.xs)] if x is None else x
-        self.moe.moe_layer_forward(self.descs[l], xx, self.T, shp.k,
-                                   self.wr[l], None, None, None, self.out,
-                                   None, self.idx, self.w, None, self.ws,
-                                   self.ws_bytes)
+        xx = b["xs"][i % self.n_x] if x is None else x
+        self.moe.moe_layer_forward(self.descs[l], xx, T, shp.k, self.wr[l],
+                                   None, None, None, b["out"], None, b["idx"],
+                                   b["w"], None, b["ws"], b["ws_bytes"])
 
-    def unique_experts(self, i: int) -> int:
+    def unique_experts(self, T: int, i: int) -> int:
         """Distinct experts of step i (untimed: routing only)."""
-        import torch
-        shp = synth.BIG
+        b, shp = self.buffers(T), synth.BIG
         l = i % self.L
-        self.moe.moe_route_topk(self.xs[i % len(self.xs)], self.T, shp.H,
-                                self.wr[l], shp.E, None, shp.k, self.idx,
-                                self.w, self.lg)
-        return int(torch.unique(self.idx).numel())
+        self.moe.moe_route_topk(b["xs"][i % self.n_x], T, shp.H, self.wr[l],
+                                shp.E, None, shp.k, b["idx"], b["w"], b["lg"])
+        return int(self.torch.unique(b["idx"]).numel())
 
 
-def time_steps(layers, steps, warmup, fn):
+def graph_time(steps: int, warmup: int, fn, per_graph: int) -> float:
+    """Device time (ms) of `steps` calls fn(i), replayed from CUDA graphs of
+    `per_graph` steps, after `warmup` eager steps and one graph warm-up."""
     import torch
     for i in range(warmup):
         fn(i)
     torch.cuda.synchronize()
+    G = min(per_graph, steps)
+    full, rem = divmod(steps, G)
+    graphs = []
+    for n, reps in ((G, full), (rem, 1 if rem else 0)):
+        if not reps:
+            continue
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for i in range(n):
+                fn(warmup + i)
+        graphs.append((g, reps))
+    for g, _ in graphs:
+        g.replay()
+    torch.cuda.synchronize()
     s = torch.cuda.current_stream()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(
-        enable_timing=True)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
     e0.record(s)
-    for i in range(steps):
-        fn(warmup + i)
+    for g, reps in graphs:
+        for _ in range(reps):
+            g.replay()
     e1.record(s)
     e1.synchronize()
-    return e0.elapsed_time(e1)
+    ms = e0.elapsed_time(e1)
+    del graphs
+    return ms
 
 
-def kernel_timing(lay, steps, warmup):
-    """Average device time of the up/gate and down kernels, each timed with
-    CUDA events around its own C-ABI call (route and grouping untimed)."""
+def kernel_timing(lay, T, steps, warmup):
+    """Average device time of one layer launch (the one-kernel decode
+    layer), timed with CUDA events around its C-ABI call; a spin kernel
+    keeps the GPU busy while the host enqueues, so no host latency falls
+    between the events."""
     import torch
-    moe, shp, T = lay.moe, synth.BIG, lay.T
     s = torch.cuda.current_stream()
-    t_up = t_dn = 0.0
-    u_sum = 0
+    tot = 0.0
     for i in range(warmup + steps):
-        l = i % lay.L
-        x = lay.xs[i % len(lay.xs)]
-        moe.moe_route_topk(x, T, shp.H, lay.wr[l], shp.E, None, shp.k, lay.idx,
-                           lay.w, lay.lg)
-        moe.moe_group_tokens(lay.idx, T, shp.k, shp.E, lay.off, lay.pairs,
-                             lay.act, lay.na, lay.gws, lay.gws_bytes)
-        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        torch.cuda._sleep(200000)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
         ev[0].record(s)
-        moe.moe_expert_up_q(lay.descs[l], x, T, shp.k, lay.off, lay.pairs,
-                            lay.act, lay.na, None, lay.ffn_ws,
-                            lay.ffn_ws_bytes)
+        lay.step(T, i)
         ev[1].record(s)
-        moe.moe_expert_down_q(lay.descs[l], T, shp.k, lay.off, lay.pairs,
-                              lay.act, lay.na, None, None, lay.w, None,
-                              lay.out, None, lay.ffn_ws, lay.ffn_ws_bytes)
-        ev[2].record(s)
-        ev[2].synchronize()
+        ev[1].synchronize()
         if i >= warmup:
-            t_up += ev[0].elapsed_time(ev[1])
-            t_dn += ev[1].elapsed_time(ev[2])
-            u_sum += int(lay.na.item())
-    return t_up / steps, t_dn / steps, u_sum / steps
+            tot += ev[0].elapsed_time(ev[1])
+    return tot / steps
+
+
+def decode_measure(lay, T, K, W):
+    """tokens/s, ms/step and layer GB/s of K decode steps (graph replay)."""
+    uniq = [lay.unique_experts(T, W + i) for i in range(min(K, lay.L * 4))]
+    u_avg = sum(uniq) / len(uniq)
+    ms = graph_time(K, W, lambda i: lay.step(T, i), per_graph=lay.L * 4)
+    bytes_step = WR_BYTES + u_avg * BLOB + T * 3072 * 6
+    return {"tokens_per_s": T * K / (ms / 1e3), "ms_per_step": ms / K,
+            "layer_gbs": bytes_step / (ms / K * 1e-3) / 1e9,
+            "unique_experts_per_step": u_avg}, ms
+
+
+def run_profile(args) -> None:
+    """Launches for ncu: W warm-up steps then K steps, eager (5 kernels
+    each), nothing else on the GPU after the pools are built."""
+    import torch
+    lay = Layers(args.layers)
+    for i in range(args.warmup + args.steps):
+        lay.step(args.T, i)
+    torch.cuda.synchronize()
+    print("profile run done", flush=True)
 
 
 def run_ours(args) -> None:
@@ -314,12 +350,12 @@ def run_ours(args) -> None:
         import datetime
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
-    lay = Layers(args.layers, args.T)
+    lay = Layers(args.layers)
     T, K, W = args.T, args.steps, args.warmup
-
-    # algorithmic bytes of the timed steps (routing replayed untimed)
-    uniq = [lay.unique_experts(W + i) for i in range(K)]
-    bytes_steps = sum(WR_BYTES + u * BLOB + T * 3072 * 6 for u in uniq)
+    uniq = [lay.unique_experts(T, W + i) for i in range(min(K, lay.L * 4))]
+    u_avg = sum(uniq) / len(uniq)
+    for i in range(W):
+        lay.step(T, i)
     torch.cuda.synchronize()
 
     props = torch.cuda.get_device_properties(local)
@@ -329,34 +365,35 @@ def run_ours(args) -> None:
         dist.barrier()
     torch.cuda.synchronize()
     clk.start()
-    ms = time_steps(lay, K, W, lay.step)
+    ms = graph_time(K, W, lambda i: lay.step(T, i), per_graph=lay.L * 4)
     clocks = clk.stop()
     if dist:
         t = torch.tensor([ms], device="cuda")
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms = float(t.item())
     tok_s = T * K * world / (ms / 1e3)
+    bytes_step = WR_BYTES + u_avg * BLOB + T * 3072 * 6
 
     line = None
     if rank == 0:
         hbm, tf, src = peaks()
-        # dominant kernel: up/gate + SwiGLU, timed on its own
-        kt_up, kt_dn, u_avg = kernel_timing(lay, min(K, 50), 3)
-        up_bytes = u_avg * UP_BYTES + T * 3072 * 2 + u_avg * 32 * 512
-        dn_bytes = u_avg * DOWN_BYTES + u_avg * 32 * 512 + T * 3072 * 4
-        up_gbs = up_bytes / (kt_up * 1e-3) / 1e9
-        dn_gbs = dn_bytes / (kt_dn * 1e-3) / 1e9
-        # end to end: host x in, host out back, through the C ABI
+        kt = kernel_timing(lay, T, 64, 4)
+        k_gbs = bytes_step / (kt * 1e-3) / 1e9
+        # end to end: x from pinned host memory in, the output back to
+        # pinned host memory, every step, through the C ABI
+        bufs = lay.buffers(T)
         xh = [torch.from_numpy(synth.gen_x(0, T, 3072, s).view(np.int16))
-              .pin_memory() for s in range(8)]
+              .pin_memory() for s in range(lay.L * 4)]
         xd = torch.empty((T, 3072), dtype=torch.int16, device="cuda")
-        oh = torch.empty((T, 3072), dtype=torch.float32).pin_memory()
+        oh = [torch.empty((T, 3072), dtype=torch.float32).pin_memory()
+              for _ in range(lay.L * 4)]
 
         def e2e_step(i):
             xd.copy_(xh[i % len(xh)], non_blocking=True)
-            lay.step(i, x=xd)
-            oh.copy_(lay.out, non_blocking=True)
-        ms_e2e = time_steps(lay, K, W, e2e_step)
+            lay.step(T, i, x=xd)
+            oh[i % len(oh)].copy_(bufs["out"], non_blocking=True)
+        ms_e2e = graph_time(K, W, e2e_step, per_graph=lay.L * 4)
+        t1, _ = decode_measure(lay, 1, K, W)
         line = {
             "metric": METRIC, "value": tok_s, "unit": "tokens/s",
             "n_gpus": world, "steps": K, "warmup": W,
@@ -365,21 +402,22 @@ def run_ours(args) -> None:
             "dtype": "int8 mma (s32 accumulate) + f32",
             "data": "synthetic",
             "config": workload_config(args),
-            "layer_gbs": bytes_steps / (ms / K * K * 1e-3) / 1e9,
+            "layer_gbs": bytes_step / (ms / K * 1e-3) / 1e9,
+            "layer_frac_of_hbm": bytes_step / (ms / K * 1e-3) / 1e9 / hbm,
             "roofline": {
-                "bound": "hbm", "kernel": "ffn_up_decode (up/gate + SwiGLU)",
-                "achieved": up_gbs, "peak": hbm, "unit": "GB/s",
-                "frac": up_gbs / hbm, "peak_source": src,
+                "bound": "hbm",
+                "kernel": "decode_layer_kernel (the whole layer, one launch)",
+                "achieved": k_gbs, "peak": hbm, "unit": "GB/s",
+                "frac": k_gbs / hbm, "peak_source": src,
                 "traffic": None,
-                "algorithmic_bytes_per_launch": up_bytes,
-                "avg_launch_ms": kt_up},
-            "kernels": {"ffn_up_decode_ms": kt_up, "ffn_down_decode_ms": kt_dn,
-                        "ffn_down_gbs": dn_gbs,
-                        "unique_experts_per_step": u_avg},
+                "algorithmic_bytes_per_launch": bytes_step,
+                "avg_launch_ms": kt},
+            "unique_experts_per_step": u_avg,
+            "decode_t1": t1,
             "e2e": {"value": T * K / (ms_e2e / 1e3), "unit": "tokens/s",
                     "h2d_bytes_per_step": T * 3072 * 2,
                     "d2h_bytes_per_step": T * 3072 * 4},
-            "gpu_launches": 5 * K,
+            "gpu_launches": LAUNCHES_PER_STEP * K,
             "clocks": clocks,
         }
         if not args.no_cpu_baseline and world == 1:
@@ -394,17 +432,21 @@ def run_ours(args) -> None:
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--steps", type=int, default=100000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--layers", type=int, default=16)
+    ap.add_argument("--layers", type=int, default=8)
     ap.add_argument("--T", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", action="store_true",
+                    help="eager steps only, for ncu launch lists")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
         run_reference(args)
+    elif args.profile:
+        run_profile(args)
     else:
         run_ours(args)
 

@@ -42,6 +42,17 @@ moe_status launch_down_decode(const moe_layer_desc& d, int T, int k,
                               const float* residual, float* out,
                               uint16_t* out_bf16, cudaStream_t s, bool pdl);
 
+bool decode_layer_supported(const moe_layer_desc& d, int T, int k);
+size_t decode_layer_ws_bytes(int T, int k, int H, int F);
+moe_status launch_decode_layer(const moe_layer_desc& d, const uint16_t* x,
+                               const float* r_in, int T, int k,
+                               const uint16_t* wr, const float* bias,
+                               const int32_t* blob_index,
+                               const float* residual, float* out,
+                               uint16_t* out_bf16, int32_t* topk_idx,
+                               float* topk_w, float* logits, void* ws,
+                               int32_t* err, cudaStream_t s);
+
 int num_sms() {
   static int cached[64] = {0};
   int dev = 0;
@@ -54,6 +65,30 @@ int num_sms() {
     cached[dev] = n;
   }
   return cached[dev];
+}
+
+moe_status ensure_smem(const void* kernel, size_t bytes) {
+  struct Entry { const void* fn; int dev; int bytes; };
+  static Entry table[256];
+  static int n = 0;
+  static std::mutex mu;
+  if (bytes <= 48 * 1024) return MOE_OK;
+  int dev = 0;
+  MOE_CUDA_TRY(cudaGetDevice(&dev));
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < n; ++i)
+    if (table[i].fn == kernel && table[i].dev == dev &&
+        table[i].bytes >= (int)bytes)
+      return MOE_OK;
+  MOE_CUDA_TRY(cudaFuncSetAttribute(
+      kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes));
+  for (int i = 0; i < n; ++i)
+    if (table[i].fn == kernel && table[i].dev == dev) {
+      table[i].bytes = (int)bytes;
+      return MOE_OK;
+    }
+  if (n < 256) table[n++] = {kernel, dev, (int)bytes};
+  return MOE_OK;
 }
 
 struct Carver {
@@ -108,6 +143,7 @@ FfnWs carve_ffn_ws(void* base, int T, int k, int H, int F) {
 // Layer workspace = FFN workspace, then routing and grouping buffers.
 struct LayerWs {
   FfnWs ffn;
+  void* fused;       // workspace of the one-kernel decode layer
   float* logits;
   int32_t* offsets;
   int32_t* pair_ids;
@@ -129,7 +165,10 @@ static LayerWs carve_layer_ws(void* base, int T, int k, int E, int H, int F) {
   const size_t ac = c.take((size_t)E * 4);
   const size_t na = c.take(64);
   const size_t gr = c.take(group_ws_bytes(T, k, E));
+  const size_t fu = c.take(T <= DEC_TMAX ? decode_layer_ws_bytes(T, k, H, F)
+                                         : 0);
   uint8_t* b = static_cast<uint8_t*>(base);
+  w.fused = base ? static_cast<void*>(b + fu) : nullptr;
   w.logits = base ? reinterpret_cast<float*>(b + lo) : nullptr;
   w.offsets = base ? reinterpret_cast<int32_t*>(b + of) : nullptr;
   w.pair_ids = base ? reinterpret_cast<int32_t*>(b + pi) : nullptr;
@@ -365,6 +404,10 @@ extern "C" moe_status moe_layer_forward(
   if (ws_bytes < w.bytes) return MOE_ERR_WORKSPACE;
   cudaStream_t s = (cudaStream_t)stream;
   float* logits = logits_out ? logits_out : w.logits;
+  if (decode_layer_supported(*desc, T, k))
+    return launch_decode_layer(*desc, x, nullptr, T, k, w_router, bias,
+                               blob_index, residual, out, out_bf16, topk_idx,
+                               topk_w, logits, w.fused, w.ffn.err, s);
   st = launch_route(x, T, desc->H, w_router, desc->E, bias, k, topk_idx,
                     topk_w, logits, s);
   if (st != MOE_OK) return st;

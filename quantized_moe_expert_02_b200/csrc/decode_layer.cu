@@ -1,0 +1,898 @@
+// One whole decode layer (T <= 8 tokens) in one persistent cooperative
+// kernel: router + top-k, grouping, up/gate + SwiGLU, down, combine.
+//
+// One block per SM.  Warps 0..15 compute; warp 16 is a producer that
+// streams the chosen experts' packed tiles into a ring of four shared-
+// memory slots with 1-D bulk copies (cp.async.bulk + mbarrier), first the
+// up/gate units (one per slot), then -- without waiting for the up phase to
+// finish -- the down units (four per slot), so the expert stream does not
+// stop at the phase boundaries; warp 17 publishes finished up units to the
+// other blocks.  Only the warps that use a slot wait on it and release it.
+//
+// Phases (grid barriers marked ||):
+//   P0  router logits: the E rows are split over the blocks; x staged in
+//       shared memory (or computed as bf16(rmsnorm(r)) from a residual)
+//   ||
+//   P1  every block: top-k of every token from the logits (a warp per
+//       token, one redux.sync arg-max per round), softmax weights, grouping
+//       of the T*k pairs by expert -- all in shared memory; meanwhile the
+//       other warps turn x into int8 hi/lo B fragments (per-token 2^-sigma)
+//   P2  up/gate units (expert, 16 rows of F, all of H), two groups of eight
+//       warps taking alternate units, three tiles per warp:
+//       h = silu(g) * u of each of the expert's tokens -> global,
+//       |h| max per pair -> global; each finished unit counts towards its
+//       expert's completion counter
+//   P3  down B fragments: once the (at most two) experts of this block's
+//       down units are complete (their counters, not a grid barrier), h is
+//       quantised with one scale per pair
+//   P4  down units (expert, 16 rows of H, all of F), four per slot, one per
+//       group of four warps: y of each pair -> global
+//   ||
+//   P5  combine: out[t] = sum_j w[t,j] y[t,j] (+ residual), j ascending
+#include <float.h>
+
+#include "decode_pieces.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int CW = 16;                      // compute warps
+constexpr int LAYER_THREADS = (CW + 2) * 32;
+constexpr int PRODUCER = CW;                // warp index of the producer
+constexpr int SIGNALER = CW + 1;            // publishes finished up units
+constexpr int NSLOT = 4;                    // ring slots
+constexpr int MAXP = 96;                    // max pairs (T*k) per call
+constexpr int BAR_ALL = 1;                  // named barrier: all 16 warps
+constexpr int BAR_UP = 2;                   // 2, 3: up groups
+constexpr int BAR_DN = 4;                   // 4..7: down groups
+constexpr int BAR_XF = 8;                   // warps that build x fragments
+constexpr int UPG = 2, UPW = CW / UPG;      // up: 2 groups of 8 warps
+constexpr int DNG = 4, DNW = CW / DNG;      // down: 4 groups of 4 warps
+constexpr int EMAX_FUSED = 1024;            // widest router of this kernel
+
+struct LayerParams {
+  const uint8_t* pool;
+  int64_t stride;
+  const int32_t* blob_index;
+  int E, H, F, T, k;
+  int64_t gate_off, down_off;
+  const uint16_t* x;       // bf16 [T][H] (or null: use r_in)
+  const float* r_in;       // fp32 [T][H]: x = bf16(rmsnorm(r_in))
+  const uint16_t* wr;      // bf16 [E][H]
+  const float* bias;       // fp32 [E] or null
+  int32_t* topk_idx;       // [T][k]
+  float* topk_w;           // [T][k]
+  float* logits;           // [T][E]
+  const float* residual;   // fp32 [T][H] or null (may alias out)
+  float* out;              // fp32 [T][H]
+  uint16_t* out_bf16;      // bf16 [T][H] or null
+  float* h;                // ws [T*k][F]
+  uint32_t* hmax;          // ws [T*k]
+  float* y;                // ws [T*k][H]
+  int32_t* bar;            // ws [2]: grid barrier, exit counter
+  int32_t* up_done;        // ws [MAXP]: finished up units per expert
+  int32_t* err;
+};
+
+struct Smem {  // offsets into dynamic shared memory
+  int slot_bytes, ring, frag, red, misc, total;
+};
+
+__host__ __device__ inline int dn_unit_bytes(int F) {
+  return (F / B32_TILE_COLS) * B32_TILE_BYTES;
+}
+// Reduction buffers: an up group holds [UPW][32 lanes][NT][2 rows][2]
+// floats (double-buffered when NT == 1: then one group barrier per unit
+// suffices), a down group [DNW][32][NT][2] (double-buffered).
+__host__ __device__ inline int red_up_floats(int NT) {
+  return UPW * 32 * NT * 4;
+}
+__host__ __device__ inline int red_up_bufs(int NT) { return NT == 1 ? 2 : 1; }
+__host__ __device__ inline int red_dn_floats(int NT) {
+  return DNW * 32 * NT * 2;
+}
+__host__ __device__ inline Smem smem_layout(int fmt_ug, int H, int F, int T) {
+  Smem L;
+  const int up = 2 * (H / tile_cols(fmt_ug)) * tile_bytes(fmt_ug);
+  const int dn = dn_unit_bytes(F);
+  int slot = up > dn ? up : dn;
+  slot = (slot + 127) / 128 * 128;
+  const int NT = (T + 3) / 4;
+  const int xfrag = (H / 32) * NT * 64 * 4;
+  const int hfrag = 2 * (F / 32) * NT * 64 * 4;
+  const int red_up = UPG * red_up_bufs(NT) * red_up_floats(NT) * 4;
+  const int red_dn = DNG * 2 * red_dn_floats(NT) * 4;
+  L.slot_bytes = slot;
+  L.ring = 0;
+  L.frag = NSLOT * slot;
+  L.red = L.frag + ((xfrag > hfrag ? xfrag : hfrag) + 127) / 128 * 128;
+  L.misc = L.red + (red_up > red_dn ? red_up : red_dn);
+  L.total = L.misc + 3072;
+  return L;
+}
+
+// Small shared state (at the misc offset).
+struct Misc {
+  uint64_t full[NSLOT];
+  uint64_t empty[NSLOT];
+  float xsc[DEC_TMAX];       // 2^-sigma_t (/8 for SB3)
+  int xsig[DEC_TMAX];
+  uint32_t xmax[DEC_TMAX];   // max |x| per token (float bits)
+  int32_t tk_idx[MAXP];
+  float tk_w[MAXP];
+  int32_t sorted[MAXP];      // pair ids sorted by (expert, pair)
+  int32_t active[MAXP];      // experts with pairs, ascending
+  int32_t off[MAXP + 1];     // pairs of active[u]: sorted[off[u]..off[u+1])
+  float hsc[2][8];           // 2^-sigma of each pair slot, down experts
+  int32_t up_fin[MAXP];      // up units of each expert finished here
+  int U;
+  int flag;
+};
+
+__device__ __forceinline__ int ld_acquire(const int32_t* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p)
+               : "memory");
+  return v;
+}
+__device__ __forceinline__ void fence_acq_rel() {
+  asm volatile("fence.acq_rel.gpu;" ::: "memory");
+}
+
+// Grid barrier among the compute warps of all blocks: barrier number `n`
+// (1, 2, 3) completes when the counter reaches n * gridDim.x.  Bounded:
+// gives up after 0.5 s (MOE_ERR_TIMEOUT) so the launch always ends.
+__device__ void grid_barrier(const LayerParams& p, int n) {
+  named_bar_sync(BAR_ALL, CW * 32);
+  if (threadIdx.x == 0) {
+    fence_acq_rel();
+    atomicAdd(p.bar, 1);
+    const int target = n * (int)gridDim.x;
+    if (ld_acquire(p.bar) < target) {
+      const bool gave_up =
+          *reinterpret_cast<volatile int32_t*>(p.err) == MOE_ERR_TIMEOUT;
+      const uint64_t t0 = globaltimer();
+      while (!gave_up && ld_acquire(p.bar) < target) {
+        if (globaltimer() - t0 > 500000000ull) {
+          set_err(p.err, MOE_ERR_TIMEOUT);
+          break;
+        }
+        __nanosleep(32);
+      }
+    }
+    fence_acq_rel();
+  }
+  named_bar_sync(BAR_ALL, CW * 32);
+}
+
+__device__ __forceinline__ const uint8_t* expert_base(const LayerParams& p,
+                                                      int e) {
+  if (e < 0 || e >= p.E) { set_err(p.err, MOE_ERR_DEVICE); return nullptr; }
+  const int64_t b = p.blob_index ? (int64_t)p.blob_index[e] : e;
+  if (b < 0) { set_err(p.err, MOE_ERR_DEVICE); return nullptr; }
+  return p.pool + b * p.stride;
+}
+
+// Order-preserving uint32 of a float (-0 taken as +0).
+__device__ __forceinline__ uint32_t ord_key(float f) {
+  uint32_t u = __float_as_uint(f);
+  if (u == 0x80000000u) u = 0u;
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// int8 hi/lo B fragment word of 4 values: column n of the fragment is the
+// high (n even) or low (n odd) half of v = round(value * 2^sigma).
+__device__ __forceinline__ uint32_t frag_word(const float (&v)[4], float sc,
+                                              bool low) {
+  uint32_t word = 0;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int vq = __float2int_rn(v[q] * sc);
+    const int hi = (vq + 128) >> 8, lo = vq - hi * 256;
+    word |= ((uint32_t)(low ? lo : hi) & 0xFFu) << (8 * q);
+  }
+  return word;
+}
+
+}  // namespace
+
+template <int FUG, int FDN, int NTT, int EPL>
+__global__ void __launch_bounds__(LAYER_THREADS, 1)
+    decode_layer_kernel(LayerParams p) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const Smem L = smem_layout(FUG, p.H, p.F, p.T);
+  Misc& M = *reinterpret_cast<Misc*>(smem + L.misc);
+  uint8_t* ring = smem + L.ring;
+  uint32_t* frag = reinterpret_cast<uint32_t*>(smem + L.frag);
+  float* red = reinterpret_cast<float*>(smem + L.red);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int H = p.H, F = p.F, T = p.T, k = p.k, E = p.E;
+  constexpr int NT = NTT;            // N tiles of 4 tokens: T <= 4 * NT
+  constexpr int TM = 4 * NTT;
+  const int G = gridDim.x;
+  constexpr int TCU = FUG == MOE_SB3_256 ? SB3_TILE_COLS : B32_TILE_COLS;
+  constexpr int TBU = FUG == MOE_SB3_256 ? SB3_TILE_BYTES : B32_TILE_BYTES;
+  const int nk = H / TCU;                      // up tiles per row tile
+  const int nkd = F / B32_TILE_COLS;           // down tiles per row tile
+
+  // ---------------------------------------------------------------- P0 --
+  if (tid == 0) {
+    for (int s = 0; s < NSLOT; ++s) {
+      mbar_init(&M.full[s], 1);
+      mbar_init(&M.empty[s], CW);
+    }
+    fence_mbar_init();
+  }
+  if (tid < DEC_TMAX) M.xmax[tid] = 0u;
+  for (int i = tid; i < MAXP; i += LAYER_THREADS) M.up_fin[i] = 0;
+  uint16_t* xs = reinterpret_cast<uint16_t*>(ring);   // [T][H] bf16
+  if (p.x) {
+    for (int i = tid; i < T * H / 8; i += LAYER_THREADS)
+      reinterpret_cast<uint4*>(xs)[i] = reinterpret_cast<const uint4*>(p.x)[i];
+  } else {
+    for (int t = warp; t < T; t += LAYER_THREADS / 32) {
+      const float* r = p.r_in + (int64_t)t * H;
+      float s = 0.f;
+      for (int h = lane; h < H; h += 32) s = fmaf(r[h], r[h], s);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+      const float inv = 1.0f / sqrtf(s / (float)H + 1e-6f);
+      for (int h = lane; h < H; h += 32)
+        xs[t * H + h] = f32_to_bf16_rne(r[h] * inv);
+    }
+  }
+  if (blockIdx.x == 0)
+    for (int i = tid; i < T * k; i += LAYER_THREADS) p.hmax[i] = 0u;
+  __syncthreads();
+  // router rows of this block: four warps per row, each a quarter of H;
+  // a lane issues all its loads of the row first (up to RCH 16-byte
+  // chunks), then accumulates in fp32; lane sums by a fixed butterfly and
+  // the quarters in fixed order (deterministic)
+  {
+    constexpr int RQ = 4, RCH = 4;
+    float* part = reinterpret_cast<float*>(smem + L.red);   // [rows][RQ][T]
+    const int e0 = (int)((int64_t)E * blockIdx.x / G);
+    const int e1 = (int)((int64_t)E * (blockIdx.x + 1) / G);
+    const int nrow = e1 - e0;
+    const int nch = H / 8, qch = (nch + RQ - 1) / RQ;
+    for (int base = 0; base < nrow; base += CW / RQ) {
+      const int r = base + warp / RQ, q = warp % RQ;
+      if (warp < CW && r < nrow) {
+        const uint4* row =
+            reinterpret_cast<const uint4*>(p.wr + (int64_t)(e0 + r) * H);
+        float acc[TM];
+#pragma unroll
+        for (int t = 0; t < TM; ++t) acc[t] = 0.f;
+        for (int c0 = q * qch; c0 < (q + 1) * qch && c0 < nch; c0 += 32 * RCH) {
+          uint4 w[RCH];
+#pragma unroll
+          for (int i = 0; i < RCH; ++i) {
+            const int ch = c0 + lane + 32 * i;
+            w[i] = (ch < (q + 1) * qch && ch < nch) ? __ldg(row + ch)
+                                                   : make_uint4(0, 0, 0, 0);
+          }
+#pragma unroll
+          for (int i = 0; i < RCH; ++i) {
+            const int ch = c0 + lane + 32 * i;
+            if (!(ch < (q + 1) * qch && ch < nch)) continue;
+            const uint32_t wv[4] = {w[i].x, w[i].y, w[i].z, w[i].w};
+#pragma unroll
+            for (int t = 0; t < TM; ++t) {
+              if (t < T) {
+                const uint4 xv = reinterpret_cast<const uint4*>(xs + t * H)[ch];
+                const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+                float a = acc[t];
+#pragma unroll
+                for (int qq = 0; qq < 4; ++qq) {
+                  a = fmaf(__uint_as_float(wv[qq] << 16),
+                           __uint_as_float(xw[qq] << 16), a);
+                  a = fmaf(__uint_as_float(wv[qq] & 0xFFFF0000u),
+                           __uint_as_float(xw[qq] & 0xFFFF0000u), a);
+                }
+                acc[t] = a;
+              }
+            }
+          }
+        }
+#pragma unroll
+        for (int t = 0; t < TM; ++t) {
+          float a = acc[t];
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+          if (lane == 0 && t < T) part[(r * RQ + q) * DEC_TMAX + t] = a;
+        }
+      }
+    }
+    __syncthreads();
+    for (int i = tid; i < nrow * T; i += LAYER_THREADS) {
+      const int r = i / T, t = i % T;
+      float a = 0.f;
+      for (int q = 0; q < RQ; ++q) a += part[(r * RQ + q) * DEC_TMAX + t];
+      const float b = p.bias ? p.bias[e0 + r] : 0.f;
+      p.logits[(int64_t)t * E + e0 + r] = a + b;
+    }
+  }
+  __syncthreads();
+
+  // ------------------------------------------------------------- P0|P1 --
+  if (warp < CW) grid_barrier(p, 1);
+
+  // ---------------------------------------------------------------- P1 --
+  if (warp < CW) {
+    if (warp >= T) {
+      // the warps without a top-k: per-token activation scale, then the
+      // int8 hi/lo B fragments of x
+      const int xt = tid - T * 32, xn = (CW - T) * 32;
+      float m[TM];
+#pragma unroll
+      for (int t = 0; t < TM; ++t) m[t] = 0.f;
+      const int nch = H / 8;
+      for (int i = xt; i < T * nch; i += xn) {
+        const int t = i / nch;
+        const uint4 v = reinterpret_cast<const uint4*>(xs)[i];
+        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+        float mm = 0.f;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          mm = fmaxf(mm, fabsf(__uint_as_float(w4[q] << 16)));
+          mm = fmaxf(mm, fabsf(__uint_as_float(w4[q] & 0xFFFF0000u)));
+        }
+#pragma unroll
+        for (int tt = 0; tt < TM; ++tt)
+          if (tt == t) m[tt] = fmaxf(m[tt], mm);
+      }
+#pragma unroll
+      for (int t = 0; t < TM; ++t) {
+        float a = m[t];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+          a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+        if (lane == 0 && t < T) atomicMax(&M.xmax[t], __float_as_uint(a));
+      }
+      named_bar_sync(BAR_XF, xn);
+      if (xt < T) {
+        const int sg = pow2_sigma(__uint_as_float(M.xmax[xt]));
+        M.xsig[xt] = sg;
+        M.xsc[xt] = exp2i(-sg) * (FUG == MOE_SB3_256 ? 0.125f : 1.0f);
+      }
+      named_bar_sync(BAR_XF, xn);
+      const int nent = (H / 32) * NT * 32;
+      for (int i = xt; i < nent; i += xn) {
+        const int Ln = i & 31, nt = (i >> 5) % NT, blk = i / (32 * NT);
+        const int n = Ln >> 2, cq = Ln & 3;
+        const int t = 4 * nt + (n >> 1);
+        uint2 wv = make_uint2(0u, 0u);
+        if (t < T) {
+          const float sc = exp2i(M.xsig[t]);
+          const uint16_t* xr = xs + t * H + 32 * blk + 4 * cq;
+          const uint2 a = *reinterpret_cast<const uint2*>(xr);
+          const uint2 b = *reinterpret_cast<const uint2*>(xr + 16);
+          const float va[4] = {__uint_as_float(a.x << 16),
+                               __uint_as_float(a.x & 0xFFFF0000u),
+                               __uint_as_float(a.y << 16),
+                               __uint_as_float(a.y & 0xFFFF0000u)};
+          const float vb[4] = {__uint_as_float(b.x << 16),
+                               __uint_as_float(b.x & 0xFFFF0000u),
+                               __uint_as_float(b.y << 16),
+                               __uint_as_float(b.y & 0xFFFF0000u)};
+          wv.x = frag_word(va, sc, n & 1);
+          wv.y = frag_word(vb, sc, n & 1);
+        }
+        reinterpret_cast<uint2*>(frag)[i] = wv;
+      }
+    }
+    if (warp < T) {
+      // top-k of token t: lane-local candidates in registers, one
+      // redux.sync arg-max per round, ties to the lowest expert index;
+      // the weights exp(l_j - l_0) / sum are computed by lanes j < k
+      const int t = warp;
+      constexpr int PER = EPL;
+      uint32_t key[PER];
+#pragma unroll
+      for (int q = 0; q < PER; ++q) {
+        const int e = lane + 32 * q;
+        key[q] = e < E ? ord_key(__ldcg(p.logits + (int64_t)t * E + e)) : 0u;
+      }
+      uint32_t my_key = 0u;   // lane r keeps round r's winner
+      int my_idx = 0;
+#pragma unroll 1
+      for (int r = 0; r < k; ++r) {
+        // lane-local arg-max by a balanced tree; on equal keys the left
+        // (lower index) side wins
+        uint32_t tk[PER];
+        int tq[PER];
+#pragma unroll
+        for (int q = 0; q < PER; ++q) { tk[q] = key[q]; tq[q] = q; }
+#pragma unroll
+        for (int w = 1; w < PER; w <<= 1)
+#pragma unroll
+          for (int q = 0; q + w < PER; q += 2 * w)
+            if (tk[q + w] > tk[q]) { tk[q] = tk[q + w]; tq[q] = tq[q + w]; }
+        const uint32_t bk = tk[0];
+        const int bi = lane + 32 * tq[0];
+        const uint32_t gk = __reduce_max_sync(0xffffffffu, bk);
+        const int gi = (int)__reduce_min_sync(
+            0xffffffffu, (uint32_t)(bk == gk ? bi : 0x7fffffff));
+#pragma unroll
+        for (int q = 0; q < PER; ++q)
+          if (lane + 32 * q == gi) key[q] = 0u;
+        if (lane == r) { my_key = gk; my_idx = gi; }
+      }
+      // the key is order-preserving and invertible: recover the logits
+      const float v = __uint_as_float((my_key & 0x80000000u)
+                                          ? (my_key & 0x7FFFFFFFu) : ~my_key);
+      const float v0 = __shfl_sync(0xffffffffu, v, 0);
+      const float ex = lane < k ? expf(v - v0) : 0.f;
+      // sum in index order (lane 0 first), as a serial loop would
+      float s = 0.f;
+      for (int r = 0; r < k; ++r) s += __shfl_sync(0xffffffffu, ex, r);
+      if (lane < k) {
+        const float w = ex / s;
+        M.tk_idx[t * k + lane] = my_idx;
+        M.tk_w[t * k + lane] = w;
+        if (blockIdx.x == 0) {
+          p.topk_idx[t * k + lane] = my_idx;
+          p.topk_w[t * k + lane] = w;
+        }
+      }
+    }
+    named_bar_sync(BAR_ALL, CW * 32);
+    // grouping: rank of pair q = #{r : (e_r, r) < (e_q, q)}
+    const int P = T * k;
+    if (tid < P) {
+      const int eq = M.tk_idx[tid];
+      int rank = 0;
+      for (int r = 0; r < P; ++r) {
+        const int er = M.tk_idx[r];
+        rank += (er < eq) || (er == eq && r < tid);
+      }
+      M.sorted[rank] = tid;
+      if (eq < 0 || eq >= E) set_err(p.err, MOE_ERR_DEVICE);
+    }
+    named_bar_sync(BAR_ALL, CW * 32);
+    if (warp == 0) {
+      int U = 0;
+      for (int i0 = 0; i0 < P; i0 += 32) {
+        const int i = i0 + lane;
+        bool head = false;
+        if (i < P) {
+          const int e = M.tk_idx[M.sorted[i]];
+          head = (i == 0) || (e != M.tk_idx[M.sorted[i - 1]]);
+        }
+        const unsigned b = __ballot_sync(0xffffffffu, head);
+        if (head) {
+          const int u = U + __popc(b & ((1u << lane) - 1u));
+          M.active[u] = M.tk_idx[M.sorted[i]];
+          M.off[u] = i;
+        }
+        U += __popc(b);
+      }
+      if (lane == 0) { M.U = U; M.off[U] = P; }
+    }
+  }
+  __syncthreads();   // the producer may start now
+
+  const int U = M.U;
+  const int nrt_f = F / 16, nrt_h = H / 16;
+  // up units: (u, rt) over U x F/16; down units: (u, rt) over U x H/16
+  const int nu_all = U * nrt_f, nd_all = U * nrt_h;
+  const int u0 = (int)((int64_t)nu_all * blockIdx.x / G);
+  const int u1 = (int)((int64_t)nu_all * (blockIdx.x + 1) / G);
+  const int d0 = (int)((int64_t)nd_all * blockIdx.x / G);
+  const int d1 = (int)((int64_t)nd_all * (blockIdx.x + 1) / G);
+  const int dnb = dn_unit_bytes(F);
+  int dps = L.slot_bytes / dnb;                // down units per slot
+  if (dps > DNG) dps = DNG;
+
+  // ---------------------------------------------------------- producer --
+  if (warp == PRODUCER) {
+    if (lane == 0) {
+      int i = 0;
+      auto acquire = [&](int slot_i) {
+        const int s = slot_i % NSLOT;
+        if (slot_i >= NSLOT)
+          mbar_wait(&M.empty[s], ((slot_i / NSLOT) - 1) & 1, p.err);
+        return s;
+      };
+      for (int v = u0; v < u1; ++v, ++i) {
+        const int s = acquire(i);
+        const int u = v / nrt_f, rt = v % nrt_f;
+        const uint8_t* b = expert_base(p, M.active[u]);
+        if (!b) { mbar_arrive_expect_tx(&M.full[s], 0); continue; }
+        const uint32_t nb = (uint32_t)(nk * TBU);
+        mbar_arrive_expect_tx(&M.full[s], 2 * nb);
+        uint8_t* dst = ring + s * L.slot_bytes;
+        bulk_g2s(dst, b + (int64_t)rt * nb, nb, &M.full[s]);
+        bulk_g2s(dst + nb, b + p.gate_off + (int64_t)rt * nb, nb, &M.full[s]);
+      }
+      for (int v = d0; v < d1; v += dps, ++i) {
+        const int s = acquire(i);
+        const int n = (d1 - v) < dps ? (d1 - v) : dps;
+        uint32_t tot = 0;
+        const uint8_t* src[DNG];
+        for (int j = 0; j < n; ++j) {
+          const int uu = (v + j) / nrt_h, rt = (v + j) % nrt_h;
+          const uint8_t* b = expert_base(p, M.active[uu]);
+          src[j] = b ? b + p.down_off + (int64_t)rt * dnb : nullptr;
+          if (src[j]) tot += (uint32_t)dnb;
+        }
+        mbar_arrive_expect_tx(&M.full[s], tot);
+        for (int j = 0; j < n; ++j)
+          if (src[j])
+            bulk_g2s(ring + s * L.slot_bytes + j * dnb, src[j], (uint32_t)dnb,
+                     &M.full[s]);
+      }
+    }
+    return;
+  }
+
+  // ---------------------------------------------------------- signaler --
+  // Publishes this block's finished up units to the per-expert counters
+  // (gpu-scope release), so that the compute warps never wait on a fence.
+  if (warp == SIGNALER) {
+    if (lane == 0 && u1 > u0) {
+      const int ua = u0 / nrt_f, ub = (u1 - 1) / nrt_f;
+      int pub[4] = {0, 0, 0, 0};
+      int left = u1 - u0;
+      const uint64_t t0 = globaltimer();
+      bool gave_up = false;
+      while (left > 0 && !gave_up) {
+        for (int u = ua; u <= ub && u - ua < 4; ++u) {
+          const int d = *reinterpret_cast<volatile int32_t*>(&M.up_fin[u]);
+          if (d > pub[u - ua]) {
+            fence_acq_rel();
+            atomicAdd(p.up_done + u, d - pub[u - ua]);
+            left -= d - pub[u - ua];
+            pub[u - ua] = d;
+          }
+        }
+        if (left > 0) {
+          __nanosleep(64);
+          if (globaltimer() - t0 > 500000000ull) {
+            set_err(p.err, MOE_ERR_TIMEOUT);
+            gave_up = true;
+          }
+        }
+      }
+    }
+    return;
+  }
+
+  // ------------------------------------------------------------ compute --
+  const int c = lane & 3;
+  int slot_i = 0;
+
+  // P2: up/gate + SwiGLU.  Group ug takes units v with (v-u0) % 2 == ug.
+  {
+    const int ug = warp / UPW, wg = warp % UPW;
+    const int gtid = tid - ug * UPW * 32;
+    const int nbuf = red_up_bufs(NT);
+    const int rfl = red_up_floats(NT);
+    float xs2[2];
+    xs2[0] = M.xsc[c];
+    xs2[1] = M.xsc[4 + c];
+    int mine = 0;
+    int prev_u = -1;      // expert of this group's previous unit
+    auto signal = [&](int u) {
+      // one finished unit of expert u: the group's barrier before this made
+      // the group's h / hmax writes visible to this thread; the signaler
+      // warp releases them at gpu scope
+      if (gtid == 0 && u >= 0) {
+        __threadfence_block();
+        atomicAdd(&M.up_fin[u], 1);
+      }
+    };
+    for (int v = u0; v < u1; ++v, ++slot_i) {
+      if (((v - u0) & 1) != ug) continue;     // the other group's unit
+      const int s = slot_i % NSLOT;
+      mbar_wait(&M.full[s], (slot_i / NSLOT) & 1, p.err);
+      const uint8_t* unit = ring + s * L.slot_bytes;
+      float au[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+      float ag[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+      for (int pc = wg; pc < 2 * nk; pc += UPW) {
+        const int tz = pc / nk, kt = pc % nk;
+        const uint8_t* tp = unit + pc * TBU;
+        const uint32_t* xf = frag + kt * (TCU / 32) * NT * 64;
+        if (FUG == MOE_SB3_256) {
+          if (tz == 0) piece_sb3(tp, xf, NT, xs2, au, lane, NT);
+          else piece_sb3(tp, xf, NT, xs2, ag, lane, NT);
+        } else {
+          if (tz == 0) piece_b32<FUG>(tp, xf, NT, M.xsc + c, 0, au, lane, NT);
+          else piece_b32<FUG>(tp, xf, NT, M.xsc + c, 0, ag, lane, NT);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive_n(&M.empty[s], CW / UPW);
+      float* rb = red + (ug * nbuf + (mine % nbuf)) * rfl;
+      float* rw = rb + (wg * 32 + lane) * NT * 4;
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          rw[(nt * 2 + hh) * 2 + 0] = au[nt][hh];
+          rw[(nt * 2 + hh) * 2 + 1] = ag[nt][hh];
+        }
+      named_bar_sync(BAR_UP + ug, UPW * 32);
+      if (nbuf == 2) signal(prev_u);     // epilogue of the previous unit
+      {
+        const int u = v / nrt_f, rt = v % nrt_f;
+        const int pb = M.off[u], Tu = M.off[u + 1] - pb;
+        const int slot = gtid >> 4, rho = gtid & 15;     // gtid < 256
+        float hv = 0.f;
+        int pp = -1;
+        if (slot < Tu) {
+          pp = M.sorted[pb + slot];
+          const int t = pp / k;
+          const int Ln = 4 * (rho & 7) + (t & 3), nt = t >> 2, hh = rho >> 3;
+          float su = 0.f, sg = 0.f;
+#pragma unroll
+          for (int w = 0; w < UPW; ++w) {
+            su += rb[(w * 32 + Ln) * NT * 4 + (nt * 2 + hh) * 2 + 0];
+            sg += rb[(w * 32 + Ln) * NT * 4 + (nt * 2 + hh) * 2 + 1];
+          }
+          hv = sg / (1.0f + expf(-sg)) * su;
+          p.h[(int64_t)pp * F + 16 * rt + rho] = hv;
+        }
+        float m = fabsf(hv);
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1)
+          m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if (rho == 0 && pp >= 0) atomicMax(p.hmax + pp, __float_as_uint(m));
+      }
+      if (nbuf == 1) {
+        named_bar_sync(BAR_UP + ug, UPW * 32);
+        signal(v / nrt_f);
+      } else {
+        prev_u = v / nrt_f;
+      }
+      ++mine;
+    }
+    if (nbuf == 2 && prev_u >= 0) {
+      named_bar_sync(BAR_UP + ug, UPW * 32);
+      signal(prev_u);
+    }
+  }
+
+  // P3: B fragments of h for this block's down experts (at most two),
+  // one scale per pair: 2^-sigma with sigma from max |h| of the pair
+  const int uf = d1 > d0 ? d0 / nrt_h : 0;
+  const int ul = d1 > d0 ? (d1 - 1) / nrt_h : -1;
+  if (ul - uf > 1) set_err(p.err, MOE_ERR_DEVICE);
+  const int nexp = ul - uf + 1 < 2 ? ul - uf + 1 : 2;
+  const int hwords = (F / 32) * NT * 64;      // words per expert
+  {
+    // wait until every up unit of this block's down experts is done
+    if (tid < nexp) {
+      const int32_t* cnt = p.up_done + uf + tid;
+      if (ld_acquire(cnt) < nrt_f) {
+        const bool gave_up =
+            *reinterpret_cast<volatile int32_t*>(p.err) == MOE_ERR_TIMEOUT;
+        const uint64_t t0 = globaltimer();
+        while (!gave_up && ld_acquire(cnt) < nrt_f) {
+          if (globaltimer() - t0 > 500000000ull) {
+            set_err(p.err, MOE_ERR_TIMEOUT);
+            break;
+          }
+          __nanosleep(32);
+        }
+      }
+      fence_acq_rel();
+    }
+    named_bar_sync(BAR_ALL, CW * 32);
+    if (tid < 16) {
+      const int b = tid >> 3, sl = tid & 7;
+      float sc = 0.f;
+      if (b < nexp) {
+        const int u = uf + b;
+        const int pb = M.off[u], Tu = M.off[u + 1] - pb;
+        if (sl < Tu) {
+          const int pp = M.sorted[pb + sl];
+          sc = exp2i(-pow2_sigma(__uint_as_float(__ldcg(p.hmax + pp))));
+        }
+      }
+      M.hsc[b][sl] = sc;
+    }
+    named_bar_sync(BAR_ALL, CW * 32);
+    const int nent = (F / 32) * NT * 32;      // entries per expert
+    for (int i = tid; i < nexp * nent; i += CW * 32) {
+      const int b = i / nent, j = i % nent;
+      const int Ln = j & 31, nt = (j >> 5) % NT, blk = j / (32 * NT);
+      const int n = Ln >> 2, cc = Ln & 3;
+      const int sl = 4 * nt + (n >> 1);
+      const int u = uf + b;
+      const int pb = M.off[u], Tu = M.off[u + 1] - pb;
+      uint2 wv = make_uint2(0u, 0u);
+      if (sl < Tu) {
+        const int pp = M.sorted[pb + sl];
+        const float sc = 1.0f / M.hsc[b][sl];
+        const float* hr = p.h + (int64_t)pp * F + 32 * blk + 4 * cc;
+        const float4 ha = __ldcg(reinterpret_cast<const float4*>(hr));
+        const float4 hb = __ldcg(reinterpret_cast<const float4*>(hr + 16));
+        const float va[4] = {ha.x, ha.y, ha.z, ha.w};
+        const float vb[4] = {hb.x, hb.y, hb.z, hb.w};
+        wv.x = frag_word(va, sc, n & 1);
+        wv.y = frag_word(vb, sc, n & 1);
+      }
+      reinterpret_cast<uint2*>(frag + b * hwords)[j] = wv;
+    }
+    named_bar_sync(BAR_ALL, CW * 32);
+  }
+
+  // P4: down projection.  Slot = up to DNG units; group dg takes unit dg.
+  {
+    const int dg = warp / DNW, wd = warp % DNW;
+    const int gtid = tid - dg * DNW * 32;
+    const int rfl = red_dn_floats(NT);
+    const int kt0 = wd * nkd / DNW, kt1 = (wd + 1) * nkd / DNW;
+    int it = 0;
+    for (int v = d0; v < d1; v += dps, ++slot_i) {
+      const int n = (d1 - v) < dps ? (d1 - v) : dps;
+      const bool have = dg < n;               // a unit for this group?
+      const int s = slot_i % NSLOT;
+      mbar_wait(&M.full[s], (slot_i / NSLOT) & 1, p.err);
+      const int u = (v + dg) / nrt_h, rt = (v + dg) % nrt_h;
+      const int b = u - uf;
+      float acc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+      if (have && b >= 0 && b < nexp) {
+        const uint8_t* unit = ring + s * L.slot_bytes + dg * dnb;
+        for (int kt = kt0; kt < kt1; ++kt)
+          piece_b32<FDN>(unit + kt * B32_TILE_BYTES,
+                         frag + b * hwords + (2 * kt) * NT * 64, NT,
+                         &M.hsc[b][c], 0, acc, lane, NT);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&M.empty[s]);   // all CW warps use a slot
+      if (!have) continue;
+      ++it;
+      float* rb = red + (dg * 2 + (it & 1)) * rfl;   // it counts this group's units
+      float* rw = rb + (wd * 32 + lane) * NT * 2;
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) rw[nt * 2 + hh] = acc[nt][hh];
+      named_bar_sync(BAR_DN + dg, DNW * 32);
+      {
+        const int pb = M.off[u], Tu = M.off[u + 1] - pb;
+        const int sl = gtid >> 4, rho = gtid & 15;   // gtid < 128
+        if (sl < Tu && b >= 0 && b < nexp) {
+          const int Ln = 4 * (rho & 7) + (sl & 3), nt = sl >> 2;
+          const int hh = rho >> 3;
+          float yv = 0.f;
+#pragma unroll
+          for (int w = 0; w < DNW; ++w)
+            yv += rb[(w * 32 + Ln) * NT * 2 + nt * 2 + hh];
+          const int pp = M.sorted[pb + sl];
+          p.y[(int64_t)pp * H + 16 * rt + rho] = yv;
+        }
+      }
+    }
+  }
+
+  grid_barrier(p, 2);
+
+  // P5: combine, then the exit count that re-arms the grid barrier
+  {
+    const int64_t n = (int64_t)T * H;
+    const int64_t i0 = n * blockIdx.x / G, i1 = n * (blockIdx.x + 1) / G;
+    for (int64_t i = i0 + tid; i < i1; i += CW * 32) {
+      const int t = (int)(i / H), col = (int)(i % H);
+      float a = 0.f;
+      for (int j = 0; j < k; ++j)
+        a = fmaf(M.tk_w[t * k + j], __ldcg(p.y + ((int64_t)t * k + j) * H + col),
+                 a);
+      if (p.residual) a += p.residual[i];
+      p.out[i] = a;
+      if (p.out_bf16) p.out_bf16[i] = f32_to_bf16_rne(a);
+    }
+  }
+  named_bar_sync(BAR_ALL, CW * 32);
+  if (tid == 0) {
+    fence_acq_rel();
+    M.flag = atomicAdd(p.bar + 1, 1) == G - 1;
+  }
+  named_bar_sync(BAR_ALL, CW * 32);
+  if (M.flag) {   // last block out: re-arm the counters for the next call
+    for (int i = tid; i < U; i += CW * 32) p.up_done[i] = 0;
+    if (tid == 0) {
+      p.bar[0] = 0;
+      p.bar[1] = 0;
+    }
+  }
+}
+
+// ---------------------------------------------------------------- host --
+bool decode_layer_supported(const moe_layer_desc& d, int T, int k) {
+  if (T < 1 || T > DEC_TMAX || T * k > MAXP || k > 32) return false;
+  if (d.E > EMAX_FUSED) return false;
+  if (d.fmt_down != MOE_NL4_B32 && d.fmt_down != MOE_Q4_B32) return false;
+  if (d.F % 64 || d.H % 64) return false;
+  if (T * k > num_sms()) return false;
+  const Smem L = smem_layout(d.fmt_up_gate, d.H, d.F, T);
+  if (L.total > 227 * 1024) return false;
+  if ((int64_t)T * d.H * 2 > NSLOT * L.slot_bytes) return false;
+  return (int)sizeof(Misc) <= 3072;
+}
+
+size_t decode_layer_ws_bytes(int T, int k, int H, int F) {
+  const size_t P = (size_t)T * k;
+  return 1024 + ((P * F * 4 + 255) & ~(size_t)255) +
+         ((P * 4 + 255) & ~(size_t)255) + ((P * H * 4 + 255) & ~(size_t)255);
+}
+
+moe_status launch_decode_layer(const moe_layer_desc& d, const uint16_t* x,
+                               const float* r_in, int T, int k,
+                               const uint16_t* wr, const float* bias,
+                               const int32_t* blob_index,
+                               const float* residual, float* out,
+                               uint16_t* out_bf16, int32_t* topk_idx,
+                               float* topk_w, float* logits, void* ws,
+                               int32_t* err, cudaStream_t s) {
+  LayerParams p;
+  p.pool = d.pool;
+  p.stride = d.blob_stride;
+  p.blob_index = blob_index;
+  p.E = d.E;
+  p.H = d.H;
+  p.F = d.F;
+  p.T = T;
+  p.k = k;
+  p.gate_off = tensor_bytes_of(d.fmt_up_gate, d.F, d.H);
+  p.down_off = 2 * p.gate_off;
+  p.x = x;
+  p.r_in = r_in;
+  p.wr = wr;
+  p.bias = bias;
+  p.topk_idx = topk_idx;
+  p.topk_w = topk_w;
+  p.logits = logits;
+  p.residual = residual;
+  p.out = out;
+  p.out_bf16 = out_bf16;
+  uint8_t* b = static_cast<uint8_t*>(ws);
+  const size_t P = (size_t)T * k;
+  p.bar = reinterpret_cast<int32_t*>(b);
+  p.up_done = reinterpret_cast<int32_t*>(b + 64);
+  b += 1024;
+  p.h = reinterpret_cast<float*>(b);
+  b += (P * d.F * 4 + 255) & ~(size_t)255;
+  p.hmax = reinterpret_cast<uint32_t*>(b);
+  b += (P * 4 + 255) & ~(size_t)255;
+  p.y = reinterpret_cast<float*>(b);
+  p.err = err;
+  const Smem L = smem_layout(d.fmt_up_gate, d.H, d.F, T);
+  void (*kern)(LayerParams) = nullptr;
+  const bool q4d = d.fmt_down == MOE_Q4_B32;
+  const bool two = T > 4;
+  const bool wide = d.E > 512;
+#define MOE_PICK2(FU, FD, NTT)                                               \
+  (wide ? decode_layer_kernel<FU, FD, NTT, 32>                               \
+        : decode_layer_kernel<FU, FD, NTT, 16>)
+#define MOE_PICK(FU)                                                        \
+  kern = q4d ? (two ? MOE_PICK2(FU, MOE_Q4_B32, 2)                          \
+                    : MOE_PICK2(FU, MOE_Q4_B32, 1))                         \
+             : (two ? MOE_PICK2(FU, MOE_NL4_B32, 2)                         \
+                    : MOE_PICK2(FU, MOE_NL4_B32, 1))
+  switch (d.fmt_up_gate) {
+    case MOE_SB3_256: MOE_PICK(MOE_SB3_256); break;
+    case MOE_NL4_B32: MOE_PICK(MOE_NL4_B32); break;
+    default: MOE_PICK(MOE_Q4_B32);
+  }
+#undef MOE_PICK
+#undef MOE_PICK2
+  moe_status st = ensure_smem((const void*)kern, (size_t)L.total);
+  if (st != MOE_OK) return st;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(num_sms());
+  cfg.blockDim = dim3(LAYER_THREADS);
+  cfg.dynamicSmemBytes = (size_t)L.total;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  MOE_CUDA_TRY(cudaLaunchKernelEx(&cfg, kern, p));
+  return MOE_OK;
+}
+
+}  // namespace moe

@@ -24,7 +24,7 @@
 // a group split F.  y of each pair is written per row tile; with the fused
 // combine, the block that finishes a row tile last (over all experts) sums
 // the k expert outputs of each token in j order.
-#include "moe_internal.cuh"
+#include "decode_pieces.cuh"
 
 namespace moe {
 
@@ -64,121 +64,6 @@ __device__ __forceinline__ const uint8_t* blob_of(const DecParams& p, int e) {
   const int64_t b = p.blob_index ? (int64_t)__ldcg(p.blob_index + e) : e;
   if (b < 0) { set_err(p.err, MOE_ERR_DEVICE); return nullptr; }
   return p.pool + b * p.stride;
-}
-
-// ---- tile decoders ----------------------------------------------------
-// SB3 tile (16 x 256): acc[nt][0/1] += rows g / g+8 for column token
-// (lane&3) + 4nt.  xfb = B fragments of the tile's first 32-block,
-// [blk][BF_NT][32][2] words; xs[nt] = 2^-sigma_t / 8 of the lane's token.
-__device__ __forceinline__ void piece_sb3(const uint8_t* tp,
-                                          const uint32_t* xfb, int NT,
-                                          const float (&xs)[2],
-                                          float (&acc)[2][2], int lane) {
-  const int g = lane >> 2;
-  const uint4 L0 = *reinterpret_cast<const uint4*>(tp + 16 * lane);
-  const uint4 L1 = *reinterpret_cast<const uint4*>(tp + 512 + 16 * lane);
-  const uint4 HV = *reinterpret_cast<const uint4*>(tp + 1024 + 16 * lane);
-  const uint2 SC = *reinterpret_cast<const uint2*>(tp + 1536 + 8 * g);
-  const uint32_t DD = *reinterpret_cast<const uint32_t*>(tp + 1600 + 4 * g);
-  const uint32_t lo[8] = {L0.x, L0.y, L0.z, L0.w, L1.x, L1.y, L1.z, L1.w};
-  const uint32_t hi[4] = {HV.x, HV.y, HV.z, HV.w};
-  int32_t S[2][2] = {{0, 0}, {0, 0}};
-  const int32_t zero[4] = {0, 0, 0, 0};
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const uint32_t LO = lo[j], HH = hi[j >> 1];
-    const uint32_t ha = (j & 1) ? HH : (HH << 2);
-    const uint32_t hb = (j & 1) ? (HH >> 1) : (HH << 1);
-    const uint32_t sa = (LO & 0x33333333u) | (ha & 0x44444444u);
-    const uint32_t sb = ((LO >> 2) & 0x33333333u) | (hb & 0x44444444u);
-    uint32_t a[4];
-    a[0] = prmt(SB3_TAB0, SB3_TAB1, sa);
-    a[1] = prmt(SB3_TAB0, SB3_TAB1, sa >> 16);
-    a[2] = prmt(SB3_TAB0, SB3_TAB1, sb);
-    a[3] = prmt(SB3_TAB0, SB3_TAB1, sb >> 16);
-    const int mg = (int)((SC.x >> (4 * j)) & 15u) * 2 + 1;
-    const int mg8 = (int)((SC.y >> (4 * j)) & 15u) * 2 + 1;
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-      if (nt < NT) {
-        const uint2 b = *reinterpret_cast<const uint2*>(
-            xfb + (j * BF_NT + nt) * 64 + 2 * lane);
-        int32_t d[4];
-        mma_s8(d, a, b.x, b.y, zero);
-        S[nt][0] += (d[0] * 256 + d[1]) * mg;
-        S[nt][1] += (d[2] * 256 + d[3]) * mg8;
-      }
-    }
-  }
-  const float2 dv = __half22float2(*reinterpret_cast<const __half2*>(&DD));
-#pragma unroll
-  for (int nt = 0; nt < 2; ++nt) {
-    if (nt < NT) {
-      acc[nt][0] = fmaf((float)S[nt][0], dv.x * xs[nt], acc[nt][0]);
-      acc[nt][1] = fmaf((float)S[nt][1], dv.y * xs[nt], acc[nt][1]);
-    }
-  }
-}
-
-// Q4 / NL4 tile (16 x 64, two 32-blocks).  cs = column scales of the
-// lane's columns: value for (local block bl, nt) at cs[bl*cs_stride + 4nt].
-template <int FMT>
-__device__ __forceinline__ void piece_b32(const uint8_t* tp,
-                                          const uint32_t* bfb, int NT,
-                                          const float* cs, int cs_stride,
-                                          float (&acc)[2][2], int lane) {
-  constexpr uint32_t TA0 = FMT == MOE_NL4_B32 ? NL4_TA0 : Q4_TA0;
-  constexpr uint32_t TA1 = FMT == MOE_NL4_B32 ? NL4_TA1 : Q4_TA1;
-  constexpr uint32_t TB0 = FMT == MOE_NL4_B32 ? NL4_TB0 : Q4_TB0;
-  constexpr uint32_t TB1 = FMT == MOE_NL4_B32 ? NL4_TB1 : Q4_TB1;
-  const int g = lane >> 2;
-  const uint4 W = *reinterpret_cast<const uint4*>(tp + 16 * lane);
-  const uint2 DV = *reinterpret_cast<const uint2*>(tp + 512 + 8 * g);
-  const float2 dg = __half22float2(*reinterpret_cast<const __half2*>(&DV.x));
-  const float2 dg8 = __half22float2(*reinterpret_cast<const __half2*>(&DV.y));
-  const uint32_t w[4] = {W.x, W.y, W.z, W.w};
-  const int32_t zero[4] = {0, 0, 0, 0};
-#pragma unroll
-  for (int bl = 0; bl < 2; ++bl) {
-    const uint32_t w0 = w[2 * bl], w1 = w[2 * bl + 1];
-    const uint32_t x0 = w0 ^ 0x88888888u, x1 = w1 ^ 0x88888888u;
-    uint32_t a1[4], a2[4];
-    a1[0] = prmt(TA0, TA1, w0);
-    a1[1] = prmt(TA0, TA1, w0 >> 16);
-    a1[2] = prmt(TA0, TA1, w1);
-    a1[3] = prmt(TA0, TA1, w1 >> 16);
-    a2[0] = prmt(TB0, TB1, x0);
-    a2[1] = prmt(TB0, TB1, x0 >> 16);
-    a2[2] = prmt(TB0, TB1, x1);
-    a2[3] = prmt(TB0, TB1, x1 >> 16);
-    const float d0 = bl ? dg.y : dg.x, d8 = bl ? dg8.y : dg8.x;
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-      if (nt < NT) {
-        const uint2 b = *reinterpret_cast<const uint2*>(
-            bfb + (bl * BF_NT + nt) * 64 + 2 * lane);
-        int32_t d[4];
-        mma_s8(d, a1, b.x, b.y, zero);
-        mma_s8(d, a2, b.x, b.y, d);
-        const float c = cs[bl * cs_stride + 4 * nt];
-        acc[nt][0] = fmaf((float)(d[0] * 256 + d[1]), d0 * c, acc[nt][0]);
-        acc[nt][1] = fmaf((float)(d[2] * 256 + d[3]), d8 * c, acc[nt][1]);
-      }
-    }
-  }
-}
-
-// 2^sigma with sigma chosen so that max|v| * 2^sigma < 2^14.
-__device__ __forceinline__ int pow2_sigma(float m) {
-  if (!(m > 0.f) || !isfinite(m)) return 0;
-  const int e = (int)((__float_as_uint(m) >> 23) & 255u) - 126;  // m < 2^e
-  int s = 14 - e;
-  if (s > 100) s = 100;
-  if (s < -100) s = -100;
-  return s;
-}
-__device__ __forceinline__ float exp2i(int s) {
-  return __uint_as_float((uint32_t)(127 + s) << 23);
 }
 
 // ---------------------------------------------------------------- up ---
@@ -560,8 +445,8 @@ bool ffn_decode_supported(const moe_layer_desc& d, int T, int k) {
 template <typename K>
 static moe_status launch_pdl(K kernel, int grid, size_t smem, cudaStream_t s,
                              bool pdl, const DecParams& prm) {
-  MOE_CUDA_TRY(cudaFuncSetAttribute(
-      kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  const moe_status st = ensure_smem((const void*)kernel, smem);
+  if (st != MOE_OK) return st;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(DEC_THREADS);

@@ -121,9 +121,7 @@ __global__ void __launch_bounds__(256)
 
 static moe_status set_smem(const void* fn, size_t bytes) {
   if (bytes > 200 * 1024) return MOE_ERR_SHAPE;
-  MOE_CUDA_TRY(cudaFuncSetAttribute(
-      fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes));
-  return MOE_OK;
+  return ensure_smem(fn, bytes);
 }
 
 moe_status launch_up_generic(const moe_layer_desc& d, const uint16_t* x,

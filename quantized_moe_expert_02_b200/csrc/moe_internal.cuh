@@ -97,6 +97,9 @@ __device__ inline void set_err(int32_t* err, int code) {
 }
 
 int num_sms();  // SM count of the current device (cached)
+// Raise a kernel's dynamic shared-memory limit to at least `bytes` on the
+// current device (cached per kernel and device; thread-safe).
+moe_status ensure_smem(const void* kernel, size_t bytes);
 
 // ------------------------------------------------------- workspace -------
 // Decode path limits.
@@ -172,6 +175,13 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(void* bar,
 }
 __device__ __forceinline__ void mbar_arrive(void* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+// One arrival that counts `n` times toward the barrier's expected count.
+__device__ __forceinline__ void mbar_arrive_n(void* bar, uint32_t n) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(
+                   smem_u32(bar)),
+               "r"(n)
                : "memory");
 }
 __device__ __forceinline__ bool mbar_try_wait(void* bar, uint32_t parity) {

@@ -157,11 +157,9 @@ moe_status launch_route(const uint16_t* x, int T, int H, const uint16_t* wr,
                         float* topk_w, float* logits, cudaStream_t s) {
   if (T <= DEC_TMAX) {
     const size_t smem = (size_t)T * H * 2;
-    if (smem > 48 * 1024) {
-      MOE_CUDA_TRY(cudaFuncSetAttribute(
-          route_logits_small_kernel,
-          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-    }
+    const moe_status st =
+        ensure_smem((const void*)route_logits_small_kernel, smem);
+    if (st != MOE_OK) return st;
     int grid = (E + 7) / 8;
     if (grid > num_sms()) grid = num_sms();
     route_logits_small_kernel<<<grid, 256, smem, s>>>(x, T, H, wr, E, bias,
@@ -173,10 +171,8 @@ moe_status launch_route(const uint16_t* x, int T, int H, const uint16_t* wr,
   }
   MOE_CUDA_TRY(cudaGetLastError());
   const size_t smem = (size_t)4 * E * sizeof(float);
-  if (smem > 48 * 1024) {
-    MOE_CUDA_TRY(cudaFuncSetAttribute(
-        topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-  }
+  const moe_status st = ensure_smem((const void*)topk_kernel, smem);
+  if (st != MOE_OK) return st;
   topk_kernel<<<(T + 3) / 4, 128, smem, s>>>(logits, T, E, k, topk_idx,
                                              topk_w);
   return launch_status();
