@@ -135,6 +135,29 @@ moe_status moe_group_tokens(const int32_t* topk_idx, int T, int k, int E,
                             int32_t* active, int32_t* n_active, void* ws,
                             size_t ws_bytes, void* stream);
 
+/* Allocation-free variant of moe_group_tokens (no counterpart in the
+ * source pages: it exists for callers of this library that cannot
+ * allocate device memory where they call it -- a plugin or custom operator
+ * handed only input/output pointers, code where an allocation would
+ * synchronise the device or break a capture the caller does not own,
+ * real-time loops that forbid allocation).  Same arguments and results as
+ * moe_group_tokens, but the scratch lives in a fixed array in the
+ * library's own device memory (512.25 KiB, held by every device that loads
+ * the library until the process exits) instead of a workspace.
+ *   Limits: T*k <= 262144 and E <= 1024, else MOE_ERR_SHAPE.
+ *   err  int32 [1] device error word, or NULL to use the array's own word
+ *        (cleared at each call; then bad expert ids are not reported).
+ *   The first call on each device looks up the array's device address (a
+ *   runtime symbol lookup); make that first call before any stream
+ *   capture.  Calls that overlap on the GPU (other streams, other host
+ *   threads) share the array and race: serialise them.  Nothing is
+ *   allocated or freed by this call. */
+moe_status moe_group_tokens_static(const int32_t* topk_idx, int T, int k,
+                                   int E, int32_t* expert_offsets,
+                                   int32_t* pair_ids, int32_t* active,
+                                   int32_t* n_active, int32_t* err,
+                                   void* stream);
+
 /* ------------------------------------------------------ slot cache ---- */
 
 /* Resolve one layer's chosen experts against its slot partition

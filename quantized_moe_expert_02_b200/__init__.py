@@ -54,6 +54,8 @@ _SIGS = {
     "moe_group_workspace_bytes": (c_size_t, [c_int, c_int, c_int]),
     "moe_group_tokens": (c_int, [_P, c_int, c_int, c_int, _P, _P, _P, _P,
                                  _P, c_size_t, _P]),
+    "moe_group_tokens_static": (c_int, [_P, c_int, c_int, c_int, _P, _P,
+                                        _P, _P, _P, _P]),
     "moe_slot_resolve": (c_int, [_P, c_int, c_int, c_int, _P, _P, _P, c_int,
                                  c_int, c_uint32, _P, _P, _P, _P, _P, _P]),
     "moe_ffn_workspace_bytes": (c_size_t, [c_int, c_int, c_int, c_int]),
@@ -157,6 +159,13 @@ def moe_group_tokens(topk_idx, T, k, E, expert_offsets, pair_ids, active,
     _check("moe_group_tokens", lib.moe_group_tokens(
         _ptr(topk_idx), T, k, E, _ptr(expert_offsets), _ptr(pair_ids),
         _ptr(active), _ptr(n_active), _ptr(ws), ws_bytes, _stream(stream)))
+
+
+def moe_group_tokens_static(topk_idx, T, k, E, expert_offsets, pair_ids,
+                            active, n_active, err, stream=None):
+    _check("moe_group_tokens_static", lib.moe_group_tokens_static(
+        _ptr(topk_idx), T, k, E, _ptr(expert_offsets), _ptr(pair_ids),
+        _ptr(active), _ptr(n_active), _ptr(err), _stream(stream)))
 
 
 def moe_slot_resolve(topk_idx, T, k, E, slot_table, slot_owner, last_use,

@@ -203,3 +203,73 @@ moe_status launch_group(const int32_t* idx, int T, int k, int E,
 }
 
 }  // namespace moe
+
+// ---------------------------------------------------------------------
+// Grouping without a caller workspace.  For callers that cannot allocate
+// device memory at the call site -- a plugin or custom operator that is
+// handed only its input and output pointers by a host framework, code
+// running where an allocation would synchronise the device or break a
+// capture that the caller does not own, real-time loops that forbid
+// allocation -- this variant keeps its scratch in a fixed array in the
+// library's own device memory instead of a workspace.
+#include <mutex>
+
+namespace moe {
+namespace {
+
+constexpr int STATIC_GROUP_MAX_PAIRS = 262144;   // T*k
+constexpr int STATIC_GROUP_MAX_E = 1024;
+constexpr int STATIC_GROUP_MAX_CHUNKS =
+    (STATIC_GROUP_MAX_PAIRS + GROUP_CHUNK - 1) / GROUP_CHUNK;
+// word 0: error word; from word 64: per-chunk histograms [chunk][E].
+// 512.25 KiB, held by every device that loads the library until exit.
+constexpr size_t STATIC_GROUP_WORDS =
+    64 + (size_t)STATIC_GROUP_MAX_CHUNKS * STATIC_GROUP_MAX_E;
+
+static __device__ __align__(256) int32_t g_group_scratch[STATIC_GROUP_WORDS];
+
+// Device address of the scratch array on the current device, looked up
+// once per device (the array's name is only a host-side stand-in).
+moe_status group_scratch_address(int32_t** out) {
+  static int32_t* addr[64] = {};
+  static std::mutex mu;
+  int dev = 0;
+  MOE_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return MOE_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_group_scratch);
+    if (e != cudaSuccess || !p) return MOE_ERR_CUDA;
+    addr[dev] = static_cast<int32_t*>(p);
+  }
+  *out = addr[dev];
+  return MOE_OK;
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" moe_status moe_group_tokens_static(
+    const int32_t* topk_idx, int T, int k, int E, int32_t* expert_offsets,
+    int32_t* pair_ids, int32_t* active, int32_t* n_active, int32_t* err,
+    void* stream) {
+  if (!topk_idx || !expert_offsets || !pair_ids || !active || !n_active)
+    return MOE_ERR_INVALID;
+  if (T <= 0 || k <= 0 || E <= 0) return MOE_ERR_SHAPE;
+  if ((int64_t)T * k > STATIC_GROUP_MAX_PAIRS || E > STATIC_GROUP_MAX_E)
+    return MOE_ERR_SHAPE;   // beyond the fixed scratch array
+  int32_t* base = nullptr;
+  const moe_status st = group_scratch_address(&base);
+  if (st != MOE_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  int32_t* e = err;
+  if (!e) {
+    e = base;   // the array's own error word, cleared for this call
+    MOE_CUDA_TRY(cudaMemsetAsync(e, 0, sizeof(int32_t), s));
+  }
+  return launch_group(topk_idx, T, k, E, expert_offsets, pair_ids, active,
+                      n_active, base + 64, e, s);
+}
