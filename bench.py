@@ -39,6 +39,36 @@ WR_BYTES = synth.BIG.E * synth.BIG.H * 2   # bf16 router of one layer
 LAUNCHES_PER_STEP = 1                      # the one-kernel decode layer
 
 
+KERNEL_SOURCES = ["quantized_moe_expert_02_b200/csrc/decode_layer.cu",
+                  "quantized_moe_expert_02_b200/csrc/decode_pieces.cuh",
+                  "quantized_moe_expert_02_b200/csrc/moe_internal.cuh"]
+
+
+def captured_traffic(alg_bytes_per_launch: float):
+    """DRAM traffic per launch from the committed ncu capture of the decode
+    kernel, scaled from the captured launch's algorithmic bytes to the
+    bench's average launch; None when the kernel sources changed since."""
+    import hashlib
+    prof = os.path.join(ROOT, "profiles", "decode_layer_t3.md")
+    if not os.path.exists(prof):
+        return None
+    vals = {}
+    for line in open(prof):
+        if ":" in line and not line.startswith(("#", "|", " ")):
+            k, v = line.split(":", 1)
+            vals[k.strip()] = v.strip()
+    digests = []
+    for f in KERNEL_SOURCES:
+        digests.append(hashlib.sha256(open(os.path.join(ROOT, f), "rb")
+                                      .read()).hexdigest() + "  " + f)
+    sha = hashlib.sha256(("\n".join(digests) + "\n").encode()).hexdigest()
+    if vals.get("source_sha") != sha[:16]:
+        return None
+    t = float(vals["traffic_bytes_per_launch"])
+    a = float(vals["algorithmic_bytes_of_captured_launch"])
+    return t * alg_bytes_per_launch / a
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -409,7 +439,7 @@ def run_ours(args) -> None:
                 "kernel": "decode_layer_kernel (the whole layer, one launch)",
                 "achieved": k_gbs, "peak": hbm, "unit": "GB/s",
                 "frac": k_gbs / hbm, "peak_source": src,
-                "traffic": None,
+                "traffic": captured_traffic(bytes_step),
                 "algorithmic_bytes_per_launch": bytes_step,
                 "avg_launch_ms": kt},
             "unique_experts_per_step": u_avg,

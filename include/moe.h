@@ -122,7 +122,7 @@ moe_status moe_route_topk(const uint16_t* x, int T, int H,
 size_t moe_group_workspace_bytes(int T, int k, int E);
 
 /* Token-to-expert grouping: the pairs p = t*k + j sorted by expert, stable
- * in p ("MoE GEMM" grouping of the hybrid-placement post).
+ * in p ("MoE GEMM" grouping of the "llama-halo-hybrid" post).
  *   expert_offsets int32 [E+1]: pairs of expert e are
  *                  pair_ids[expert_offsets[e] .. expert_offsets[e+1]-1]
  *   pair_ids       int32 [T*k]

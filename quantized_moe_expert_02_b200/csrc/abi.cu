@@ -210,7 +210,7 @@ static moe_status check_ffn_args(const moe_layer_desc* desc, int T, int k,
   return MOE_OK;
 }
 
-// a7: up/gate + SwiGLU (result stays in the workspace).
+// Up/gate + SwiGLU (result stays in the workspace).
 static moe_status run_up(const moe_layer_desc& d, const uint16_t* x, int T,
                          int k, const int32_t* offsets,
                          const int32_t* pair_ids, const int32_t* active,
@@ -223,7 +223,7 @@ static moe_status run_up(const moe_layer_desc& d, const uint16_t* x, int T,
                            blob_index, w.h, w.err, s);
 }
 
-// a8 (+ a9): down projection, optionally followed by the combine.
+// Down projection, optionally followed by the combine.
 static moe_status run_down(const moe_layer_desc& d, int T, int k,
                            const int32_t* offsets, const int32_t* pair_ids,
                            const int32_t* active, const int32_t* n_active,
