@@ -42,6 +42,16 @@ moe_status launch_down_decode(const moe_layer_desc& d, int T, int k,
                               const float* residual, float* out,
                               uint16_t* out_bf16, cudaStream_t s, bool pdl);
 
+bool pf_supported(const moe_layer_desc& d, int T);
+int64_t pf_max_tiles(int64_t P);
+moe_status launch_pf_up(const moe_layer_desc& d, const uint16_t* x, int T,
+                        int k, const int32_t* offsets,
+                        const int32_t* pair_ids, const int32_t* blob_index,
+                        const FfnWs& w, cudaStream_t s);
+moe_status launch_pf_down(const moe_layer_desc& d, int k,
+                          const int32_t* pair_ids, const int32_t* blob_index,
+                          const FfnWs& w, float* y, cudaStream_t s);
+
 bool decode_layer_supported(const moe_layer_desc& d, int T, int k);
 size_t decode_layer_ws_bytes(int T, int k, int H, int F);
 moe_status launch_decode_layer(const moe_layer_desc& d, const uint16_t* x,
@@ -101,7 +111,8 @@ struct Carver {
 };
 
 struct Layout {
-  size_t err, up_cnt, dn_cnt, up_part, bfrag, bscale, y_int, h, total;
+  size_t err, up_cnt, dn_cnt, up_part, bfrag, bscale, y_int, h;
+  size_t x16, xscale, tiles, n_tiles, total;
 };
 
 static Layout ffn_layout(int T, int k, int H, int F) {
@@ -118,6 +129,10 @@ static Layout ffn_layout(int T, int k, int H, int F) {
   L.bscale = c.take(dec ? P * nrt * 8 * 4 : 0);
   L.y_int = c.take(P * H * 4);
   L.h = c.take(P * F * 4);
+  L.x16 = c.take(dec ? 0 : (int64_t)T * H * 2);
+  L.xscale = c.take(dec ? 0 : (int64_t)T * 4);
+  L.tiles = c.take(dec ? 0 : pf_max_tiles(P) * 16);
+  L.n_tiles = c.take(64);
   L.total = c.off;
   return L;
 }
@@ -134,6 +149,10 @@ FfnWs carve_ffn_ws(void* base, int T, int k, int H, int F) {
   w.bscale = reinterpret_cast<float*>(b + L.bscale);
   w.y_int = reinterpret_cast<float*>(b + L.y_int);
   w.h = reinterpret_cast<float*>(b + L.h);
+  w.x16 = reinterpret_cast<__half*>(b + L.x16);
+  w.xscale = reinterpret_cast<float*>(b + L.xscale);
+  w.tiles = reinterpret_cast<int4*>(b + L.tiles);
+  w.n_tiles = reinterpret_cast<int32_t*>(b + L.n_tiles);
   w.logits = nullptr;
   w.grp = nullptr;
   w.bytes = L.total;
@@ -219,6 +238,8 @@ static moe_status run_up(const moe_layer_desc& d, const uint16_t* x, int T,
   if (ffn_decode_supported(d, T, k))
     return launch_up_decode(d, x, T, k, offsets, pair_ids, active, n_active,
                             blob_index, w, s, pdl);
+  if (pf_supported(d, T))
+    return launch_pf_up(d, x, T, k, offsets, pair_ids, blob_index, w, s);
   return launch_up_generic(d, x, T, k, offsets, pair_ids, active, n_active,
                            blob_index, w.h, w.err, s);
 }
@@ -236,8 +257,11 @@ static moe_status run_down(const moe_layer_desc& d, int T, int k,
     return launch_down_decode(d, T, k, offsets, pair_ids, active, n_active,
                               blob_index, w, y, topk_w, residual, out,
                               out_bf16, s, pdl);
-  moe_status st = launch_down_generic(d, T, k, offsets, pair_ids, active,
-                                      n_active, blob_index, w.h, y, w.err, s);
+  moe_status st =
+      pf_supported(d, T)
+          ? launch_pf_down(d, k, pair_ids, blob_index, w, y, s)
+          : launch_down_generic(d, T, k, offsets, pair_ids, active, n_active,
+                                blob_index, w.h, y, w.err, s);
   if (st != MOE_OK || !out) return st;
   return launch_combine(y, topk_w, T, k, d.H, residual, out, out_bf16, s);
 }

@@ -8,50 +8,6 @@ namespace moe {
 constexpr int GROUP_CHUNK = 2048;   // pairs per block of the large path
 constexpr int GROUP_SMALL_MAX = 16384;
 
-// Exclusive scan of v[0..n) in place by one block of 1024 threads;
-// returns the total.  n <= 8 * 1024.
-__device__ int block_exclusive_scan(int32_t* v, int n, int32_t* tmp) {
-  const int tid = threadIdx.x, per = (n + 1023) / 1024;
-  int local = 0;
-  for (int i = 0; i < per; ++i) {
-    const int idx = tid * per + i;
-    if (idx < n) local += v[idx];
-  }
-  // warp inclusive scan
-  const int lane = tid & 31, warp = tid >> 5;
-  int x = local;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += y;
-  }
-  if (lane == 31) tmp[warp] = x;
-  __syncthreads();
-  if (warp == 0) {
-    int w = tmp[lane];
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, w, o);
-      if (lane >= o) w += y;
-    }
-    tmp[lane] = w;  // inclusive over warps
-  }
-  __syncthreads();
-  int run = x - local + (warp ? tmp[warp - 1] : 0);
-  const int total = tmp[31];
-  __syncthreads();
-  for (int i = 0; i < per; ++i) {
-    const int idx = tid * per + i;
-    if (idx < n) {
-      const int c = v[idx];
-      v[idx] = run;
-      run += c;
-    }
-  }
-  __syncthreads();
-  return total;
-}
-
 // Whole grouping in one block (P = T*k <= GROUP_SMALL_MAX, E <= EMAX).
 __global__ void __launch_bounds__(1024)
     group_small_kernel(const int32_t* __restrict__ idx, int P, int E,

@@ -118,6 +118,12 @@ struct FfnWs {
   float* h;           // [T*k][F]       generic path: SwiGLU output
   float* logits;      // [T][Emax]      route scratch when no logits_out
   int32_t* grp;       // grouping scratch
+  // tensor-core path (T > DEC_TMAX); h above then holds fp16 [T*k][F] in
+  // grouped row order
+  __half* x16;        // [T][H]  activations as fp16
+  float* xscale;      // [T]     2^sigma per token
+  int4* tiles;        // unit list: {expert, first grouped row, rows, 0}
+  int32_t* n_tiles;
   size_t bytes;
 };
 
@@ -242,6 +248,50 @@ __device__ __forceinline__ uint16_t f32_to_bf16_rne(float f) {
   uint32_t u = __float_as_uint(f);
   u += 0x7FFFu + ((u >> 16) & 1u);
   return (uint16_t)(u >> 16);
+}
+
+// Exclusive scan of v[0..n) in place by one block of 1024 threads;
+// returns the total.  n <= 8 * 1024.
+__device__ inline int block_exclusive_scan(int32_t* v, int n, int32_t* tmp) {
+  const int tid = threadIdx.x, per = (n + 1023) / 1024;
+  int local = 0;
+  for (int i = 0; i < per; ++i) {
+    const int idx = tid * per + i;
+    if (idx < n) local += v[idx];
+  }
+  // warp inclusive scan
+  const int lane = tid & 31, warp = tid >> 5;
+  int x = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) tmp[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int w = tmp[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    tmp[lane] = w;  // inclusive over warps
+  }
+  __syncthreads();
+  int run = x - local + (warp ? tmp[warp - 1] : 0);
+  const int total = tmp[31];
+  __syncthreads();
+  for (int i = 0; i < per; ++i) {
+    const int idx = tid * per + i;
+    if (idx < n) {
+      const int c = v[idx];
+      v[idx] = run;
+      run += c;
+    }
+  }
+  __syncthreads();
+  return total;
 }
 
 // ---------------------------------------------------- packed decoding ----

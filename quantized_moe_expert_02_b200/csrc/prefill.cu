@@ -1,0 +1,706 @@
+// Prefill expert FFN (many tokens per expert) on the 5th-generation tensor
+// cores: grouped GEMMs over the per-expert token lists of the MoE layer of
+// the "Avalon" README (512 experts, 10 active), with the expert tensors in
+// the quant types of the Avalon GGUF model card ("Files").
+//
+// One persistent CTA per SM walks a list of units.  A unit is 128 weight
+// rows of one expert times up to 256 of that expert's token rows:
+//   up   : [u | g] = W_{up,gate}[128 rows x H] . x[tokens]^T, then
+//          h = silu(g) * u  -> fp16, grouped row order
+//   down : y = W_down[128 rows x F] . h[tokens]^T -> fp32 rows of y_pairs
+// Warp roles inside the CTA:
+//   warps 0-3   epilogue: TMEM -> registers -> global (TMEM lane quadrants)
+//   warp  4     TMEM owner; lane 0 issues tcgen05.mma and the commits
+//   warp  5     B operand: cp.async gathers of activation rows (fp16)
+//   warps 6-13  A operand: quantised tiles -> fp16 in shared memory
+// Operands are K-major fp16 with the 128-byte swizzle, accumulators fp32 in
+// tensor memory.  The A tiles hold the round-to-nearest-even fp16 value of
+// each dequantised weight (d * (2s+1) * c / 8 or d * cb[q], formed with
+// exact fp16 products and one rounding).
+#include "moe_internal.cuh"
+#include "tc_ptx.cuh"
+
+#include <type_traits>
+
+namespace moe {
+namespace {
+
+constexpr int PF_BM = 128;   // weight rows per unit (MMA M)
+constexpr int PF_BK = 64;    // K per pipeline stage (one swizzle row)
+constexpr int PF_BN = 256;   // token rows per unit at most (MMA N)
+constexpr int PF_EPI = 4;    // epilogue warps
+constexpr int PF_WMMA = 4, PF_WLOAD = 5, PF_WDQ0 = 6, PF_NDQ = 8;
+constexpr int PF_THREADS = (PF_WDQ0 + PF_NDQ) * 32;   // 448
+constexpr int PF_A_BYTES = PF_BM * PF_BK * 2;         // 16 KB
+constexpr int PF_B_BYTES = PF_BN * PF_BK * 2;         // 32 KB
+constexpr int PF_TMEM_COLS = 512;
+
+template <bool UP>
+struct PfCfg {
+  static constexpr int NA = UP ? 2 : 1;            // A tensors per unit
+  static constexpr int STAGES = UP ? 3 : 4;
+  static constexpr int STAGE_BYTES = NA * PF_A_BYTES + PF_B_BYTES;
+  static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
+  static constexpr int SMEM = BAR_OFF + 256 + 1024;   // + alignment slack
+};
+
+struct PfParams {
+  const uint8_t* pool;
+  int64_t blob_stride;
+  const int32_t* blob_index;   // [E] or null (blob e)
+  int64_t off_a0, off_a1;      // A tensors inside a blob (bytes)
+  int K;                       // contraction length
+  int rows;                    // rows of the A tensors
+  int k;                       // pairs per token
+  const int32_t* pair_ids;     // grouped order
+  const int4* tiles;           // {expert, first grouped row, rows, 0}
+  const int32_t* n_tiles;
+  const __half* bsrc;          // up: x16 [T][K]; down: h16 [P][K]
+  const float* xscale;         // up: 2^sigma per token
+  __half* h16;                 // up output [P][rows], grouped rows
+  float* y;                    // down output [P][rows], pair order
+  uint32_t tab[4];             // B32 decode tables (NL4 or Q4)
+  int32_t* err;
+};
+
+__device__ __forceinline__ uint32_t hmul2u(uint32_t a, uint32_t b) {
+  __half2 r = __hmul2(*reinterpret_cast<__half2*>(&a),
+                      *reinterpret_cast<__half2*>(&b));
+  return *reinterpret_cast<uint32_t*>(&r);
+}
+__device__ __forceinline__ uint32_t hsub2u(uint32_t a, uint32_t b) {
+  __half2 r = __hsub2(*reinterpret_cast<__half2*>(&a),
+                      *reinterpret_cast<__half2*>(&b));
+  return *reinterpret_cast<uint32_t*>(&r);
+}
+__device__ __forceinline__ uint32_t half_bcast(uint16_t h) {
+  return (uint32_t)h | ((uint32_t)h << 16);
+}
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a,
+                                             uint32_t b, uint32_t c,
+                                             uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(a),
+               "r"(b), "r"(c), "r"(d)
+               : "memory");
+}
+__device__ __forceinline__ uint32_t ldg_u32(const uint8_t* p) {
+  return __ldg(reinterpret_cast<const uint32_t*>(p));
+}
+__device__ __forceinline__ uint2 ldg_u64(const uint8_t* p) {
+  return __ldg(reinterpret_cast<const uint2*>(p));
+}
+__device__ __forceinline__ uint4 ldg_u128(const uint8_t* p) {
+  return __ldg(reinterpret_cast<const uint4*>(p));
+}
+
+// Byte offset of 16-byte chunk `chunk` of row `r` in a swizzled K-major
+// operand tile (rows of 128 bytes).
+__device__ __forceinline__ uint32_t sw128(int r, int chunk) {
+  return (uint32_t)(r * 128 + ((chunk ^ (r & 7)) << 4));
+}
+
+// ------------------------------------------------------------- SB3 ----
+// fp16 high bytes of c = 2q - 7 for q = 0..3 and 4..7 (the low bytes are 0).
+constexpr uint32_t SB3_H16_LO = 0xBCC2C5C7u;   // -1,-3,-5,-7 (bytes 3..0)
+constexpr uint32_t SB3_H16_HI = 0x4745423Cu;   //  7, 5, 3, 1
+
+struct Sb3Q {
+  uint2 lo0, lo1;     // LO[j0], LO[j0+1] of lanes L0, L0+1
+  uint32_t hi0, hi1;  // HI[j0/2] of lanes L0, L0+1
+  uint2 sc;           // sub-scale words of rows g, g+8
+  uint32_t d;         // fp16 d of rows g (low), g+8 (high)
+};
+
+// One thread's share of a 16-row SB3 tile for the 64 columns starting at
+// sub-block j0 (even): rows g and g+8, columns 8p..8p+7 of each 16-column
+// half of sub-blocks j0 and j0+1.
+__device__ __forceinline__ Sb3Q sb3_load(const uint8_t* tp, int g, int p,
+                                         int j0) {
+  const int L0 = 4 * g + 2 * p;
+  const uint8_t* seg = tp + 512 * (j0 >> 2) + 4 * (j0 & 3) + 16 * L0;
+  Sb3Q q;
+  q.lo0 = ldg_u64(seg);
+  q.lo1 = ldg_u64(seg + 16);
+  q.hi0 = ldg_u32(tp + 1024 + 16 * L0 + 4 * (j0 >> 1));
+  q.hi1 = ldg_u32(tp + 1024 + 16 * L0 + 16 + 4 * (j0 >> 1));
+  q.sc = ldg_u64(tp + 1536 + 8 * g);
+  q.d = ldg_u32(tp + 1600 + 4 * g);
+  return q;
+}
+
+// 8 codes of one lane word (nibble n = 4*rowhalf + w) -> fp16 c values as
+// two half2 words per row: out[0..1] row g (w = 0,1 | 2,3), out[2..3] row
+// g+8.  Q holds one 3-bit code per nibble (bit 3 clear).
+__device__ __forceinline__ void sb3_codes_to_h16(uint32_t Q,
+                                                 uint32_t (&o)[4]) {
+  const uint32_t S = Q << 4;
+  // selector nibbles [C, q(n), C, q(n+1)]: C = 0xC picks a zero byte
+  const uint32_t X0 = (prmt(Q, S, 0x1504u) & 0xF0F0F0F0u) | 0x0C0C0C0Cu;
+  const uint32_t X1 = (prmt(Q, S, 0x3726u) & 0xF0F0F0F0u) | 0x0C0C0C0Cu;
+  o[0] = prmt(SB3_H16_LO, SB3_H16_HI, X0);
+  o[1] = prmt(SB3_H16_LO, SB3_H16_HI, X0 >> 16);
+  o[2] = prmt(SB3_H16_LO, SB3_H16_HI, X1);
+  o[3] = prmt(SB3_H16_LO, SB3_H16_HI, X1 >> 16);
+}
+
+__device__ __forceinline__ void sb3_store(const Sb3Q& q, int g, int p,
+                                          int j0, int row0,
+                                          uint32_t a_smem) {
+  const uint32_t dg = half_bcast((uint16_t)(q.d & 0xFFFFu));
+  const uint32_t dg8 = half_bcast((uint16_t)(q.d >> 16));
+#pragma unroll
+  for (int jj = 0; jj < 2; ++jj) {
+    const int j = j0 + jj;
+    const int sg = (q.sc.x >> (4 * j)) & 15, sg8 = (q.sc.y >> (4 * j)) & 15;
+    // (2s+1)/8, exact in fp16
+    const __half tg = __float2half_rn((float)(2 * sg + 1) * 0.125f);
+    const __half tg8 = __float2half_rn((float)(2 * sg8 + 1) * 0.125f);
+    const uint32_t t2g = half_bcast(__half_as_ushort(tg));
+    const uint32_t t2g8 = half_bcast(__half_as_ushort(tg8));
+    uint32_t w[2][2][4];   // [lane][h][words]
+#pragma unroll
+    for (int l = 0; l < 2; ++l) {
+      const uint32_t lo = jj ? (l ? q.lo1.y : q.lo0.y) : (l ? q.lo1.x : q.lo0.x);
+      const uint32_t hi = (l ? q.hi1 : q.hi0) >> (2 * jj);
+      const uint32_t Q0 = (lo & 0x33333333u) | ((hi << 2) & 0x44444444u);
+      const uint32_t Q1 = ((lo >> 2) & 0x33333333u) | ((hi << 1) & 0x44444444u);
+      sb3_codes_to_h16(Q0, w[l][0]);
+      sb3_codes_to_h16(Q1, w[l][1]);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        w[l][h][0] = hmul2u(hmul2u(w[l][h][0], t2g), dg);
+        w[l][h][1] = hmul2u(hmul2u(w[l][h][1], t2g), dg);
+        w[l][h][2] = hmul2u(hmul2u(w[l][h][2], t2g8), dg8);
+        w[l][h][3] = hmul2u(hmul2u(w[l][h][3], t2g8), dg8);
+      }
+    }
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int chunk = 4 * jj + 2 * h + p;
+      st_shared_v4(a_smem + sw128(row0 + g, chunk), w[0][h][0], w[0][h][1],
+                   w[1][h][0], w[1][h][1]);
+      st_shared_v4(a_smem + sw128(row0 + g + 8, chunk), w[0][h][2],
+                   w[0][h][3], w[1][h][2], w[1][h][3]);
+    }
+  }
+}
+
+// ------------------------------------------------------------- B32 ----
+struct B32Q {
+  uint4 w0, w1;   // W[0..3] of lanes L0, L0+1
+  uint2 d;        // fp16 d: (row g, b0), (g, b1), (g+8, b0), (g+8, b1)
+};
+
+__device__ __forceinline__ B32Q b32_load(const uint8_t* tp, int g, int p) {
+  const int L0 = 4 * g + 2 * p;
+  B32Q q;
+  q.w0 = ldg_u128(tp + 16 * L0);
+  q.w1 = ldg_u128(tp + 16 * L0 + 16);
+  q.d = ldg_u64(tp + 512 + 8 * g);
+  return q;
+}
+
+// 4 codes (selector nibbles in the low 16 bits of `sel`) -> two half2
+// words of d * value(q).  A1 + A2 = value (the byte-table split of the
+// packed layout); both halves are widened to 16 bits and offset into the
+// fp16 range [1024, 2048) so one subtraction gives the exact integer.
+__device__ __forceinline__ void b32_codes(uint32_t sel, const uint32_t (&tab)[4],
+                                          uint32_t d2, uint32_t& o01,
+                                          uint32_t& o23) {
+  const uint32_t A1 = prmt(tab[0], tab[1], sel);
+  const uint32_t A2 = prmt(tab[2], tab[3], sel ^ 0x8888u);
+  // u8(A1) + A2 = 256 + value, no carry across the 16-bit halves
+  const uint32_t v01 = prmt(A1, A2, 0xC1C0u) + prmt(A2, A2, 0x8180u) +
+                       0x64006400u;
+  const uint32_t v23 = prmt(A1, A2, 0xC3C2u) + prmt(A2, A2, 0x8382u) +
+                       0x64006400u;
+  const uint32_t k1280 = 0x65006500u;   // fp16 1280
+  o01 = hmul2u(hsub2u(v01, k1280), d2);
+  o23 = hmul2u(hsub2u(v23, k1280), d2);
+}
+
+__device__ __forceinline__ void b32_store(const B32Q& q, int g, int p,
+                                          int rh, int row0,
+                                          const uint32_t (&tab)[4],
+                                          uint32_t a_smem) {
+  const uint32_t dw = rh ? q.d.y : q.d.x;
+  const uint32_t d2[2] = {half_bcast((uint16_t)(dw & 0xFFFFu)),
+                          half_bcast((uint16_t)(dw >> 16))};
+  const uint32_t W0[4] = {q.w0.x, q.w0.y, q.w0.z, q.w0.w};
+  const uint32_t W1[4] = {q.w1.x, q.w1.y, q.w1.z, q.w1.w};
+  const int r = row0 + g + 8 * rh;
+#pragma unroll
+  for (int b = 0; b < 2; ++b)
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      uint32_t a0, a1, c0, c1;
+      b32_codes(W0[2 * b + h] >> (16 * rh), tab, d2[b], a0, a1);
+      b32_codes(W1[2 * b + h] >> (16 * rh), tab, d2[b], c0, c1);
+      st_shared_v4(a_smem + sw128(r, 4 * b + 2 * h + p), a0, a1, c0, c1);
+    }
+}
+
+// --------------------------------------------------------------- kernel --
+template <bool UP, bool SB3>
+__global__ void __launch_bounds__(PF_THREADS, 1)
+    pf_gemm_kernel(const PfParams p) {
+  using C = PfCfg<UP>;
+  constexpr int NA = C::NA, S = C::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (sbase - raw);
+  uint64_t* full_a = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
+  uint64_t* full_b = full_a + S;
+  uint64_t* empty = full_b + S;
+  uint64_t* acc_full = empty + S;      // [2]
+  uint64_t* acc_empty = acc_full + 2;  // [2]
+  uint64_t* drain = acc_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full_a[s], PF_NDQ);
+      mbar_init(&full_b[s], 32);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], PF_EPI);
+    }
+    mbar_init(drain, 1);
+    fence_mbar_init();
+  }
+  if (warp == PF_WMMA) {
+    tc::tmem_alloc(tmem_slot, PF_TMEM_COLS);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+
+  const int MT = p.rows / PF_BM;   // row blocks per expert tensor
+  const int nk = p.K / PF_BK;
+  const int n_units = *p.n_tiles * MT;
+  int32_t* err = p.err;
+
+  if (warp == PF_WMMA) {
+    // ------------------------------------------------ MMA issuer ------
+    if (lane == 0) {
+      uint32_t kstep = 0;
+      int uses[2] = {0, 0};
+      int it = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x, ++it) {
+        const int4 tile = p.tiles[u / MT];
+        const int nmma = (tile.z + 15) & ~15;
+        const int ab = UP ? 0 : (it & 1);
+        if (uses[ab] > 0 &&
+            !mbar_wait(&acc_empty[ab], (uses[ab] - 1) & 1, err)) {
+          ok = false;
+          break;
+        }
+        tc::fence_after_sync();
+        const uint32_t idesc = tc::idesc_f16_f32(PF_BM, nmma);
+        const uint32_t d0 = tmem + (uint32_t)(ab * 256);
+        for (int ks = 0; ks < nk; ++ks, ++kstep) {
+          const int s = (int)(kstep % S);
+          const uint32_t par = (kstep / S) & 1;
+          if (!mbar_wait(&full_a[s], par, err) ||
+              !mbar_wait(&full_b[s], par, err)) {
+            ok = false;
+            break;
+          }
+          tc::fence_proxy_async_smem();
+          tc::fence_after_sync();
+          const uint32_t st = sbase + (uint32_t)(s * C::STAGE_BYTES);
+          const uint32_t bst = st + NA * PF_A_BYTES;
+#pragma unroll
+          for (int a = 0; a < NA; ++a)
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              tc::mma_f16(d0 + (uint32_t)(a * 256),
+                          tc::sdesc_sw128(st + a * PF_A_BYTES + 32 * kk),
+                          tc::sdesc_sw128(bst + 32 * kk), idesc,
+                          (ks | kk) != 0);
+          tc::commit(&empty[s]);
+        }
+        if (!ok) break;
+        tc::commit(&acc_full[ab]);
+        ++uses[ab];
+      }
+      // all issued MMAs complete before the allocation is released
+      tc::commit(drain);
+      mbar_wait(drain, 0, err);
+    }
+  } else if (warp == PF_WLOAD) {
+    // ------------------------------------------- B operand loader -----
+    uint32_t kstep = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
+      const int4 tile = p.tiles[u / MT];
+      const int nlen = tile.z, nmma = (nlen + 15) & ~15;
+      const __half* src[PF_BN / 32];
+      uint32_t nbytes[PF_BN / 32];
+#pragma unroll
+      for (int i = 0; i < PF_BN / 32; ++i) {
+        const int n = lane + 32 * i;
+        int64_t row = 0;
+        nbytes[i] = 0;
+        if (n < nlen) {
+          const int pr = tile.y + n;
+          row = UP ? (int64_t)(p.pair_ids[pr] / p.k) : (int64_t)pr;
+          nbytes[i] = 16;
+        }
+        src[i] = p.bsrc + row * p.K;
+      }
+      for (int ks = 0; ks < nk; ++ks, ++kstep) {
+        const int s = (int)(kstep % S);
+        const uint32_t use = kstep / S;
+        if (use > 0 && !mbar_wait(&empty[s], (use - 1) & 1, err)) {
+          ok = false;
+          break;
+        }
+        const uint32_t bst =
+            sbase + (uint32_t)(s * C::STAGE_BYTES + NA * PF_A_BYTES);
+#pragma unroll
+        for (int i = 0; i < PF_BN / 32; ++i) {
+          const int n = lane + 32 * i;
+          if (n < nmma) {
+            const __half* sp = src[i] + ks * PF_BK;
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+              tc::cp_async16(bst + sw128(n, c), sp + 8 * c, nbytes[i]);
+          }
+        }
+        tc::cp_async_arrive_noinc(&full_b[s]);
+      }
+    }
+    tc::cp_async_wait_all();
+  } else if (warp >= PF_WDQ0) {
+    // ------------------------------------------ A operand dequant -----
+    const int t = threadIdx.x - PF_WDQ0 * 32;   // 0..255
+    constexpr int ITEMS = (SB3 ? 128 : 256) * NA;
+    constexpr int IPT = (ITEMS + 255) / 256;
+    const int tcols = SB3 ? SB3_TILE_COLS : B32_TILE_COLS;
+    const int tbytes = SB3 ? SB3_TILE_BYTES : B32_TILE_BYTES;
+    const int64_t trow_stride = (int64_t)(p.K / tcols) * tbytes;  // 16 rows
+    uint32_t tab[4] = {p.tab[0], p.tab[1], p.tab[2], p.tab[3]};
+    // item geometry (fixed per thread)
+    int it_g[IPT], it_p[IPT], it_rh[IPT], it_ti[IPT], it_a[IPT];
+    bool it_on[IPT];
+#pragma unroll
+    for (int i = 0; i < IPT; ++i) {
+      const int item = t + 256 * i;
+      it_on[i] = item < ITEMS;
+      it_g[i] = item & 7;
+      it_p[i] = (item >> 3) & 1;
+      if (SB3) {
+        it_rh[i] = 0;
+        it_ti[i] = (item >> 4) & 7;
+        it_a[i] = item >> 7;
+      } else {
+        it_rh[i] = (item >> 4) & 1;
+        it_ti[i] = (item >> 5) & 7;
+        it_a[i] = item >> 8;
+      }
+    }
+    using Q = typename std::conditional<SB3, Sb3Q, B32Q>::type;
+    // prefetch position (unit, k-step) and its tile pointers
+    int pu = blockIdx.x, pks = 0;
+    const uint8_t* ptp[IPT];
+    auto set_unit = [&](int u) {
+      const int4 tile = p.tiles[u / MT];
+      const int m = u % MT;
+      const int e = tile.x;
+      int64_t bi = p.blob_index ? (int64_t)p.blob_index[e] : (int64_t)e;
+      if (bi < 0) {   // no blob: report, and read blob 0 so the unit completes
+        if (t == 0) set_err(err, MOE_ERR_DEVICE);
+        bi = 0;
+      }
+      const uint8_t* blob = p.pool + bi * p.blob_stride;
+#pragma unroll
+      for (int i = 0; i < IPT; ++i)
+        ptp[i] = blob + (it_a[i] ? p.off_a1 : p.off_a0) +
+                 (int64_t)(m * (PF_BM / 16) + it_ti[i]) * trow_stride;
+    };
+    auto fetch = [&](Q (&q)[IPT]) {
+      if (pu >= n_units) return;
+      const int kc = SB3 ? (pks >> 2) : pks;
+#pragma unroll
+      for (int i = 0; i < IPT; ++i) {
+        if (!it_on[i]) continue;
+        const uint8_t* tp = ptp[i] + (int64_t)kc * tbytes;
+        if constexpr (SB3)
+          q[i] = sb3_load(tp, it_g[i], it_p[i], 2 * (pks & 3));
+        else
+          q[i] = b32_load(tp, it_g[i], it_p[i]);
+      }
+      if (++pks == nk) {
+        pks = 0;
+        pu += gridDim.x;
+        if (pu < n_units) set_unit(pu);
+      }
+    };
+    if (pu < n_units) set_unit(pu);
+    Q q0[IPT], q1[IPT], q2[IPT];
+    fetch(q0);
+    fetch(q1);
+    uint32_t kstep = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
+      for (int ks = 0; ks < nk; ++ks, ++kstep) {
+        fetch(q2);
+        const int s = (int)(kstep % S);
+        const uint32_t use = kstep / S;
+        if (use > 0 && !mbar_wait(&empty[s], (use - 1) & 1, err)) {
+          ok = false;
+          break;
+        }
+        const uint32_t st = sbase + (uint32_t)(s * C::STAGE_BYTES);
+#pragma unroll
+        for (int i = 0; i < IPT; ++i) {
+          if (!it_on[i]) continue;
+          const uint32_t a_smem = st + it_a[i] * PF_A_BYTES;
+          if constexpr (SB3)
+            sb3_store(q0[i], it_g[i], it_p[i], 2 * (ks & 3), 16 * it_ti[i],
+                      a_smem);
+          else
+            b32_store(q0[i], it_g[i], it_p[i], it_rh[i], 16 * it_ti[i], tab,
+                      a_smem);
+        }
+        tc::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&full_a[s]);
+#pragma unroll
+        for (int i = 0; i < IPT; ++i) {
+          q0[i] = q1[i];
+          q1[i] = q2[i];
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------- epilogue -------
+    int uses[2] = {0, 0};
+    int it = 0;
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++it) {
+      const int4 tile = p.tiles[u / MT];
+      const int nlen = tile.z, row0 = tile.y;
+      const int ab = UP ? 0 : (it & 1);
+      if (!mbar_wait(&acc_full[ab], uses[ab] & 1, err)) break;
+      tc::fence_after_sync();
+      const int col = (u % MT) * PF_BM + warp * 32 + lane;  // output column
+      for (int c0 = 0; c0 < nlen; c0 += 16) {
+        const int nl = c0 + (lane & 15);
+        const bool lv = nl < nlen;
+        if constexpr (UP) {
+          float uacc[16], gacc[16];
+          tc::ld_32x32b_x16(tmem + lane_base + (uint32_t)c0, uacc);
+          tc::ld_32x32b_x16(tmem + lane_base + 256u + (uint32_t)c0, gacc);
+          tc::wait_ld();
+          const float sc_l = lv ? p.xscale[p.pair_ids[row0 + nl] / p.k] : 1.f;
+          bool bad = false;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float sc = __shfl_sync(0xffffffffu, sc_l, i);
+            if (c0 + i < nlen) {
+              const float uu = uacc[i] * sc, gg = gacc[i] * sc;
+              const float hv = gg / (1.0f + __expf(-gg)) * uu;
+              const __half hh = __float2half_rn(hv);
+              bad |= __hisinf(hh) != 0;
+              p.h16[(int64_t)(row0 + c0 + i) * p.rows + col] = hh;
+            }
+          }
+          if (bad) set_err(err, MOE_ERR_DEVICE);
+        } else {
+          float acc[16];
+          tc::ld_32x32b_x16(tmem + lane_base + (uint32_t)(ab * 256 + c0), acc);
+          tc::wait_ld();
+          const int pr_l = lv ? p.pair_ids[row0 + nl] : 0;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int pr = __shfl_sync(0xffffffffu, pr_l, i);
+            if (c0 + i < nlen) p.y[(int64_t)pr * p.rows + col] = acc[i];
+          }
+        }
+      }
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[ab]);
+      ++uses[ab];
+    }
+  }
+
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == PF_WMMA) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, PF_TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------- plan and inputs ---
+// Unit list: token tiles of <= 256 grouped rows per expert; all full tiles
+// first (expert order), then the partial tiles by descending size in
+// 16-row buckets (expert order inside a bucket).
+__global__ void __launch_bounds__(1024)
+    pf_plan_kernel(const int32_t* __restrict__ offsets, int E,
+                   int4* __restrict__ tiles, int32_t* __restrict__ n_tiles) {
+  __shared__ int32_t first[EMAX + 1];
+  __shared__ int32_t tmp[32];
+  __shared__ int32_t hist[17], base[17];
+  const int tid = threadIdx.x;
+  if (tid < 17) hist[tid] = 0;
+  for (int e = tid; e <= E; e += blockDim.x)
+    first[e] = e < E ? (offsets[e + 1] - offsets[e]) / PF_BN : 0;
+  __syncthreads();
+  const int nfull = block_exclusive_scan(first, E + 1, tmp);
+  for (int e = tid; e < E; e += blockDim.x) {
+    const int o = offsets[e], cnt = offsets[e + 1] - o;
+    const int nf = cnt / PF_BN, rem = cnt % PF_BN;
+    for (int i = 0; i < nf; ++i)
+      tiles[first[e] + i] = make_int4(e, o + i * PF_BN, PF_BN, 0);
+    if (rem) atomicAdd(&hist[(rem + 15) >> 4], 1);
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int b0 = nfull;
+    for (int b = 16; b >= 1; --b) {
+      base[b] = b0;
+      b0 += hist[b];
+    }
+    *n_tiles = b0;
+  }
+  __syncthreads();
+  if (tid < 32) {
+    for (int e0 = 0; e0 < E; e0 += 32) {
+      const int e = e0 + tid;
+      int rem = 0, o = 0;
+      if (e < E) {
+        o = offsets[e];
+        rem = (offsets[e + 1] - o) % PF_BN;
+      }
+      const int b = rem ? (rem + 15) >> 4 : 0;
+      const unsigned m = __match_any_sync(0xffffffffu, b);
+      const int rank = __popc(m & ((1u << tid) - 1u));
+      if (b) {
+        const int cnt = offsets[e + 1] - o;
+        tiles[base[b] + rank] = make_int4(e, o + cnt - rem, rem, 0);
+      }
+      __syncwarp();
+      if (b && rank == 0) base[b] += __popc(m);
+      __syncwarp();
+    }
+  }
+}
+
+// x (bf16) -> fp16 with a per-token power-of-two scale that keeps every
+// value below 2^15 (2^sigma = 1 unless max|x_t| >= 2^15).
+__global__ void __launch_bounds__(256)
+    pf_x16_kernel(const uint16_t* __restrict__ x, int H,
+                  __half* __restrict__ x16, float* __restrict__ xscale) {
+  __shared__ float red[8];
+  const int t = blockIdx.x;
+  const uint16_t* xr = x + (int64_t)t * H;
+  float m = 0.f;
+  for (int i = threadIdx.x; i < H; i += blockDim.x)
+    m = fmaxf(m, fabsf(bf16_to_f32(xr[i])));
+#pragma unroll
+  for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  m = red[0];
+  for (int w = 1; w < (int)(blockDim.x >> 5); ++w) m = fmaxf(m, red[w]);
+  int sigma = 0;
+  if (m >= 32768.f && m <= 3.0e38f) sigma = ilogbf(m) - 14;
+  const float inv = ldexpf(1.f, -sigma);
+  if (threadIdx.x == 0) xscale[t] = ldexpf(1.f, sigma);
+  __half* o = x16 + (int64_t)t * H;
+  for (int i = threadIdx.x; i < H; i += blockDim.x)
+    o[i] = __float2half_rn(bf16_to_f32(xr[i]) * inv);
+}
+
+}  // namespace
+
+// ------------------------------------------------------------ launchers --
+bool pf_supported(const moe_layer_desc& d, int T) {
+  return T > DEC_TMAX && d.F % PF_BM == 0 && d.H % PF_BM == 0 &&
+         d.H % PF_BK == 0 && d.F % PF_BK == 0;
+}
+
+int64_t pf_max_tiles(int64_t P) { return P / PF_BN + P + 1; }
+
+static void pf_tables(int fmt, uint32_t (&t)[4]) {
+  if (fmt == MOE_NL4_B32) {
+    t[0] = NL4_TA0; t[1] = NL4_TA1; t[2] = NL4_TB0; t[3] = NL4_TB1;
+  } else {
+    t[0] = Q4_TA0; t[1] = Q4_TA1; t[2] = Q4_TB0; t[3] = Q4_TB1;
+  }
+}
+
+template <bool UP, bool SB3>
+static moe_status pf_launch(const PfParams& prm, cudaStream_t s) {
+  const void* fn = reinterpret_cast<const void*>(&pf_gemm_kernel<UP, SB3>);
+  moe_status st = ensure_smem(fn, PfCfg<UP>::SMEM);
+  if (st != MOE_OK) return st;
+  pf_gemm_kernel<UP, SB3>
+      <<<num_sms(), PF_THREADS, PfCfg<UP>::SMEM, s>>>(prm);
+  return launch_status();
+}
+
+moe_status launch_pf_up(const moe_layer_desc& d, const uint16_t* x, int T,
+                        int k, const int32_t* offsets,
+                        const int32_t* pair_ids, const int32_t* blob_index,
+                        const FfnWs& w, cudaStream_t s) {
+  pf_x16_kernel<<<T, 256, 0, s>>>(x, d.H, w.x16, w.xscale);
+  pf_plan_kernel<<<1, 1024, 0, s>>>(offsets, d.E, w.tiles, w.n_tiles);
+  moe_status st = launch_status();
+  if (st != MOE_OK) return st;
+  PfParams prm{};
+  prm.pool = d.pool;
+  prm.blob_stride = d.blob_stride;
+  prm.blob_index = blob_index;
+  prm.off_a0 = 0;
+  prm.off_a1 = tensor_bytes_of(d.fmt_up_gate, d.F, d.H);
+  prm.K = d.H;
+  prm.rows = d.F;
+  prm.k = k;
+  prm.pair_ids = pair_ids;
+  prm.tiles = w.tiles;
+  prm.n_tiles = w.n_tiles;
+  prm.bsrc = w.x16;
+  prm.xscale = w.xscale;
+  prm.h16 = reinterpret_cast<__half*>(w.h);
+  prm.err = w.err;
+  pf_tables(d.fmt_up_gate, prm.tab);
+  return d.fmt_up_gate == MOE_SB3_256 ? pf_launch<true, true>(prm, s)
+                                      : pf_launch<true, false>(prm, s);
+}
+
+moe_status launch_pf_down(const moe_layer_desc& d, int k,
+                          const int32_t* pair_ids, const int32_t* blob_index,
+                          const FfnWs& w, float* y, cudaStream_t s) {
+  PfParams prm{};
+  prm.pool = d.pool;
+  prm.blob_stride = d.blob_stride;
+  prm.blob_index = blob_index;
+  prm.off_a0 = 2 * tensor_bytes_of(d.fmt_up_gate, d.F, d.H);
+  prm.off_a1 = prm.off_a0;
+  prm.K = d.F;
+  prm.rows = d.H;
+  prm.k = k;
+  prm.pair_ids = pair_ids;
+  prm.tiles = w.tiles;
+  prm.n_tiles = w.n_tiles;
+  prm.bsrc = reinterpret_cast<const __half*>(w.h);
+  prm.y = y;
+  prm.err = w.err;
+  pf_tables(d.fmt_down, prm.tab);
+  return d.fmt_down == MOE_SB3_256 ? pf_launch<false, true>(prm, s)
+                                   : pf_launch<false, false>(prm, s);
+}
+
+}  // namespace moe
