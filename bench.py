@@ -156,6 +156,28 @@ def oracle_step(layer: int, step: int, T: int, tokens, n_experts=None):
     return done
 
 
+def cpu_baseline_prefill(n_tokens: int = 4) -> dict:
+    """The oracle on a bounded sample of the prefill chunk: routing (with
+    the layer's Zipf bias) and the whole expert FFN + combine of its first
+    `n_tokens` tokens."""
+    import oracle as o
+    shp = synth.BIG
+    t0 = time.perf_counter()
+    x = o.bf16_to_f64(synth.gen_x(0, PF_T, shp.H, 0)[:n_tokens])
+    wr = o.bf16_to_f64(synth.gen_router(0, 0, shp.E, shp.H))
+    bias = synth.gen_zipf_bias(0, 0, shp.E)[0]
+    src = o.ExpertSource(shp.H, shp.F, shp.fmt_up_gate, shp.fmt_down,
+                         lambda e: synth.gen_expert_blob(shp, 0, 0, e))
+    o.moe_layer(x, wr, bias, shp.k, src)
+    dt = time.perf_counter() - t0
+    return {"value": n_tokens / dt, "unit": "tokens/s",
+            "cores": blas_threads(), "kind": "oracle",
+            "sample": (f"the first {n_tokens} tokens of the {PF_T}-token "
+                       f"prefill chunk: fp64 routing with the Zipf bias, "
+                       f"dequantisation and fp64 SwiGLU FFN of their chosen "
+                       f"experts, combine ({dt:.1f} s)")}
+
+
 def blas_threads() -> int:
     try:
         from threadpoolctl import threadpool_info
@@ -358,10 +380,139 @@ def decode_measure(lay, T, K, W):
             "unique_experts_per_step": u_avg}, ms
 
 
+# -------------------------------------------------------------- prefill ---
+PF_T = synth.WORKLOADS["prefill"].T
+
+
+def prefill_flops(T: int) -> dict:
+    shp = synth.BIG
+    P = T * shp.k
+    up = P * 4 * shp.F * shp.H
+    down = P * 2 * shp.H * shp.F
+    router = 2 * T * shp.E * shp.H
+    return {"up": up, "down": down, "router": router,
+            "total": up + down + router}
+
+
+class Prefill:
+    """One prefill chunk (9536 tokens, Zipf(1.1)-biased routing) on one
+    resident layer, through the C ABI."""
+
+    def __init__(self, pool, desc, l: int = 0, T: int = PF_T):
+        import torch
+        from synth.pools import dev
+        import quantized_moe_expert_02_b200 as moe
+        shp = synth.BIG
+        self.moe, self.torch, self.T = moe, torch, T
+        self.desc = desc
+        self.x = dev(synth.gen_x(0, T, shp.H, 0))
+        self.wr = dev(synth.gen_router(0, l, shp.E, shp.H))
+        self.bias = dev(synth.gen_zipf_bias(0, l, shp.E)[0])
+        k, E, H, F = shp.k, shp.E, shp.H, shp.F
+        self.ws_bytes = moe.moe_layer_workspace_bytes(T, k, E, H, F)
+        self.ws = torch.zeros(self.ws_bytes, dtype=torch.uint8, device="cuda")
+        self.idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
+        self.w = torch.empty((T, k), device="cuda")
+        self.lg = torch.empty((T, E), device="cuda")
+        self.out = torch.empty((T, H), device="cuda")
+        # pieces
+        self.off = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+        self.pairs = torch.empty(T * k, dtype=torch.int32, device="cuda")
+        self.act = torch.empty(E, dtype=torch.int32, device="cuda")
+        self.na = torch.zeros(1, dtype=torch.int32, device="cuda")
+        self.gws_bytes = moe.moe_group_workspace_bytes(T, k, E)
+        self.gws = torch.zeros(self.gws_bytes, dtype=torch.uint8,
+                               device="cuda")
+        self.fws_bytes = moe.moe_ffn_workspace_bytes(T, k, H, F)
+        self.fws = torch.zeros(self.fws_bytes, dtype=torch.uint8,
+                               device="cuda")
+        self.y = torch.empty((T * k, H), device="cuda")
+
+    def step(self, x=None):
+        shp = synth.BIG
+        self.moe.moe_layer_forward(self.desc, self.x if x is None else x,
+                                   self.T, shp.k, self.wr, self.bias, None,
+                                   None, self.out, None, self.idx, self.w,
+                                   self.lg, self.ws, self.ws_bytes)
+
+    def piece_fns(self):
+        moe, shp, T = self.moe, synth.BIG, self.T
+        k, E, H = shp.k, shp.E, shp.H
+        return {
+            "route": lambda: moe.moe_route_topk(self.x, T, H, self.wr, E,
+                                                self.bias, k, self.idx,
+                                                self.w, self.lg),
+            "group": lambda: moe.moe_group_tokens(self.idx, T, k, E, self.off,
+                                                  self.pairs, self.act,
+                                                  self.na, self.gws,
+                                                  self.gws_bytes),
+            "up": lambda: moe.moe_expert_up_q(self.desc, self.x, T, k,
+                                              self.off, self.pairs, self.act,
+                                              self.na, None, self.fws,
+                                              self.fws_bytes),
+            "down": lambda: moe.moe_expert_down_q(self.desc, T, k, self.off,
+                                                  self.pairs, self.act,
+                                                  self.na, None, self.y, None,
+                                                  None, None, None, self.fws,
+                                                  self.fws_bytes),
+            "combine": lambda: moe.moe_combine(self.y, self.w, T, k, H, None,
+                                               self.out, None),
+        }
+
+
+def events_time(fn, steps: int, warmup: int) -> float:
+    """Average device ms of fn() over `steps` back-to-back calls (CUDA
+    events on the launching stream, after `warmup` calls)."""
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    s = torch.cuda.current_stream()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    for _ in range(steps):
+        fn()
+    e1.record(s)
+    e1.synchronize()
+    return e0.elapsed_time(e1) / steps
+
+
+def prefill_measure(pf: "Prefill", steps: int, warmup: int) -> dict:
+    """Whole prefill layer (tokens/s, TFLOP/s) and its parts."""
+    fl = prefill_flops(pf.T)
+    ms = events_time(pf.step, steps, warmup)
+    parts = {}
+    for name, fn in pf.piece_fns().items():
+        parts[name] = events_time(fn, max(2, steps // 2), 2)
+    _, tf, _ = peaks()
+    return {
+        "workload": (f"prefill chunk, one MoE layer: {pf.T} tokens, "
+                     "Zipf(1.1)-biased routing, 512 experts top-10"),
+        "tokens_per_s": pf.T / (ms / 1e3), "ms_per_step": ms,
+        "tflops": fl["total"] / (ms * 1e-3) / 1e12,
+        "frac_of_bf16_peak": fl["total"] / (ms * 1e-3) / 1e12 / tf,
+        "parts_ms": parts,
+        "up_tflops": fl["up"] / (parts["up"] * 1e-3) / 1e12,
+        "down_tflops": fl["down"] / (parts["down"] * 1e-3) / 1e12,
+        "router_tflops": fl["router"] / (parts["route"] * 1e-3) / 1e12,
+        "flops_per_step": fl,
+    }
+
+
 def run_profile(args) -> None:
     """Launches for ncu: W warm-up steps then K steps, eager (5 kernels
     each), nothing else on the GPU after the pools are built."""
     import torch
+    if args.workload == "prefill":
+        from synth.pools import build_pool, layer_desc
+        pool = build_pool(synth.BIG, 0, 0)
+        pf = Prefill(pool, layer_desc(synth.BIG, pool))
+        for i in range(args.warmup + args.steps):
+            pf.step()
+        torch.cuda.synchronize()
+        print("profile run done", flush=True)
+        return
     lay = Layers(args.layers)
     for i in range(args.warmup + args.steps):
         lay.step(args.T, i)
@@ -450,8 +601,102 @@ def run_ours(args) -> None:
             "gpu_launches": LAUNCHES_PER_STEP * K,
             "clocks": clocks,
         }
+        if not args.no_prefill:
+            pf = Prefill(lay.pools[0], lay.descs[0])
+            line["prefill"] = prefill_measure(pf, 10, 3)
+            del pf
         if not args.no_cpu_baseline and world == 1:
             line["cpu_baseline"] = cpu_baseline(T)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    if line is not None:
+        print(json.dumps(line), flush=True)
+
+
+PF_LAUNCHES_PER_STEP = 10   # route 2, group 3, x16 + plan + up, down, combine
+
+
+def run_prefill(args) -> None:
+    """`--workload prefill`: the prefill chunk as the headline line (one
+    GPU; other ranks, if any, run the same replica)."""
+    import torch
+    from synth.pools import build_pool, layer_desc
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    pool = build_pool(synth.BIG, 0, 0)
+    pf = Prefill(pool, layer_desc(synth.BIG, pool))
+    K, W = args.steps, args.warmup
+    for _ in range(W):
+        pf.step()
+    torch.cuda.synchronize()
+    props = torch.cuda.get_device_properties(local)
+    uuid = getattr(props, "uuid", None)
+    clk = ClockSampler(f"GPU-{uuid}" if uuid else None)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clk.start()
+    ms = events_time(pf.step, K, 0) * K
+    clocks = clk.stop()
+    if dist:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    line = None
+    if rank == 0:
+        hbm, tf, src = peaks()
+        m = prefill_measure(pf, max(3, min(K, 10)), 2)
+        fl = prefill_flops(pf.T)
+        up_ms = m["parts_ms"]["up"]
+        # end to end: x in from pinned host memory, out back, every step
+        xh = torch.from_numpy(synth.gen_x(0, pf.T, 3072, 0).view(np.int16)) \
+            .pin_memory()
+        xd = torch.empty((pf.T, 3072), dtype=torch.int16, device="cuda")
+        oh = torch.empty((pf.T, 3072), dtype=torch.float32).pin_memory()
+
+        def e2e():
+            xd.copy_(xh, non_blocking=True)
+            pf.step(x=xd)
+            oh.copy_(pf.out, non_blocking=True)
+        ms_e2e = events_time(e2e, max(3, min(K, 10)), 2)
+        line = {
+            "metric": METRIC, "value": pf.T * K * world / (ms / 1e3),
+            "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W,
+            "ms_per_step": ms / K, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": "f16 tcgen05 (f32 accumulate) + f32",
+            "data": "synthetic",
+            "config": {"workload": m["workload"], "T": pf.T, "H": 3072,
+                       "F": 1024, "E": 512, "k": 10,
+                       "l2": "inputs larger than L2: 2.19 GB of experts, "
+                             "1.17 GB y_pairs per step",
+                       "parallelism": f"replicas x{world}"},
+            "tflops": fl["total"] / (ms / K * 1e-3) / 1e12,
+            "roofline": {
+                "bound": "tensor",
+                "kernel": "pf_gemm_kernel<up, SB3> (up/gate + SwiGLU)",
+                "achieved": m["up_tflops"], "peak": tf, "unit": "TFLOP/s",
+                "frac": m["up_tflops"] / tf, "peak_source": src,
+                "traffic": None,
+                "algorithmic_flops_per_launch": fl["up"],
+                "avg_launch_ms": up_ms},
+            "prefill": m,
+            "e2e": {"value": pf.T / (ms_e2e / 1e3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": pf.T * 3072 * 2,
+                    "d2h_bytes_per_step": pf.T * 3072 * 4},
+            "gpu_launches": PF_LAUNCHES_PER_STEP * K,
+            "clocks": clocks,
+        }
+        if not args.no_cpu_baseline and world == 1:
+            line["cpu_baseline"] = cpu_baseline_prefill()
     if dist:
         dist.barrier()
         dist.destroy_process_group()
@@ -470,6 +715,10 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile", action="store_true",
                     help="eager steps only, for ncu launch lists")
+    ap.add_argument("--workload", default="decode",
+                    choices=["decode", "prefill"])
+    ap.add_argument("--no-prefill", action="store_true",
+                    help="leave the prefill figures out of the decode line")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -477,6 +726,10 @@ def main():
         run_reference(args)
     elif args.profile:
         run_profile(args)
+    elif args.workload == "prefill":
+        if args.steps == 100000:
+            args.steps = 50
+        run_prefill(args)
     else:
         run_ours(args)
 

@@ -48,7 +48,7 @@ moe_status launch_pf_up(const moe_layer_desc& d, const uint16_t* x, int T,
                         int k, const int32_t* offsets,
                         const int32_t* pair_ids, const int32_t* blob_index,
                         const FfnWs& w, cudaStream_t s);
-moe_status launch_pf_down(const moe_layer_desc& d, int k,
+moe_status launch_pf_down(const moe_layer_desc& d, int T, int k,
                           const int32_t* pair_ids, const int32_t* blob_index,
                           const FfnWs& w, float* y, cudaStream_t s);
 
@@ -129,8 +129,8 @@ static Layout ffn_layout(int T, int k, int H, int F) {
   L.bscale = c.take(dec ? P * nrt * 8 * 4 : 0);
   L.y_int = c.take(P * H * 4);
   L.h = c.take(P * F * 4);
-  L.x16 = c.take(dec ? 0 : (int64_t)T * H * 2);
-  L.xscale = c.take(dec ? 0 : (int64_t)T * 4);
+  L.x16 = c.take(dec ? 0 : P * H * 2);
+  L.xscale = c.take(dec ? 0 : P * 4);
   L.tiles = c.take(dec ? 0 : pf_max_tiles(P) * 16);
   L.n_tiles = c.take(64);
   L.total = c.off;
@@ -259,7 +259,7 @@ static moe_status run_down(const moe_layer_desc& d, int T, int k,
                               out_bf16, s, pdl);
   moe_status st =
       pf_supported(d, T)
-          ? launch_pf_down(d, k, pair_ids, blob_index, w, y, s)
+          ? launch_pf_down(d, T, k, pair_ids, blob_index, w, y, s)
           : launch_down_generic(d, T, k, offsets, pair_ids, active, n_active,
                                 blob_index, w.h, y, w.err, s);
   if (st != MOE_OK || !out) return st;
@@ -344,7 +344,7 @@ extern "C" moe_status moe_expert_up_q(
     const int32_t* expert_offsets, const int32_t* pair_ids,
     const int32_t* active, const int32_t* n_active,
     const int32_t* blob_index, void* ws, size_t ws_bytes, void* stream) {
-  if (!x) return MOE_ERR_INVALID;
+  if (!x || ((uintptr_t)x & 15)) return MOE_ERR_INVALID;
   moe_status st = check_ffn_args(desc, T, k, expert_offsets, pair_ids, active,
                                  n_active, ws, ws_bytes);
   if (st != MOE_OK) return st;
@@ -376,7 +376,7 @@ extern "C" moe_status moe_expert_ffn_q(
     const int32_t* active, const int32_t* n_active,
     const int32_t* blob_index, float* y_pairs, void* ws, size_t ws_bytes,
     void* stream) {
-  if (!y_pairs || !x) return MOE_ERR_INVALID;
+  if (!y_pairs || !x || ((uintptr_t)x & 15)) return MOE_ERR_INVALID;
   moe_status st = check_ffn_args(desc, T, k, expert_offsets, pair_ids, active,
                                  n_active, ws, ws_bytes);
   if (st != MOE_OK) return st;
@@ -397,7 +397,7 @@ extern "C" moe_status moe_expert_ffn_combine_q(
     const int32_t* blob_index, const float* topk_w, const float* residual,
     float* out, uint16_t* out_bf16, void* ws, size_t ws_bytes,
     void* stream) {
-  if (!out || !topk_w || !x) return MOE_ERR_INVALID;
+  if (!out || !topk_w || !x || ((uintptr_t)x & 15)) return MOE_ERR_INVALID;
   moe_status st = check_ffn_args(desc, T, k, expert_offsets, pair_ids, active,
                                  n_active, ws, ws_bytes);
   if (st != MOE_OK) return st;

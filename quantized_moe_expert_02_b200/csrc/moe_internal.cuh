@@ -120,8 +120,8 @@ struct FfnWs {
   int32_t* grp;       // grouping scratch
   // tensor-core path (T > DEC_TMAX); h above then holds fp16 [T*k][F] in
   // grouped row order
-  __half* x16;        // [T][H]  activations as fp16
-  float* xscale;      // [T]     2^sigma per token
+  __half* x16;        // [T*k][H] activations as fp16, grouped row order
+  float* xscale;      // [T*k]    2^sigma per grouped row
   int4* tiles;        // unit list: {expert, first grouped row, rows, 0}
   int32_t* n_tiles;
   size_t bytes;

@@ -11,7 +11,9 @@
 // Warp roles inside the CTA:
 //   warps 0-3   epilogue: TMEM -> registers -> global (TMEM lane quadrants)
 //   warp  4     TMEM owner; lane 0 issues tcgen05.mma and the commits
-//   warp  5     B operand: cp.async gathers of activation rows (fp16)
+//   warp  5     B operand: TMA copies of 16-row boxes of activations in
+//               grouped row order (up: x gathered to fp16 by a pre-pass;
+//               down: h as the up/gate epilogue wrote it)
 //   warps 6-13  A operand: quantised tiles -> fp16 in shared memory
 // Operands are K-major fp16 with the 128-byte swizzle, accumulators fp32 in
 // tensor memory.  The A tiles hold the round-to-nearest-even fp16 value of
@@ -20,7 +22,10 @@
 #include "moe_internal.cuh"
 #include "tc_ptx.cuh"
 
-#include <type_traits>
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
 
 namespace moe {
 namespace {
@@ -41,7 +46,9 @@ struct PfCfg {
   static constexpr int STAGES = UP ? 3 : 4;
   static constexpr int STAGE_BYTES = NA * PF_A_BYTES + PF_B_BYTES;
   static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
-  static constexpr int SMEM = BAR_OFF + 256 + 1024;   // + alignment slack
+  static constexpr int META_OFF = BAR_OFF + 256;   // epilogue row metadata
+  static constexpr int META_BYTES = PF_EPI * PF_BN * 4;
+  static constexpr int SMEM = META_OFF + META_BYTES + 1024;   // + alignment
 };
 
 struct PfParams {
@@ -55,8 +62,7 @@ struct PfParams {
   const int32_t* pair_ids;     // grouped order
   const int4* tiles;           // {expert, first grouped row, rows, 0}
   const int32_t* n_tiles;
-  const __half* bsrc;          // up: x16 [T][K]; down: h16 [P][K]
-  const float* xscale;         // up: 2^sigma per token
+  const float* xscale;         // up: 2^sigma per grouped row
   __half* h16;                 // up output [P][rows], grouped rows
   float* y;                    // down output [P][rows], pair order
   uint32_t tab[4];             // B32 decode tables (NL4 or Q4)
@@ -104,28 +110,32 @@ __device__ __forceinline__ uint32_t sw128(int r, int chunk) {
 constexpr uint32_t SB3_H16_LO = 0xBCC2C5C7u;   // -1,-3,-5,-7 (bytes 3..0)
 constexpr uint32_t SB3_H16_HI = 0x4745423Cu;   //  7, 5, 3, 1
 
-struct Sb3Q {
-  uint2 lo0, lo1;     // LO[j0], LO[j0+1] of lanes L0, L0+1
-  uint32_t hi0, hi1;  // HI[j0/2] of lanes L0, L0+1
-  uint2 sc;           // sub-scale words of rows g, g+8
-  uint32_t d;         // fp16 d of rows g (low), g+8 (high)
+// One thread's share of a 16-row SB3 tile (one super-block per row): the
+// 16-byte LO and HI words of lanes L0 = 4g + 2p and L0 + 1, and the
+// sub-scale words and fp16 d of rows g and g+8.  Loaded once per
+// super-block, used by its four 64-column k-steps.
+struct Sb3SB {
+  uint4 lo[2][2];   // [segment (sub-blocks 0-3 | 4-7)][lane]
+  uint4 hi[2];      // [lane]: HI[0..3]
+  uint2 sc;         // sub-scale words of rows g, g+8
+  uint32_t d;       // fp16 d of rows g (low), g+8 (high)
 };
 
-// One thread's share of a 16-row SB3 tile for the 64 columns starting at
-// sub-block j0 (even): rows g and g+8, columns 8p..8p+7 of each 16-column
-// half of sub-blocks j0 and j0+1.
-__device__ __forceinline__ Sb3Q sb3_load(const uint8_t* tp, int g, int p,
-                                         int j0) {
+__device__ __forceinline__ void sb3_load(const uint8_t* tp, int g, int p,
+                                         Sb3SB& q) {
   const int L0 = 4 * g + 2 * p;
-  const uint8_t* seg = tp + 512 * (j0 >> 2) + 4 * (j0 & 3) + 16 * L0;
-  Sb3Q q;
-  q.lo0 = ldg_u64(seg);
-  q.lo1 = ldg_u64(seg + 16);
-  q.hi0 = ldg_u32(tp + 1024 + 16 * L0 + 4 * (j0 >> 1));
-  q.hi1 = ldg_u32(tp + 1024 + 16 * L0 + 16 + 4 * (j0 >> 1));
+#pragma unroll
+  for (int l = 0; l < 2; ++l) {
+    q.lo[0][l] = ldg_u128(tp + 16 * (L0 + l));
+    q.lo[1][l] = ldg_u128(tp + 512 + 16 * (L0 + l));
+    q.hi[l] = ldg_u128(tp + 1024 + 16 * (L0 + l));
+  }
   q.sc = ldg_u64(tp + 1536 + 8 * g);
   q.d = ldg_u32(tp + 1600 + 4 * g);
-  return q;
+}
+
+__device__ __forceinline__ uint32_t u4_get(const uint4& v, int i) {
+  return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
 }
 
 // 8 codes of one lane word (nibble n = 4*rowhalf + w) -> fp16 c values as
@@ -143,15 +153,17 @@ __device__ __forceinline__ void sb3_codes_to_h16(uint32_t Q,
   o[3] = prmt(SB3_H16_LO, SB3_H16_HI, X1 >> 16);
 }
 
-__device__ __forceinline__ void sb3_store(const Sb3Q& q, int g, int p,
-                                          int j0, int row0,
-                                          uint32_t a_smem) {
-  const uint32_t dg = half_bcast((uint16_t)(q.d & 0xFFFFu));
-  const uint32_t dg8 = half_bcast((uint16_t)(q.d >> 16));
+// k-step `q` (0..3) of the super-block: sub-blocks j0 = 2q and 2q+1 ->
+// fp16 rows g and g+8 of the swizzled A tile.
+__device__ __forceinline__ void sb3_store(const Sb3SB& sb, int g, int p,
+                                          int q, int row0, uint32_t a_smem) {
+  const int j0 = 2 * q;
+  const uint32_t dg = half_bcast((uint16_t)(sb.d & 0xFFFFu));
+  const uint32_t dg8 = half_bcast((uint16_t)(sb.d >> 16));
 #pragma unroll
   for (int jj = 0; jj < 2; ++jj) {
     const int j = j0 + jj;
-    const int sg = (q.sc.x >> (4 * j)) & 15, sg8 = (q.sc.y >> (4 * j)) & 15;
+    const int sg = (sb.sc.x >> (4 * j)) & 15, sg8 = (sb.sc.y >> (4 * j)) & 15;
     // (2s+1)/8, exact in fp16
     const __half tg = __float2half_rn((float)(2 * sg + 1) * 0.125f);
     const __half tg8 = __float2half_rn((float)(2 * sg8 + 1) * 0.125f);
@@ -160,8 +172,8 @@ __device__ __forceinline__ void sb3_store(const Sb3Q& q, int g, int p,
     uint32_t w[2][2][4];   // [lane][h][words]
 #pragma unroll
     for (int l = 0; l < 2; ++l) {
-      const uint32_t lo = jj ? (l ? q.lo1.y : q.lo0.y) : (l ? q.lo1.x : q.lo0.x);
-      const uint32_t hi = (l ? q.hi1 : q.hi0) >> (2 * jj);
+      const uint32_t lo = u4_get(sb.lo[q >> 1][l], (j & 3));
+      const uint32_t hi = u4_get(sb.hi[l], q) >> (2 * jj);
       const uint32_t Q0 = (lo & 0x33333333u) | ((hi << 2) & 0x44444444u);
       const uint32_t Q1 = ((lo >> 2) & 0x33333333u) | ((hi << 1) & 0x44444444u);
       sb3_codes_to_h16(Q0, w[l][0]);
@@ -204,11 +216,15 @@ __device__ __forceinline__ B32Q b32_load(const uint8_t* tp, int g, int p) {
 // words of d * value(q).  A1 + A2 = value (the byte-table split of the
 // packed layout); both halves are widened to 16 bits and offset into the
 // fp16 range [1024, 2048) so one subtraction gives the exact integer.
-__device__ __forceinline__ void b32_codes(uint32_t sel, const uint32_t (&tab)[4],
+struct B32Tab {
+  uint32_t a0, a1, b0, b1;
+};
+
+__device__ __forceinline__ void b32_codes(uint32_t sel, const B32Tab tab,
                                           uint32_t d2, uint32_t& o01,
                                           uint32_t& o23) {
-  const uint32_t A1 = prmt(tab[0], tab[1], sel);
-  const uint32_t A2 = prmt(tab[2], tab[3], sel ^ 0x8888u);
+  const uint32_t A1 = prmt(tab.a0, tab.a1, sel);
+  const uint32_t A2 = prmt(tab.b0, tab.b1, sel ^ 0x8888u);
   // u8(A1) + A2 = 256 + value, no carry across the 16-bit halves
   const uint32_t v01 = prmt(A1, A2, 0xC1C0u) + prmt(A2, A2, 0x8180u) +
                        0x64006400u;
@@ -221,7 +237,7 @@ __device__ __forceinline__ void b32_codes(uint32_t sel, const uint32_t (&tab)[4]
 
 __device__ __forceinline__ void b32_store(const B32Q& q, int g, int p,
                                           int rh, int row0,
-                                          const uint32_t (&tab)[4],
+                                          const B32Tab tab,
                                           uint32_t a_smem) {
   const uint32_t dw = rh ? q.d.y : q.d.x;
   const uint32_t d2[2] = {half_bcast((uint16_t)(dw & 0xFFFFu)),
@@ -241,9 +257,11 @@ __device__ __forceinline__ void b32_store(const B32Q& q, int g, int p,
 }
 
 // --------------------------------------------------------------- kernel --
+// tmap_b: up: x_g [P][H], down: h16 [P][F], both fp16 in grouped row
+// order, box {64 columns, 16 rows}, 128-byte swizzle.
 template <bool UP, bool SB3>
 __global__ void __launch_bounds__(PF_THREADS, 1)
-    pf_gemm_kernel(const PfParams p) {
+    pf_gemm_kernel(const PfParams p, const __grid_constant__ CUtensorMap tmap_b) {
   using C = PfCfg<UP>;
   constexpr int NA = C::NA, S = C::STAGES;
   extern __shared__ uint8_t smem_raw[];
@@ -262,7 +280,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&full_a[s], PF_NDQ);
-      mbar_init(&full_b[s], 32);
+      mbar_init(&full_b[s], 1);
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -290,15 +308,14 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
     // ------------------------------------------------ MMA issuer ------
     if (lane == 0) {
       uint32_t kstep = 0;
-      int uses[2] = {0, 0};
       int it = 0;
       bool ok = true;
       for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x, ++it) {
         const int4 tile = p.tiles[u / MT];
         const int nmma = (tile.z + 15) & ~15;
         const int ab = UP ? 0 : (it & 1);
-        if (uses[ab] > 0 &&
-            !mbar_wait(&acc_empty[ab], (uses[ab] - 1) & 1, err)) {
+        const int use_ab = UP ? it : (it >> 1);   // earlier uses of buffer ab
+        if (use_ab > 0 && !mbar_wait(&acc_empty[ab], (use_ab - 1) & 1, err)) {
           ok = false;
           break;
         }
@@ -313,7 +330,6 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
             ok = false;
             break;
           }
-          tc::fence_proxy_async_smem();
           tc::fence_after_sync();
           const uint32_t st = sbase + (uint32_t)(s * C::STAGE_BYTES);
           const uint32_t bst = st + NA * PF_A_BYTES;
@@ -329,7 +345,6 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         }
         if (!ok) break;
         tc::commit(&acc_full[ab]);
-        ++uses[ab];
       }
       // all issued MMAs complete before the allocation is released
       tc::commit(drain);
@@ -337,48 +352,32 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
     }
   } else if (warp == PF_WLOAD) {
     // ------------------------------------------- B operand loader -----
-    uint32_t kstep = 0;
-    bool ok = true;
-    for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
-      const int4 tile = p.tiles[u / MT];
-      const int nlen = tile.z, nmma = (nlen + 15) & ~15;
-      const __half* src[PF_BN / 32];
-      uint32_t nbytes[PF_BN / 32];
-#pragma unroll
-      for (int i = 0; i < PF_BN / 32; ++i) {
-        const int n = lane + 32 * i;
-        int64_t row = 0;
-        nbytes[i] = 0;
-        if (n < nlen) {
-          const int pr = tile.y + n;
-          row = UP ? (int64_t)(p.pair_ids[pr] / p.k) : (int64_t)pr;
-          nbytes[i] = 16;
-        }
-        src[i] = p.bsrc + row * p.K;
-      }
-      for (int ks = 0; ks < nk; ++ks, ++kstep) {
-        const int s = (int)(kstep % S);
-        const uint32_t use = kstep / S;
-        if (use > 0 && !mbar_wait(&empty[s], (use - 1) & 1, err)) {
-          ok = false;
-          break;
-        }
-        const uint32_t bst =
-            sbase + (uint32_t)(s * C::STAGE_BYTES + NA * PF_A_BYTES);
-#pragma unroll
-        for (int i = 0; i < PF_BN / 32; ++i) {
-          const int n = lane + 32 * i;
-          if (n < nmma) {
-            const __half* sp = src[i] + ks * PF_BK;
-#pragma unroll
-            for (int c = 0; c < 8; ++c)
-              tc::cp_async16(bst + sw128(n, c), sp + 8 * c, nbytes[i]);
+    // Lane 0 issues the TMA copies of every k-step: 16-row boxes of the
+    // unit's grouped rows; rows past the tile (up to the 16-row MMA
+    // granularity) belong to the next expert or read zeros past the end.
+    if (lane == 0) {
+      uint32_t kstep = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
+        const int4 tile = p.tiles[u / MT];
+        const int nmma = (tile.z + 15) & ~15;
+        const uint32_t bytes = (uint32_t)nmma * (PF_BK * 2);
+        for (int ks = 0; ks < nk; ++ks, ++kstep) {
+          const int s = (int)(kstep % S);
+          const uint32_t use = kstep / S;
+          if (use > 0 && !mbar_wait(&empty[s], (use - 1) & 1, err)) {
+            ok = false;
+            break;
           }
+          const uint32_t bst =
+              sbase + (uint32_t)(s * C::STAGE_BYTES + NA * PF_A_BYTES);
+          mbar_arrive_expect_tx(&full_b[s], bytes);
+          for (int n = 0; n < nmma; n += 16)
+            tc::tma_load_2d(bst + n * 128, &tmap_b, ks * PF_BK, tile.y + n,
+                            &full_b[s]);
         }
-        tc::cp_async_arrive_noinc(&full_b[s]);
       }
     }
-    tc::cp_async_wait_all();
   } else if (warp >= PF_WDQ0) {
     // ------------------------------------------ A operand dequant -----
     const int t = threadIdx.x - PF_WDQ0 * 32;   // 0..255
@@ -387,7 +386,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
     const int tcols = SB3 ? SB3_TILE_COLS : B32_TILE_COLS;
     const int tbytes = SB3 ? SB3_TILE_BYTES : B32_TILE_BYTES;
     const int64_t trow_stride = (int64_t)(p.K / tcols) * tbytes;  // 16 rows
-    uint32_t tab[4] = {p.tab[0], p.tab[1], p.tab[2], p.tab[3]};
+    const B32Tab tab = {p.tab[0], p.tab[1], p.tab[2], p.tab[3]};
     // item geometry (fixed per thread)
     int it_g[IPT], it_p[IPT], it_rh[IPT], it_ti[IPT], it_a[IPT];
     bool it_on[IPT];
@@ -407,7 +406,6 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         it_a[i] = item >> 8;
       }
     }
-    using Q = typename std::conditional<SB3, Sb3Q, B32Q>::type;
     // prefetch position (unit, k-step) and its tile pointers
     int pu = blockIdx.x, pks = 0;
     const uint8_t* ptp[IPT];
@@ -426,111 +424,164 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         ptp[i] = blob + (it_a[i] ? p.off_a1 : p.off_a0) +
                  (int64_t)(m * (PF_BM / 16) + it_ti[i]) * trow_stride;
     };
-    auto fetch = [&](Q (&q)[IPT]) {
-      if (pu >= n_units) return;
-      const int kc = SB3 ? (pks >> 2) : pks;
-#pragma unroll
-      for (int i = 0; i < IPT; ++i) {
-        if (!it_on[i]) continue;
-        const uint8_t* tp = ptp[i] + (int64_t)kc * tbytes;
-        if constexpr (SB3)
-          q[i] = sb3_load(tp, it_g[i], it_p[i], 2 * (pks & 3));
-        else
-          q[i] = b32_load(tp, it_g[i], it_p[i]);
-      }
-      if (++pks == nk) {
-        pks = 0;
-        pu += gridDim.x;
-        if (pu < n_units) set_unit(pu);
-      }
+    // One k-step: wait for the stage, write the A tile(s), publish.
+    uint32_t kstep = 0;
+    auto stage_begin = [&](uint32_t& st) -> bool {
+      const int s = (int)(kstep % S);
+      const uint32_t use = kstep / S;
+      if (use > 0 && !mbar_wait(&empty[s], (use - 1) & 1, err)) return false;
+      st = sbase + (uint32_t)(s * C::STAGE_BYTES);
+      return true;
+    };
+    auto stage_end = [&]() {
+      tc::fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&full_a[kstep % S]);
+      ++kstep;
     };
     if (pu < n_units) set_unit(pu);
-    Q q0[IPT], q1[IPT], q2[IPT];
-    fetch(q0);
-    fetch(q1);
-    uint32_t kstep = 0;
     bool ok = true;
-    for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
-      for (int ks = 0; ks < nk; ++ks, ++kstep) {
-        fetch(q2);
-        const int s = (int)(kstep % S);
-        const uint32_t use = kstep / S;
-        if (use > 0 && !mbar_wait(&empty[s], (use - 1) & 1, err)) {
-          ok = false;
-          break;
+    if constexpr (SB3) {
+      // super-block granularity (4 k-steps), prefetched one ahead
+      static_assert(IPT == 1, "one SB3 item per thread");
+      const int nsb = nk / 4;
+      auto fetch = [&](Sb3SB& q) {
+        if (pu >= n_units) return;
+        if (it_on[0])
+          sb3_load(ptp[0] + (int64_t)pks * SB3_TILE_BYTES, it_g[0], it_p[0], q);
+        if (++pks == nsb) {
+          pks = 0;
+          pu += gridDim.x;
+          if (pu < n_units) set_unit(pu);
         }
-        const uint32_t st = sbase + (uint32_t)(s * C::STAGE_BYTES);
+      };
+      Sb3SB cur, nxt;
+      fetch(cur);
+      for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
+        for (int sb = 0; ok && sb < nsb; ++sb) {
+          fetch(nxt);
 #pragma unroll
-        for (int i = 0; i < IPT; ++i) {
-          if (!it_on[i]) continue;
-          const uint32_t a_smem = st + it_a[i] * PF_A_BYTES;
-          if constexpr (SB3)
-            sb3_store(q0[i], it_g[i], it_p[i], 2 * (ks & 3), 16 * it_ti[i],
-                      a_smem);
-          else
-            b32_store(q0[i], it_g[i], it_p[i], it_rh[i], 16 * it_ti[i], tab,
-                      a_smem);
+          for (int q = 0; q < 4; ++q) {
+            uint32_t st;
+            if (!stage_begin(st)) {
+              ok = false;
+              break;
+            }
+            if (it_on[0])
+              sb3_store(cur, it_g[0], it_p[0], q, 16 * it_ti[0],
+                        st + it_a[0] * PF_A_BYTES);
+            stage_end();
+          }
+          cur = nxt;
         }
-        tc::fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&full_a[s]);
+      }
+    } else {
+      // k-step granularity, prefetched two ahead
+      auto fetch = [&](B32Q (&q)[IPT]) {
+        if (pu >= n_units) return;
 #pragma unroll
-        for (int i = 0; i < IPT; ++i) {
-          q0[i] = q1[i];
-          q1[i] = q2[i];
+        for (int i = 0; i < IPT; ++i)
+          if (it_on[i])
+            q[i] = b32_load(ptp[i] + (int64_t)pks * B32_TILE_BYTES, it_g[i],
+                            it_p[i]);
+        if (++pks == nk) {
+          pks = 0;
+          pu += gridDim.x;
+          if (pu < n_units) set_unit(pu);
+        }
+      };
+      B32Q q0[IPT], q1[IPT], q2[IPT];
+      fetch(q0);
+      fetch(q1);
+      for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
+        for (int ks = 0; ks < nk; ++ks) {
+          fetch(q2);
+          uint32_t st;
+          if (!stage_begin(st)) {
+            ok = false;
+            break;
+          }
+#pragma unroll
+          for (int i = 0; i < IPT; ++i)
+            if (it_on[i])
+              b32_store(q0[i], it_g[i], it_p[i], it_rh[i], 16 * it_ti[i], tab,
+                        st + it_a[i] * PF_A_BYTES);
+          stage_end();
+#pragma unroll
+          for (int i = 0; i < IPT; ++i) {
+            q0[i] = q1[i];
+            q1[i] = q2[i];
+          }
         }
       }
     }
   } else {
     // ------------------------------------------------- epilogue -------
-    int uses[2] = {0, 0};
+    // Per unit, the rows' metadata (up: the token's x scale; down: the
+    // pair id) goes to this warp's slice of shared memory before the
+    // accumulator wait, so its global latency overlaps the MMAs.
     int it = 0;
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    float* meta_f = reinterpret_cast<float*>(smem + C::META_OFF) + warp * PF_BN;
+    int32_t* meta_i = reinterpret_cast<int32_t*>(meta_f);
     for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++it) {
       const int4 tile = p.tiles[u / MT];
       const int nlen = tile.z, row0 = tile.y;
       const int ab = UP ? 0 : (it & 1);
-      if (!mbar_wait(&acc_full[ab], uses[ab] & 1, err)) break;
+      __syncwarp();
+      for (int n = lane; n < nlen; n += 32) {
+        if constexpr (UP)
+          meta_f[n] = p.xscale[row0 + n];
+        else
+          meta_i[n] = p.pair_ids[row0 + n];
+      }
+      __syncwarp();
+      const int use_ab = UP ? it : (it >> 1);
+      if (!mbar_wait(&acc_full[ab], use_ab & 1, err)) break;
       tc::fence_after_sync();
       const int col = (u % MT) * PF_BM + warp * 32 + lane;  // output column
-      for (int c0 = 0; c0 < nlen; c0 += 16) {
-        const int nl = c0 + (lane & 15);
-        const bool lv = nl < nlen;
-        if constexpr (UP) {
-          float uacc[16], gacc[16];
-          tc::ld_32x32b_x16(tmem + lane_base + (uint32_t)c0, uacc);
-          tc::ld_32x32b_x16(tmem + lane_base + 256u + (uint32_t)c0, gacc);
+      if constexpr (UP) {
+        float hmax = 0.f;
+        __half* hp = p.h16 + (int64_t)row0 * p.rows + col;
+        for (int c0 = 0; c0 < nlen; c0 += 32) {
+          float ua[32], ga[32];
+          tc::ld_32x32b_x16(tmem + lane_base + (uint32_t)c0, *(float(*)[16])&ua[0]);
+          tc::ld_32x32b_x16(tmem + lane_base + (uint32_t)(c0 + 16),
+                            *(float(*)[16])&ua[16]);
+          tc::ld_32x32b_x16(tmem + lane_base + 256u + (uint32_t)c0,
+                            *(float(*)[16])&ga[0]);
+          tc::ld_32x32b_x16(tmem + lane_base + 256u + (uint32_t)(c0 + 16),
+                            *(float(*)[16])&ga[16]);
           tc::wait_ld();
-          const float sc_l = lv ? p.xscale[p.pair_ids[row0 + nl] / p.k] : 1.f;
-          bool bad = false;
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float sc = __shfl_sync(0xffffffffu, sc_l, i);
+          for (int i = 0; i < 32; ++i) {
             if (c0 + i < nlen) {
-              const float uu = uacc[i] * sc, gg = gacc[i] * sc;
-              const float hv = gg / (1.0f + __expf(-gg)) * uu;
-              const __half hh = __float2half_rn(hv);
-              bad |= __hisinf(hh) != 0;
-              p.h16[(int64_t)(row0 + c0 + i) * p.rows + col] = hh;
+              const float sc = meta_f[c0 + i];
+              const float uu = ua[i] * sc, gg = ga[i] * sc;
+              const float hv = __fdividef(gg, 1.0f + __expf(-gg)) * uu;
+              hmax = fmaxf(hmax, fabsf(hv));
+              hp[(int64_t)(c0 + i) * p.rows] = __float2half_rn(hv);
             }
           }
-          if (bad) set_err(err, MOE_ERR_DEVICE);
-        } else {
-          float acc[16];
-          tc::ld_32x32b_x16(tmem + lane_base + (uint32_t)(ab * 256 + c0), acc);
+        }
+        if (!(hmax < 65520.f)) set_err(err, MOE_ERR_DEVICE);   // fp16 range
+      } else {
+        float* yp = p.y + col;
+        for (int c0 = 0; c0 < nlen; c0 += 32) {
+          float acc[32];
+          tc::ld_32x32b_x16(tmem + lane_base + (uint32_t)(ab * 256 + c0),
+                            *(float(*)[16])&acc[0]);
+          tc::ld_32x32b_x16(tmem + lane_base + (uint32_t)(ab * 256 + c0 + 16),
+                            *(float(*)[16])&acc[16]);
           tc::wait_ld();
-          const int pr_l = lv ? p.pair_ids[row0 + nl] : 0;
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int pr = __shfl_sync(0xffffffffu, pr_l, i);
-            if (c0 + i < nlen) p.y[(int64_t)pr * p.rows + col] = acc[i];
-          }
+          for (int i = 0; i < 32; ++i)
+            if (c0 + i < nlen) yp[(int64_t)meta_i[c0 + i] * p.rows] = acc[i];
         }
       }
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[ab]);
-      ++uses[ab];
     }
   }
 
@@ -597,17 +648,27 @@ __global__ void __launch_bounds__(1024)
   }
 }
 
-// x (bf16) -> fp16 with a per-token power-of-two scale that keeps every
-// value below 2^15 (2^sigma = 1 unless max|x_t| >= 2^15).
+// Grouped row r = x[pair_ids[r] / k] as fp16, scaled by a per-row power of
+// two 2^-sigma that keeps every value below 2^15 (sigma = 0 unless
+// max|x_t| >= 2^15); xscale[r] = 2^sigma.  H a multiple of 8.
 __global__ void __launch_bounds__(256)
-    pf_x16_kernel(const uint16_t* __restrict__ x, int H,
-                  __half* __restrict__ x16, float* __restrict__ xscale) {
+    pf_xg_kernel(const uint16_t* __restrict__ x, int H,
+                 const int32_t* __restrict__ pair_ids, int k,
+                 __half* __restrict__ xg, float* __restrict__ xscale) {
   __shared__ float red[8];
-  const int t = blockIdx.x;
-  const uint16_t* xr = x + (int64_t)t * H;
+  const int64_t r = blockIdx.x;
+  const uint4* xr =
+      reinterpret_cast<const uint4*>(x + (int64_t)(pair_ids[r] / k) * H);
+  const int nch = H / 8;
   float m = 0.f;
-  for (int i = threadIdx.x; i < H; i += blockDim.x)
-    m = fmaxf(m, fabsf(bf16_to_f32(xr[i])));
+  for (int c = threadIdx.x; c < nch; c += blockDim.x) {
+    const uint4 v = __ldg(xr + c);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      m = fmaxf(m, fmaxf(fabsf(__uint_as_float(w[i] << 16)),
+                         fabsf(__uint_as_float(w[i] & 0xFFFF0000u))));
+  }
 #pragma unroll
   for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
@@ -617,10 +678,20 @@ __global__ void __launch_bounds__(256)
   int sigma = 0;
   if (m >= 32768.f && m <= 3.0e38f) sigma = ilogbf(m) - 14;
   const float inv = ldexpf(1.f, -sigma);
-  if (threadIdx.x == 0) xscale[t] = ldexpf(1.f, sigma);
-  __half* o = x16 + (int64_t)t * H;
-  for (int i = threadIdx.x; i < H; i += blockDim.x)
-    o[i] = __float2half_rn(bf16_to_f32(xr[i]) * inv);
+  if (threadIdx.x == 0) xscale[r] = ldexpf(1.f, sigma);
+  uint4* o = reinterpret_cast<uint4*>(xg + r * H);
+  for (int c = threadIdx.x; c < nch; c += blockDim.x) {
+    const uint4 v = __ldg(xr + c);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t h[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const __half2 t = __floats2half2_rn(__uint_as_float(w[i] << 16) * inv,
+                                          __uint_as_float(w[i] & 0xFFFF0000u) * inv);
+      h[i] = *reinterpret_cast<const uint32_t*>(&t);
+    }
+    o[c] = make_uint4(h[0], h[1], h[2], h[3]);
+  }
 }
 
 }  // namespace
@@ -641,13 +712,45 @@ static void pf_tables(int fmt, uint32_t (&t)[4]) {
   }
 }
 
+// fp16 [outer][inner] row-major tensor map with the 128-byte swizzle and
+// zero fill out of range; encoded through the driver entry point.
+static moe_status encode_f16_map(CUtensorMap* m, const void* base,
+                                 uint64_t inner, uint64_t outer,
+                                 uint32_t box_rows) {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::mutex mu;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (!fn) {
+      void* f = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f,
+                                  cudaEnableDefault, &q) != cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || !f)
+        return MOE_ERR_CUDA;
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    }
+  }
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {inner * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)PF_BK, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r =
+      fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims,
+         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
+}
+
 template <bool UP, bool SB3>
-static moe_status pf_launch(const PfParams& prm, cudaStream_t s) {
+static moe_status pf_launch(const PfParams& prm, const CUtensorMap& map,
+                            cudaStream_t s) {
   const void* fn = reinterpret_cast<const void*>(&pf_gemm_kernel<UP, SB3>);
   moe_status st = ensure_smem(fn, PfCfg<UP>::SMEM);
   if (st != MOE_OK) return st;
   pf_gemm_kernel<UP, SB3>
-      <<<num_sms(), PF_THREADS, PfCfg<UP>::SMEM, s>>>(prm);
+      <<<num_sms(), PF_THREADS, PfCfg<UP>::SMEM, s>>>(prm, map);
   return launch_status();
 }
 
@@ -655,9 +758,14 @@ moe_status launch_pf_up(const moe_layer_desc& d, const uint16_t* x, int T,
                         int k, const int32_t* offsets,
                         const int32_t* pair_ids, const int32_t* blob_index,
                         const FfnWs& w, cudaStream_t s) {
-  pf_x16_kernel<<<T, 256, 0, s>>>(x, d.H, w.x16, w.xscale);
+  const int64_t P = (int64_t)T * k;
+  CUtensorMap map;
+  moe_status st = encode_f16_map(&map, w.x16, (uint64_t)d.H, (uint64_t)P, 16);
+  if (st != MOE_OK) return st;
+  pf_xg_kernel<<<(unsigned)P, 256, 0, s>>>(x, d.H, pair_ids, k, w.x16,
+                                           w.xscale);
   pf_plan_kernel<<<1, 1024, 0, s>>>(offsets, d.E, w.tiles, w.n_tiles);
-  moe_status st = launch_status();
+  st = launch_status();
   if (st != MOE_OK) return st;
   PfParams prm{};
   prm.pool = d.pool;
@@ -671,18 +779,21 @@ moe_status launch_pf_up(const moe_layer_desc& d, const uint16_t* x, int T,
   prm.pair_ids = pair_ids;
   prm.tiles = w.tiles;
   prm.n_tiles = w.n_tiles;
-  prm.bsrc = w.x16;
   prm.xscale = w.xscale;
   prm.h16 = reinterpret_cast<__half*>(w.h);
   prm.err = w.err;
   pf_tables(d.fmt_up_gate, prm.tab);
-  return d.fmt_up_gate == MOE_SB3_256 ? pf_launch<true, true>(prm, s)
-                                      : pf_launch<true, false>(prm, s);
+  return d.fmt_up_gate == MOE_SB3_256 ? pf_launch<true, true>(prm, map, s)
+                                      : pf_launch<true, false>(prm, map, s);
 }
 
-moe_status launch_pf_down(const moe_layer_desc& d, int k,
+moe_status launch_pf_down(const moe_layer_desc& d, int T, int k,
                           const int32_t* pair_ids, const int32_t* blob_index,
                           const FfnWs& w, float* y, cudaStream_t s) {
+  const int64_t P = (int64_t)T * k;
+  CUtensorMap map;
+  moe_status st = encode_f16_map(&map, w.h, (uint64_t)d.F, (uint64_t)P, 16);
+  if (st != MOE_OK) return st;
   PfParams prm{};
   prm.pool = d.pool;
   prm.blob_stride = d.blob_stride;
@@ -695,12 +806,11 @@ moe_status launch_pf_down(const moe_layer_desc& d, int k,
   prm.pair_ids = pair_ids;
   prm.tiles = w.tiles;
   prm.n_tiles = w.n_tiles;
-  prm.bsrc = reinterpret_cast<const __half*>(w.h);
   prm.y = y;
   prm.err = w.err;
   pf_tables(d.fmt_down, prm.tab);
-  return d.fmt_down == MOE_SB3_256 ? pf_launch<false, true>(prm, s)
-                                   : pf_launch<false, false>(prm, s);
+  return d.fmt_down == MOE_SB3_256 ? pf_launch<false, true>(prm, map, s)
+                                   : pf_launch<false, false>(prm, map, s);
 }
 
 }  // namespace moe

@@ -1,5 +1,6 @@
 // PTX wrappers for the 5th-generation tensor cores (tcgen05) and the
-// Ampere-style asynchronous copies that feed them.  sm_100a only.
+// copies that feed them (TMA tensor copies, Ampere-style cp.async).
+// sm_100a only.
 #pragma once
 
 #include "moe_internal.cuh"
@@ -96,6 +97,30 @@ __device__ __forceinline__ void ld_32x32b_x16(uint32_t taddr, float (&v)[16]) {
 }
 __device__ __forceinline__ void wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// ---- tensor memory accelerator (TMA) copies ----------------------------
+// 2-D tile load of box {64, rows} at element coordinates (x, y) into
+// shared memory; completion counted in bytes on `bar`.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* map,
+                                            int x, int y, void* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::"
+      "complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+// Four rows y0..y3 (box one row high), columns x.., written back to back.
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const void* map,
+                                            int x, int y0, int y1, int y2,
+                                            int y3, void* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4."
+      "mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::
+          "r"(dst),
+      "l"(map), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3),
+      "r"(smem_u32(bar))
+      : "memory");
 }
 
 // ---- Ampere-style asynchronous copies --------------------------------
