@@ -8,7 +8,8 @@ namespace moe {
 
 moe_status launch_route(const uint16_t* x, int T, int H, const uint16_t* wr,
                         int E, const float* bias, int k, int32_t* topk_idx,
-                        float* topk_w, float* logits, cudaStream_t s);
+                        float* topk_w, float* logits, int32_t* err,
+                        cudaStream_t s);
 moe_status launch_group(const int32_t* idx, int T, int k, int E,
                         int32_t* offsets, int32_t* pair_ids, int32_t* active,
                         int32_t* n_active, int32_t* scratch, int32_t* err,
@@ -297,7 +298,7 @@ extern "C" moe_status moe_route_topk(const uint16_t* x, int T, int H,
     return MOE_ERR_SHAPE;
   if (((uintptr_t)x | (uintptr_t)w_router) % 16) return MOE_ERR_INVALID;
   return launch_route(x, T, H, w_router, E, bias, k, topk_idx, topk_w,
-                      logits_out, (cudaStream_t)stream);
+                      logits_out, nullptr, (cudaStream_t)stream);
 }
 
 extern "C" size_t moe_group_workspace_bytes(int T, int k, int E) {
@@ -433,7 +434,7 @@ extern "C" moe_status moe_layer_forward(
                                blob_index, residual, out, out_bf16, topk_idx,
                                topk_w, logits, w.fused, w.ffn.err, s);
   st = launch_route(x, T, desc->H, w_router, desc->E, bias, k, topk_idx,
-                    topk_w, logits, s);
+                    topk_w, logits, w.ffn.err, s);
   if (st != MOE_OK) return st;
   st = launch_group(topk_idx, T, k, desc->E, w.offsets, w.pair_ids, w.active,
                     w.n_active, w.grp, w.ffn.err, s);

@@ -152,10 +152,20 @@ __global__ void __launch_bounds__(128)
   }
 }
 
+bool route_tc_supported(int T, int H);
+moe_status launch_route_tc(const uint16_t* x, int T, int H,
+                           const uint16_t* wr, int E, const float* bias,
+                           float* logits, int32_t* err, cudaStream_t s);
+
 moe_status launch_route(const uint16_t* x, int T, int H, const uint16_t* wr,
                         int E, const float* bias, int k, int32_t* topk_idx,
-                        float* topk_w, float* logits, cudaStream_t s) {
-  if (T <= DEC_TMAX) {
+                        float* topk_w, float* logits, int32_t* err,
+                        cudaStream_t s) {
+  if (route_tc_supported(T, H)) {
+    const moe_status st =
+        launch_route_tc(x, T, H, wr, E, bias, logits, err, s);
+    if (st != MOE_OK) return st;
+  } else if (T <= DEC_TMAX) {
     const size_t smem = (size_t)T * H * 2;
     const moe_status st =
         ensure_smem((const void*)route_logits_small_kernel, smem);

@@ -44,6 +44,7 @@ def _check_route(x_bits, wr_bits, bias, k):
 @pytest.mark.parametrize("T,shape,zipf", [
     (8, synth.TINY, False), (1, synth.BIG, False), (3, synth.BIG, False),
     (3, synth.BIG, True), (8, synth.BIG, True), (300, synth.BIG, True),
+    (9536, synth.BIG, True), (40, synth.TINY, False),
 ])
 def test_route_topk_vs_oracle(T, shape, zipf):
     x, wr, bias = route_inputs(shape, 0, 1, T, zipf=zipf)
