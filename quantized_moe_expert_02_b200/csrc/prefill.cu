@@ -51,6 +51,13 @@ struct PfCfg {
   static constexpr int SMEM = META_OFF + META_BYTES + 1024;   // + alignment
 };
 
+// B operand tensor maps: the same fp16 [P][K] tensor with box heights
+// 256, 128, 64, 32, 16 rows (a tile of n rows takes at most one of each).
+constexpr int PF_NMAPS = 5;
+struct PfMaps {
+  CUtensorMap m[PF_NMAPS];
+};
+
 struct PfParams {
   const uint8_t* pool;
   int64_t blob_stride;
@@ -257,11 +264,11 @@ __device__ __forceinline__ void b32_store(const B32Q& q, int g, int p,
 }
 
 // --------------------------------------------------------------- kernel --
-// tmap_b: up: x_g [P][H], down: h16 [P][F], both fp16 in grouped row
-// order, box {64 columns, 16 rows}, 128-byte swizzle.
+// maps: up: x_g [P][H], down: h16 [P][F], both fp16 in grouped row
+// order, boxes of 64 columns, 128-byte swizzle.
 template <bool UP, bool SB3>
 __global__ void __launch_bounds__(PF_THREADS, 1)
-    pf_gemm_kernel(const PfParams p, const __grid_constant__ CUtensorMap tmap_b) {
+    pf_gemm_kernel(const PfParams p, const __grid_constant__ PfMaps maps) {
   using C = PfCfg<UP>;
   constexpr int NA = C::NA, S = C::STAGES;
   extern __shared__ uint8_t smem_raw[];
@@ -352,9 +359,10 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
     }
   } else if (warp == PF_WLOAD) {
     // ------------------------------------------- B operand loader -----
-    // Lane 0 issues the TMA copies of every k-step: 16-row boxes of the
-    // unit's grouped rows; rows past the tile (up to the 16-row MMA
-    // granularity) belong to the next expert or read zeros past the end.
+    // Lane 0 issues the TMA copies of every k-step: the unit's grouped
+    // rows in boxes of 256/128/64/32/16 rows; rows past the tile (up to the
+    // 16-row MMA granularity) belong to the next expert or read zeros past
+    // the end.
     if (lane == 0) {
       uint32_t kstep = 0;
       bool ok = true;
@@ -372,9 +380,16 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
           const uint32_t bst =
               sbase + (uint32_t)(s * C::STAGE_BYTES + NA * PF_A_BYTES);
           mbar_arrive_expect_tx(&full_b[s], bytes);
-          for (int n = 0; n < nmma; n += 16)
-            tc::tma_load_2d(bst + n * 128, &tmap_b, ks * PF_BK, tile.y + n,
-                            &full_b[s]);
+          int n = 0;
+#pragma unroll
+          for (int b = 0; b < PF_NMAPS; ++b) {
+            const int rows = 256 >> b;
+            if (nmma - n >= rows) {
+              tc::tma_load_2d(bst + n * 128, &maps.m[b], ks * PF_BK,
+                              tile.y + n, &full_b[s]);
+              n += rows;
+            }
+          }
         }
       }
     }
@@ -529,22 +544,24 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
       const int nlen = tile.z, row0 = tile.y;
       const int ab = UP ? 0 : (it & 1);
       __syncwarp();
-      for (int n = lane; n < nlen; n += 32) {
+      for (int n = lane; n < ((nlen + 31) & ~31); n += 32) {
         if constexpr (UP)
-          meta_f[n] = p.xscale[row0 + n];
+          meta_f[n] = n < nlen ? p.xscale[row0 + n] : 1.f;
         else
-          meta_i[n] = p.pair_ids[row0 + n];
+          meta_i[n] = n < nlen ? p.pair_ids[row0 + n] : 0;
       }
       __syncwarp();
       const int use_ab = UP ? it : (it >> 1);
       if (!mbar_wait(&acc_full[ab], use_ab & 1, err)) break;
       tc::fence_after_sync();
       const int col = (u % MT) * PF_BM + warp * 32 + lane;  // output column
+      // Each 32-column chunk reads its metadata into registers first, so
+      // no shared-memory load waits behind a global store.
       if constexpr (UP) {
         float hmax = 0.f;
         __half* hp = p.h16 + (int64_t)row0 * p.rows + col;
         for (int c0 = 0; c0 < nlen; c0 += 32) {
-          float ua[32], ga[32];
+          float ua[32], ga[32], sc[32];
           tc::ld_32x32b_x16(tmem + lane_base + (uint32_t)c0, *(float(*)[16])&ua[0]);
           tc::ld_32x32b_x16(tmem + lane_base + (uint32_t)(c0 + 16),
                             *(float(*)[16])&ua[16]);
@@ -552,31 +569,43 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                             *(float(*)[16])&ga[0]);
           tc::ld_32x32b_x16(tmem + lane_base + 256u + (uint32_t)(c0 + 16),
                             *(float(*)[16])&ga[16]);
+#pragma unroll
+          for (int i = 0; i < 32; i += 4) {
+            const float4 v = *reinterpret_cast<const float4*>(meta_f + c0 + i);
+            sc[i] = v.x; sc[i + 1] = v.y; sc[i + 2] = v.z; sc[i + 3] = v.w;
+          }
           tc::wait_ld();
+          __half hv16[32];
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
-            if (c0 + i < nlen) {
-              const float sc = meta_f[c0 + i];
-              const float uu = ua[i] * sc, gg = ga[i] * sc;
-              const float hv = __fdividef(gg, 1.0f + __expf(-gg)) * uu;
-              hmax = fmaxf(hmax, fabsf(hv));
-              hp[(int64_t)(c0 + i) * p.rows] = __float2half_rn(hv);
-            }
+            const float uu = ua[i] * sc[i], gg = ga[i] * sc[i];
+            const float hv = __fdividef(gg, 1.0f + __expf(-gg)) * uu;
+            if (c0 + i < nlen) hmax = fmaxf(hmax, fabsf(hv));
+            hv16[i] = __float2half_rn(hv);
           }
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (c0 + i < nlen) hp[(int64_t)(c0 + i) * p.rows] = hv16[i];
         }
         if (!(hmax < 65520.f)) set_err(err, MOE_ERR_DEVICE);   // fp16 range
       } else {
         float* yp = p.y + col;
         for (int c0 = 0; c0 < nlen; c0 += 32) {
           float acc[32];
+          int pr[32];
           tc::ld_32x32b_x16(tmem + lane_base + (uint32_t)(ab * 256 + c0),
                             *(float(*)[16])&acc[0]);
           tc::ld_32x32b_x16(tmem + lane_base + (uint32_t)(ab * 256 + c0 + 16),
                             *(float(*)[16])&acc[16]);
+#pragma unroll
+          for (int i = 0; i < 32; i += 4) {
+            const int4 v = *reinterpret_cast<const int4*>(meta_i + c0 + i);
+            pr[i] = v.x; pr[i + 1] = v.y; pr[i + 2] = v.z; pr[i + 3] = v.w;
+          }
           tc::wait_ld();
 #pragma unroll
           for (int i = 0; i < 32; ++i)
-            if (c0 + i < nlen) yp[(int64_t)meta_i[c0 + i] * p.rows] = acc[i];
+            if (c0 + i < nlen) yp[(int64_t)pr[i] * p.rows] = acc[i];
         }
       }
       tc::fence_before_sync();
@@ -743,8 +772,18 @@ static moe_status encode_f16_map(CUtensorMap* m, const void* base,
   return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
 }
 
+static moe_status encode_maps(PfMaps* maps, const void* base, uint64_t inner,
+                              uint64_t outer) {
+  for (int b = 0; b < PF_NMAPS; ++b) {
+    const moe_status st =
+        encode_f16_map(&maps->m[b], base, inner, outer, 256u >> b);
+    if (st != MOE_OK) return st;
+  }
+  return MOE_OK;
+}
+
 template <bool UP, bool SB3>
-static moe_status pf_launch(const PfParams& prm, const CUtensorMap& map,
+static moe_status pf_launch(const PfParams& prm, const PfMaps& map,
                             cudaStream_t s) {
   const void* fn = reinterpret_cast<const void*>(&pf_gemm_kernel<UP, SB3>);
   moe_status st = ensure_smem(fn, PfCfg<UP>::SMEM);
@@ -759,8 +798,8 @@ moe_status launch_pf_up(const moe_layer_desc& d, const uint16_t* x, int T,
                         const int32_t* pair_ids, const int32_t* blob_index,
                         const FfnWs& w, cudaStream_t s) {
   const int64_t P = (int64_t)T * k;
-  CUtensorMap map;
-  moe_status st = encode_f16_map(&map, w.x16, (uint64_t)d.H, (uint64_t)P, 16);
+  PfMaps map;
+  moe_status st = encode_maps(&map, w.x16, (uint64_t)d.H, (uint64_t)P);
   if (st != MOE_OK) return st;
   pf_xg_kernel<<<(unsigned)P, 256, 0, s>>>(x, d.H, pair_ids, k, w.x16,
                                            w.xscale);
@@ -791,8 +830,8 @@ moe_status launch_pf_down(const moe_layer_desc& d, int T, int k,
                           const int32_t* pair_ids, const int32_t* blob_index,
                           const FfnWs& w, float* y, cudaStream_t s) {
   const int64_t P = (int64_t)T * k;
-  CUtensorMap map;
-  moe_status st = encode_f16_map(&map, w.h, (uint64_t)d.F, (uint64_t)P, 16);
+  PfMaps map;
+  moe_status st = encode_maps(&map, w.h, (uint64_t)d.F, (uint64_t)P);
   if (st != MOE_OK) return st;
   PfParams prm{};
   prm.pool = d.pool;
