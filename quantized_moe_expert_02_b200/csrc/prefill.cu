@@ -117,32 +117,32 @@ __device__ __forceinline__ uint32_t sw128(int r, int chunk) {
 constexpr uint32_t SB3_H16_LO = 0xBCC2C5C7u;   // -1,-3,-5,-7 (bytes 3..0)
 constexpr uint32_t SB3_H16_HI = 0x4745423Cu;   //  7, 5, 3, 1
 
-// One thread's share of a 16-row SB3 tile (one super-block per row): the
-// 16-byte LO and HI words of lanes L0 = 4g + 2p and L0 + 1, and the
-// sub-scale words and fp16 d of rows g and g+8.  Loaded once per
-// super-block, used by its four 64-column k-steps.
-struct Sb3SB {
-  uint4 lo[2][2];   // [segment (sub-blocks 0-3 | 4-7)][lane]
-  uint4 hi[2];      // [lane]: HI[0..3]
+// One thread's share of a 16-row SB3 tile (one super-block per row) for
+// one of the two dequant groups: group gamma takes k-steps q = gamma and
+// gamma + 2 of the super-block's four 64-column k-steps.  Holds, for lanes
+// L0 = 4g + 2p and L0 + 1, the LO words 2*gamma, 2*gamma+1 of both
+// segments and the HI words gamma, gamma+2, plus the sub-scale words and
+// fp16 d of rows g and g+8.
+struct Sb3Half {
+  uint2 lo[2][2];   // [segment][lane]
+  uint2 hi[2];      // [lane]: HI[gamma], HI[gamma+2]
   uint2 sc;         // sub-scale words of rows g, g+8
   uint32_t d;       // fp16 d of rows g (low), g+8 (high)
 };
 
 __device__ __forceinline__ void sb3_load(const uint8_t* tp, int g, int p,
-                                         Sb3SB& q) {
+                                         int gamma, Sb3Half& q) {
   const int L0 = 4 * g + 2 * p;
 #pragma unroll
   for (int l = 0; l < 2; ++l) {
-    q.lo[0][l] = ldg_u128(tp + 16 * (L0 + l));
-    q.lo[1][l] = ldg_u128(tp + 512 + 16 * (L0 + l));
-    q.hi[l] = ldg_u128(tp + 1024 + 16 * (L0 + l));
+    const uint8_t* lw = tp + 16 * (L0 + l);
+    q.lo[0][l] = ldg_u64(lw + 8 * gamma);
+    q.lo[1][l] = ldg_u64(lw + 512 + 8 * gamma);
+    q.hi[l] = make_uint2(ldg_u32(lw + 1024 + 4 * gamma),
+                         ldg_u32(lw + 1024 + 8 + 4 * gamma));
   }
   q.sc = ldg_u64(tp + 1536 + 8 * g);
   q.d = ldg_u32(tp + 1600 + 4 * g);
-}
-
-__device__ __forceinline__ uint32_t u4_get(const uint4& v, int i) {
-  return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
 }
 
 // 8 codes of one lane word (nibble n = 4*rowhalf + w) -> fp16 c values as
@@ -160,10 +160,13 @@ __device__ __forceinline__ void sb3_codes_to_h16(uint32_t Q,
   o[3] = prmt(SB3_H16_LO, SB3_H16_HI, X1 >> 16);
 }
 
-// k-step `q` (0..3) of the super-block: sub-blocks j0 = 2q and 2q+1 ->
-// fp16 rows g and g+8 of the swizzled A tile.
-__device__ __forceinline__ void sb3_store(const Sb3SB& sb, int g, int p,
-                                          int q, int row0, uint32_t a_smem) {
+// The group's k-step qh (0/1) of the super-block, i.e. k-step
+// q = gamma + 2*qh: sub-blocks j0 = 2q and 2q+1 -> fp16 rows g and g+8 of
+// the swizzled A tile.
+__device__ __forceinline__ void sb3_store(const Sb3Half& sb, int g, int p,
+                                          int gamma, int qh, int row0,
+                                          uint32_t a_smem) {
+  const int q = gamma + 2 * qh;
   const int j0 = 2 * q;
   const uint32_t dg = half_bcast((uint16_t)(sb.d & 0xFFFFu));
   const uint32_t dg8 = half_bcast((uint16_t)(sb.d >> 16));
@@ -179,8 +182,8 @@ __device__ __forceinline__ void sb3_store(const Sb3SB& sb, int g, int p,
     uint32_t w[2][2][4];   // [lane][h][words]
 #pragma unroll
     for (int l = 0; l < 2; ++l) {
-      const uint32_t lo = u4_get(sb.lo[q >> 1][l], (j & 3));
-      const uint32_t hi = u4_get(sb.hi[l], q) >> (2 * jj);
+      const uint32_t lo = jj ? sb.lo[qh][l].y : sb.lo[qh][l].x;
+      const uint32_t hi = (qh ? sb.hi[l].y : sb.hi[l].x) >> (2 * jj);
       const uint32_t Q0 = (lo & 0x33333333u) | ((hi << 2) & 0x44444444u);
       const uint32_t Q1 = ((lo >> 2) & 0x33333333u) | ((hi << 1) & 0x44444444u);
       sb3_codes_to_h16(Q0, w[l][0]);
@@ -286,7 +289,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      mbar_init(&full_a[s], PF_NDQ);
+      mbar_init(&full_a[s], PF_NDQ / 2);   // the warps of one dequant group
       mbar_init(&full_b[s], 1);
       mbar_init(&empty[s], 1);
     }
@@ -395,36 +398,25 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
     }
   } else if (warp >= PF_WDQ0) {
     // ------------------------------------------ A operand dequant -----
-    const int t = threadIdx.x - PF_WDQ0 * 32;   // 0..255
-    constexpr int ITEMS = (SB3 ? 128 : 256) * NA;
-    constexpr int IPT = (ITEMS + 255) / 256;
+    // Two groups of four warps take alternate k-steps (group gamma the
+    // steps whose index in this CTA's sequence has parity gamma); each
+    // thread covers one (tile, g, p) position of every A tensor of the
+    // stage: rows g and g+8 (both row halves), columns 8p..8p+7 of each
+    // 16-column half of the stage's 64 columns.
+    const int gamma = (warp - PF_WDQ0) >> 2;
+    const int t = threadIdx.x - (PF_WDQ0 + 4 * gamma) * 32;   // 0..127
+    const int tg = t & 7, tp_ = (t >> 3) & 1, tti = t >> 4;
     const int tcols = SB3 ? SB3_TILE_COLS : B32_TILE_COLS;
     const int tbytes = SB3 ? SB3_TILE_BYTES : B32_TILE_BYTES;
     const int64_t trow_stride = (int64_t)(p.K / tcols) * tbytes;  // 16 rows
     const B32Tab tab = {p.tab[0], p.tab[1], p.tab[2], p.tab[3]};
-    // item geometry (fixed per thread)
-    int it_g[IPT], it_p[IPT], it_rh[IPT], it_ti[IPT], it_a[IPT];
-    bool it_on[IPT];
-#pragma unroll
-    for (int i = 0; i < IPT; ++i) {
-      const int item = t + 256 * i;
-      it_on[i] = item < ITEMS;
-      it_g[i] = item & 7;
-      it_p[i] = (item >> 3) & 1;
-      if (SB3) {
-        it_rh[i] = 0;
-        it_ti[i] = (item >> 4) & 7;
-        it_a[i] = item >> 7;
-      } else {
-        it_rh[i] = (item >> 4) & 1;
-        it_ti[i] = (item >> 5) & 7;
-        it_a[i] = item >> 8;
-      }
-    }
-    // prefetch position (unit, k-step) and its tile pointers
-    int pu = blockIdx.x, pks = 0;
-    const uint8_t* ptp[IPT];
-    auto set_unit = [&](int u) {
+    // tile pointers of the prefetch position's unit
+    const uint8_t* ptp[NA];
+    int pf_it = -1;
+    auto set_unit = [&](int it) {
+      pf_it = it;
+      const int u = blockIdx.x + it * gridDim.x;
+      if (u >= n_units) return;
       const int4 tile = p.tiles[u / MT];
       const int m = u % MT;
       const int e = tile.x;
@@ -435,98 +427,95 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
       }
       const uint8_t* blob = p.pool + bi * p.blob_stride;
 #pragma unroll
-      for (int i = 0; i < IPT; ++i)
-        ptp[i] = blob + (it_a[i] ? p.off_a1 : p.off_a0) +
-                 (int64_t)(m * (PF_BM / 16) + it_ti[i]) * trow_stride;
+      for (int a = 0; a < NA; ++a)
+        ptp[a] = blob + (a ? p.off_a1 : p.off_a0) +
+                 (int64_t)(m * (PF_BM / 16) + tti) * trow_stride;
     };
-    // One k-step: wait for the stage, write the A tile(s), publish.
-    uint32_t kstep = 0;
-    auto stage_begin = [&](uint32_t& st) -> bool {
-      const int s = (int)(kstep % S);
-      const uint32_t use = kstep / S;
+    auto stage_begin = [&](uint32_t ks_glob, uint32_t& st) -> bool {
+      const int s = (int)(ks_glob % S);
+      const uint32_t use = ks_glob / S;
       if (use > 0 && !mbar_wait(&empty[s], (use - 1) & 1, err)) return false;
       st = sbase + (uint32_t)(s * C::STAGE_BYTES);
       return true;
     };
-    auto stage_end = [&]() {
+    auto stage_end = [&](uint32_t ks_glob) {
       tc::fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&full_a[kstep % S]);
-      ++kstep;
+      if (lane == 0) mbar_arrive(&full_a[ks_glob % S]);
     };
-    if (pu < n_units) set_unit(pu);
+    const int n_my = (n_units - (int)blockIdx.x + (int)gridDim.x - 1) /
+                     (int)gridDim.x;   // units of this CTA
     bool ok = true;
     if constexpr (SB3) {
-      // super-block granularity (4 k-steps), prefetched one ahead
-      static_assert(IPT == 1, "one SB3 item per thread");
+      // super-block granularity (the group's two k-steps of it),
+      // prefetched one super-block ahead
       const int nsb = nk / 4;
-      auto fetch = [&](Sb3SB& q) {
-        if (pu >= n_units) return;
-        if (it_on[0])
-          sb3_load(ptp[0] + (int64_t)pks * SB3_TILE_BYTES, it_g[0], it_p[0], q);
-        if (++pks == nsb) {
-          pks = 0;
-          pu += gridDim.x;
-          if (pu < n_units) set_unit(pu);
-        }
+      const int total_sb = n_my * nsb;
+      int pf_sb = 0;
+      auto fetch = [&](Sb3Half (&q)[NA]) {
+        if (pf_sb >= total_sb) return;
+        const int it = pf_sb / nsb, sb = pf_sb % nsb;
+        if (it != pf_it) set_unit(it);
+#pragma unroll
+        for (int a = 0; a < NA; ++a)
+          sb3_load(ptp[a] + (int64_t)sb * SB3_TILE_BYTES, tg, tp_, gamma, q[a]);
+        ++pf_sb;
       };
-      Sb3SB cur, nxt;
+      Sb3Half cur[NA], nxt[NA];
       fetch(cur);
-      for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
-        for (int sb = 0; ok && sb < nsb; ++sb) {
-          fetch(nxt);
+      for (int gsb = 0; ok && gsb < total_sb; ++gsb) {
+        fetch(nxt);
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            uint32_t st;
-            if (!stage_begin(st)) {
-              ok = false;
-              break;
-            }
-            if (it_on[0])
-              sb3_store(cur, it_g[0], it_p[0], q, 16 * it_ti[0],
-                        st + it_a[0] * PF_A_BYTES);
-            stage_end();
-          }
-          cur = nxt;
-        }
-      }
-    } else {
-      // k-step granularity, prefetched two ahead
-      auto fetch = [&](B32Q (&q)[IPT]) {
-        if (pu >= n_units) return;
-#pragma unroll
-        for (int i = 0; i < IPT; ++i)
-          if (it_on[i])
-            q[i] = b32_load(ptp[i] + (int64_t)pks * B32_TILE_BYTES, it_g[i],
-                            it_p[i]);
-        if (++pks == nk) {
-          pks = 0;
-          pu += gridDim.x;
-          if (pu < n_units) set_unit(pu);
-        }
-      };
-      B32Q q0[IPT], q1[IPT], q2[IPT];
-      fetch(q0);
-      fetch(q1);
-      for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
-        for (int ks = 0; ks < nk; ++ks) {
-          fetch(q2);
+        for (int qh = 0; qh < 2; ++qh) {
+          const uint32_t ksg = (uint32_t)gsb * 4 + gamma + 2 * qh;
           uint32_t st;
-          if (!stage_begin(st)) {
+          if (!stage_begin(ksg, st)) {
             ok = false;
             break;
           }
 #pragma unroll
-          for (int i = 0; i < IPT; ++i)
-            if (it_on[i])
-              b32_store(q0[i], it_g[i], it_p[i], it_rh[i], 16 * it_ti[i], tab,
-                        st + it_a[i] * PF_A_BYTES);
-          stage_end();
+          for (int a = 0; a < NA; ++a)
+            sb3_store(cur[a], tg, tp_, gamma, qh, 16 * tti,
+                      st + a * PF_A_BYTES);
+          stage_end(ksg);
+        }
 #pragma unroll
-          for (int i = 0; i < IPT; ++i) {
-            q0[i] = q1[i];
-            q1[i] = q2[i];
-          }
+        for (int a = 0; a < NA; ++a) cur[a] = nxt[a];
+      }
+    } else {
+      // the group's k-steps, prefetched two of them ahead
+      const uint32_t total = (uint32_t)n_my * nk;
+      uint32_t pf_k = gamma;   // global k-step of the next fetch
+      auto fetch = [&](B32Q (&q)[NA]) {
+        if (pf_k >= total) return;
+        const int it = (int)(pf_k / nk), ks = (int)(pf_k % nk);
+        if (it != pf_it) set_unit(it);
+#pragma unroll
+        for (int a = 0; a < NA; ++a)
+          q[a] = b32_load(ptp[a] + (int64_t)ks * B32_TILE_BYTES, tg, tp_);
+        pf_k += 2;
+      };
+      B32Q q0[NA], q1[NA], q2[NA];
+      fetch(q0);
+      fetch(q1);
+      for (uint32_t ksg = gamma; ok && ksg < total; ksg += 2) {
+        fetch(q2);
+        uint32_t st;
+        if (!stage_begin(ksg, st)) {
+          ok = false;
+          break;
+        }
+#pragma unroll
+        for (int a = 0; a < NA; ++a)
+#pragma unroll
+          for (int rh = 0; rh < 2; ++rh)
+            b32_store(q0[a], tg, tp_, rh, 16 * tti, tab,
+                      st + a * PF_A_BYTES);
+        stage_end(ksg);
+#pragma unroll
+        for (int a = 0; a < NA; ++a) {
+          q0[a] = q1[a];
+          q1[a] = q2[a];
         }
       }
     }
@@ -623,31 +612,31 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
 }
 
 // ---------------------------------------------------- plan and inputs ---
-// Unit list: token tiles of <= 256 grouped rows per expert; all full tiles
-// first (expert order), then the partial tiles by descending size in
-// 16-row buckets (expert order inside a bucket).
+// Unit list.  Expert e's cnt grouped rows are cut into nt = ceil(cnt/256)
+// tiles of nearly equal size in whole 16-row blocks (so no expert leaves a
+// small remainder tile; the last tile holds the partial block), and the
+// tiles are ordered by size in 16-row blocks, largest first; one expert's
+// tiles of one size stay contiguous.  The order inside a size class
+// depends on atomics; every unit writes its own outputs, so results do
+// not depend on it.
 __global__ void __launch_bounds__(1024)
     pf_plan_kernel(const int32_t* __restrict__ offsets, int E,
                    int4* __restrict__ tiles, int32_t* __restrict__ n_tiles) {
-  __shared__ int32_t first[EMAX + 1];
-  __shared__ int32_t tmp[32];
-  __shared__ int32_t hist[17], base[17];
+  __shared__ int32_t hist[18], base[18];
   const int tid = threadIdx.x;
-  if (tid < 17) hist[tid] = 0;
-  for (int e = tid; e <= E; e += blockDim.x)
-    first[e] = e < E ? (offsets[e + 1] - offsets[e]) / PF_BN : 0;
+  if (tid < 18) hist[tid] = 0;
   __syncthreads();
-  const int nfull = block_exclusive_scan(first, E + 1, tmp);
   for (int e = tid; e < E; e += blockDim.x) {
-    const int o = offsets[e], cnt = offsets[e + 1] - o;
-    const int nf = cnt / PF_BN, rem = cnt % PF_BN;
-    for (int i = 0; i < nf; ++i)
-      tiles[first[e] + i] = make_int4(e, o + i * PF_BN, PF_BN, 0);
-    if (rem) atomicAdd(&hist[(rem + 15) >> 4], 1);
+    const int cnt = offsets[e + 1] - offsets[e];
+    if (!cnt) continue;
+    const int nb = (cnt + 15) >> 4, nt = (nb + 15) >> 4;
+    const int q = nb / nt, r = nb % nt;   // r tiles of q+1 blocks, rest q
+    if (r) atomicAdd(&hist[q + 1], r);
+    atomicAdd(&hist[q], nt - r);
   }
   __syncthreads();
   if (tid == 0) {
-    int b0 = nfull;
+    int b0 = 0;
     for (int b = 16; b >= 1; --b) {
       base[b] = b0;
       b0 += hist[b];
@@ -655,24 +644,20 @@ __global__ void __launch_bounds__(1024)
     *n_tiles = b0;
   }
   __syncthreads();
-  if (tid < 32) {
-    for (int e0 = 0; e0 < E; e0 += 32) {
-      const int e = e0 + tid;
-      int rem = 0, o = 0;
-      if (e < E) {
-        o = offsets[e];
-        rem = (offsets[e + 1] - o) % PF_BN;
-      }
-      const int b = rem ? (rem + 15) >> 4 : 0;
-      const unsigned m = __match_any_sync(0xffffffffu, b);
-      const int rank = __popc(m & ((1u << tid) - 1u));
-      if (b) {
-        const int cnt = offsets[e + 1] - o;
-        tiles[base[b] + rank] = make_int4(e, o + cnt - rem, rem, 0);
-      }
-      __syncwarp();
-      if (b && rank == 0) base[b] += __popc(m);
-      __syncwarp();
+  for (int e = tid; e < E; e += blockDim.x) {
+    const int o = offsets[e], cnt = offsets[e + 1] - o;
+    if (!cnt) continue;
+    const int nb = (cnt + 15) >> 4, nt = (nb + 15) >> 4;
+    const int q = nb / nt, r = nb % nt;
+    int p1 = 0, p0;
+    if (r) p1 = atomicAdd(&base[q + 1], r);
+    p0 = atomicAdd(&base[q], nt - r);
+    int row = o;
+    for (int i = 0; i < nt; ++i) {
+      const int blocks = i < r ? q + 1 : q;
+      const int rows = min(16 * blocks, o + cnt - row);
+      tiles[i < r ? p1 + i : p0 + (i - r)] = make_int4(e, row, rows, 0);
+      row += rows;
     }
   }
 }
