@@ -9,12 +9,15 @@
 //          h = silu(g) * u  -> fp16, grouped row order
 //   down : y = W_down[128 rows x F] . h[tokens]^T -> fp32 rows of y_pairs
 // Warp roles inside the CTA:
-//   warps 0-3   epilogue: TMEM -> registers -> global (TMEM lane quadrants)
-//   warp  4     TMEM owner; lane 0 issues tcgen05.mma and the commits
-//   warp  5     B operand: TMA copies of 16-row boxes of activations in
+//   warps 0..E-1  epilogue: TMEM -> registers -> global (warp w reads TMEM
+//                 lane quadrant w % 4; with E = 8 (up/gate, whose single
+//                 accumulator buffer makes the epilogue stall the MMAs)
+//                 warp w / 4 takes every other 32 columns)
+//   warp  E     TMEM owner; lane 0 issues tcgen05.mma and the commits
+//   warp  E+1   B operand: TMA copies of 16-row boxes of activations in
 //               grouped row order (up: x gathered to fp16 by a pre-pass;
 //               down: h as the up/gate epilogue wrote it)
-//   warps 6-13  A operand: quantised tiles -> fp16 in shared memory
+//   warps E+2.. A operand: quantised tiles -> fp16 in shared memory (8)
 // Operands are K-major fp16 with the 128-byte swizzle, accumulators fp32 in
 // tensor memory.  The A tiles hold the round-to-nearest-even fp16 value of
 // each dequantised weight (d * (2s+1) * c / 8 or d * cb[q], formed with
@@ -33,21 +36,22 @@ namespace {
 constexpr int PF_BM = 128;   // weight rows per unit (MMA M)
 constexpr int PF_BK = 64;    // K per pipeline stage (one swizzle row)
 constexpr int PF_BN = 256;   // token rows per unit at most (MMA N)
-constexpr int PF_EPI = 4;    // epilogue warps
-constexpr int PF_WMMA = 4, PF_WLOAD = 5, PF_WDQ0 = 6, PF_NDQ = 8;
-constexpr int PF_THREADS = (PF_WDQ0 + PF_NDQ) * 32;   // 448
+constexpr int PF_NDQ = 8;    // dequant warps
 constexpr int PF_A_BYTES = PF_BM * PF_BK * 2;         // 16 KB
 constexpr int PF_B_BYTES = PF_BN * PF_BK * 2;         // 32 KB
 constexpr int PF_TMEM_COLS = 512;
 
 template <bool UP>
 struct PfCfg {
+  static constexpr int EPI = UP ? 8 : 4;           // epilogue warps
+  static constexpr int WMMA = EPI, WLOAD = EPI + 1, WDQ0 = EPI + 2;
+  static constexpr int THREADS = (WDQ0 + PF_NDQ) * 32;
   static constexpr int NA = UP ? 2 : 1;            // A tensors per unit
   static constexpr int STAGES = UP ? 3 : 4;
   static constexpr int STAGE_BYTES = NA * PF_A_BYTES + PF_B_BYTES;
   static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
   static constexpr int META_OFF = BAR_OFF + 256;   // epilogue row metadata
-  static constexpr int META_BYTES = PF_EPI * PF_BN * 4;
+  static constexpr int META_BYTES = EPI * PF_BN * 4;
   static constexpr int SMEM = META_OFF + META_BYTES + 1024;   // + alignment
 };
 
@@ -85,6 +89,11 @@ __device__ __forceinline__ uint32_t hsub2u(uint32_t a, uint32_t b) {
   __half2 r = __hsub2(*reinterpret_cast<__half2*>(&a),
                       *reinterpret_cast<__half2*>(&b));
   return *reinterpret_cast<uint32_t*>(&r);
+}
+__device__ __forceinline__ float tanh_approx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 __device__ __forceinline__ uint32_t half_bcast(uint16_t h) {
   return (uint32_t)h | ((uint32_t)h << 16);
@@ -270,7 +279,7 @@ __device__ __forceinline__ void b32_store(const B32Q& q, int g, int p,
 // maps: up: x_g [P][H], down: h16 [P][F], both fp16 in grouped row
 // order, boxes of 64 columns, 128-byte swizzle.
 template <bool UP, bool SB3>
-__global__ void __launch_bounds__(PF_THREADS, 1)
+__global__ void __launch_bounds__(PfCfg<UP>::THREADS, 1)
     pf_gemm_kernel(const PfParams p, const __grid_constant__ PfMaps maps) {
   using C = PfCfg<UP>;
   constexpr int NA = C::NA, S = C::STAGES;
@@ -295,12 +304,12 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], PF_EPI);
+      mbar_init(&acc_empty[b], C::EPI);
     }
     mbar_init(drain, 1);
     fence_mbar_init();
   }
-  if (warp == PF_WMMA) {
+  if (warp == C::WMMA) {
     tc::tmem_alloc(tmem_slot, PF_TMEM_COLS);
     tc::tmem_relinquish();
   }
@@ -314,7 +323,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
   const int n_units = *p.n_tiles * MT;
   int32_t* err = p.err;
 
-  if (warp == PF_WMMA) {
+  if (warp == C::WMMA) {
     // ------------------------------------------------ MMA issuer ------
     if (lane == 0) {
       uint32_t kstep = 0;
@@ -360,7 +369,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
       tc::commit(drain);
       mbar_wait(drain, 0, err);
     }
-  } else if (warp == PF_WLOAD) {
+  } else if (warp == C::WLOAD) {
     // ------------------------------------------- B operand loader -----
     // Lane 0 issues the TMA copies of every k-step: the unit's grouped
     // rows in boxes of 256/128/64/32/16 rows; rows past the tile (up to the
@@ -396,15 +405,15 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         }
       }
     }
-  } else if (warp >= PF_WDQ0) {
+  } else if (warp >= C::WDQ0) {
     // ------------------------------------------ A operand dequant -----
     // Two groups of four warps take alternate k-steps (group gamma the
     // steps whose index in this CTA's sequence has parity gamma); each
     // thread covers one (tile, g, p) position of every A tensor of the
     // stage: rows g and g+8 (both row halves), columns 8p..8p+7 of each
     // 16-column half of the stage's 64 columns.
-    const int gamma = (warp - PF_WDQ0) >> 2;
-    const int t = threadIdx.x - (PF_WDQ0 + 4 * gamma) * 32;   // 0..127
+    const int gamma = (warp - C::WDQ0) >> 2;
+    const int t = threadIdx.x - (C::WDQ0 + 4 * gamma) * 32;   // 0..127
     const int tg = t & 7, tp_ = (t >> 3) & 1, tti = t >> 4;
     const int tcols = SB3 ? SB3_TILE_COLS : B32_TILE_COLS;
     const int tbytes = SB3 ? SB3_TILE_BYTES : B32_TILE_BYTES;
@@ -525,7 +534,9 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
     // pair id) goes to this warp's slice of shared memory before the
     // accumulator wait, so its global latency overlaps the MMAs.
     int it = 0;
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const int quad = warp & 3, chalf = warp >> 2;
+    constexpr int CSTEP = 32 * (C::EPI / 4);   // column stride of a warp
+    const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
     float* meta_f = reinterpret_cast<float*>(smem + C::META_OFF) + warp * PF_BN;
     int32_t* meta_i = reinterpret_cast<int32_t*>(meta_f);
     for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++it) {
@@ -533,7 +544,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
       const int nlen = tile.z, row0 = tile.y;
       const int ab = UP ? 0 : (it & 1);
       __syncwarp();
-      for (int n = lane; n < ((nlen + 31) & ~31); n += 32) {
+      for (int n = 32 * chalf + lane; n < ((nlen + 31) & ~31); n += CSTEP) {
         if constexpr (UP)
           meta_f[n] = n < nlen ? p.xscale[row0 + n] : 1.f;
         else
@@ -543,13 +554,13 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
       const int use_ab = UP ? it : (it >> 1);
       if (!mbar_wait(&acc_full[ab], use_ab & 1, err)) break;
       tc::fence_after_sync();
-      const int col = (u % MT) * PF_BM + warp * 32 + lane;  // output column
+      const int col = (u % MT) * PF_BM + quad * 32 + lane;  // output column
       // Each 32-column chunk reads its metadata into registers first, so
       // no shared-memory load waits behind a global store.
       if constexpr (UP) {
         float hmax = 0.f;
         __half* hp = p.h16 + (int64_t)row0 * p.rows + col;
-        for (int c0 = 0; c0 < nlen; c0 += 32) {
+        for (int c0 = 32 * chalf; c0 < nlen; c0 += CSTEP) {
           float ua[32], ga[32], sc[32];
           tc::ld_32x32b_x16(tmem + lane_base + (uint32_t)c0, *(float(*)[16])&ua[0]);
           tc::ld_32x32b_x16(tmem + lane_base + (uint32_t)(c0 + 16),
@@ -564,22 +575,33 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
             sc[i] = v.x; sc[i + 1] = v.y; sc[i + 2] = v.z; sc[i + 3] = v.w;
           }
           tc::wait_ld();
-          __half hv16[32];
+          // silu(g) u = g u (1 + tanh(g/2)) / 2, one hardware tanh each
+          __half2 hv2[16];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float uu = ua[i] * sc[i], gg = ga[i] * sc[i];
-            const float hv = __fdividef(gg, 1.0f + __expf(-gg)) * uu;
-            if (c0 + i < nlen) hmax = fmaxf(hmax, fabsf(hv));
-            hv16[i] = __float2half_rn(hv);
+          for (int i = 0; i < 32; i += 2) {
+            float hv[2];
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+              const float uu = ua[i + j] * sc[i + j];
+              const float gg = ga[i + j] * sc[i + j];
+              const float th = tanh_approx(0.5f * gg);
+              hv[j] = (0.5f * gg * uu) * (1.0f + th);
+              if (c0 + i + j < nlen) hmax = fmaxf(hmax, fabsf(hv[j]));
+            }
+            hv2[i / 2] = __floats2half2_rn(hv[0], hv[1]);
           }
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (c0 + i < nlen) hp[(int64_t)(c0 + i) * p.rows] = hv16[i];
+          for (int i = 0; i < 32; i += 2) {
+            if (c0 + i < nlen)
+              hp[(int64_t)(c0 + i) * p.rows] = __low2half(hv2[i / 2]);
+            if (c0 + i + 1 < nlen)
+              hp[(int64_t)(c0 + i + 1) * p.rows] = __high2half(hv2[i / 2]);
+          }
         }
         if (!(hmax < 65520.f)) set_err(err, MOE_ERR_DEVICE);   // fp16 range
       } else {
         float* yp = p.y + col;
-        for (int c0 = 0; c0 < nlen; c0 += 32) {
+        for (int c0 = 32 * chalf; c0 < nlen; c0 += CSTEP) {
           float acc[32];
           int pr[32];
           tc::ld_32x32b_x16(tmem + lane_base + (uint32_t)(ab * 256 + c0),
@@ -605,7 +627,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
 
   tc::fence_before_sync();
   __syncthreads();
-  if (warp == PF_WMMA) {
+  if (warp == C::WMMA) {
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, PF_TMEM_COLS);
   }
@@ -774,7 +796,7 @@ static moe_status pf_launch(const PfParams& prm, const PfMaps& map,
   moe_status st = ensure_smem(fn, PfCfg<UP>::SMEM);
   if (st != MOE_OK) return st;
   pf_gemm_kernel<UP, SB3>
-      <<<num_sms(), PF_THREADS, PfCfg<UP>::SMEM, s>>>(prm, map);
+      <<<num_sms(), PfCfg<UP>::THREADS, PfCfg<UP>::SMEM, s>>>(prm, map);
   return launch_status();
 }
 
