@@ -108,10 +108,14 @@ moe_status moe_dequant(int fmt, const uint8_t* packed, int rows, int cols,
 /* Router and top-k ("Avalon": 512 experts, 10 active; softmax over all E,
  * top-k by probability with ties to the lower index, renormalised).
  *   x        bf16 [T x H] row-major        w_router bf16 [E x H] row-major
+ *            (both 16-byte aligned, else MOE_ERR_INVALID)
  *   bias     fp32 [E] added to the logits, or NULL
  *   topk_idx int32 [T x k]: experts by descending weight
  *   topk_w   fp32 [T x k]: renormalised softmax weights (sum to 1)
- *   logits_out fp32 [T x E] (the fp32 logits the selection used), or NULL
+ *   logits_out fp32 [T x E]: receives the fp32 logits the selection used;
+ *            required (NULL returns MOE_ERR_WORKSPACE)
+ * Logits: exact bf16 products, fp32 accumulation, one fp32 bias add; for
+ * T > 8 and H % 64 == 0 on the 5th-generation tensor cores.
  * Needs 1 <= k <= min(E, 32), E <= 4096, H % 8 == 0. */
 moe_status moe_route_topk(const uint16_t* x, int T, int H,
                           const uint16_t* w_router, int E, const float* bias,
@@ -199,10 +203,21 @@ moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream);
 /* Expert FFN on the grouped pairs: for every pair p of expert e,
  *   h = silu(Wg_e x_t) * (Wu_e x_t),  y_pairs[p] = Wd_e h
  * with the weights dequantised inside the kernel.
- *   x          bf16 [T x H];  y_pairs fp32 [T*k x H] (row p = pair p)
+ *   x          bf16 [T x H], 16-byte aligned (else MOE_ERR_INVALID);
+ *              y_pairs fp32 [T*k x H] (row p = pair p)
  *   expert_offsets/pair_ids/active/n_active: moe_group_tokens' outputs
- *   blob_index int32 [E] or NULL (NULL: expert e's blob is blob e)
- * Needs H, F multiples of 256 (SB3) or 64 (Q4/NL4) and of 16. */
+ *   blob_index int32 [E] or NULL (NULL: expert e's blob is blob e); a
+ *              negative entry of a chosen expert sets MOE_ERR_DEVICE
+ * Needs H, F multiples of 256 (SB3) or 64 (Q4/NL4) and of 16.
+ * T <= 8: exact int8 tensor-core decode kernels (activations split into
+ *   int8 halves, fp32 scale folds).
+ * T > 8 with H, F multiples of 128 (the prefill path): grouped GEMMs on the
+ *   5th-generation tensor cores in fp16 with fp32 accumulation.  Each
+ *   weight enters as the round-to-nearest fp16 of its exact value, each
+ *   activation row as fp16 after a per-row power-of-two scale that keeps
+ *   it below 2^15, and h = silu(g) u is kept as fp16 (silu formed with the
+ *   hardware tanh); an |h| beyond the fp16 range sets MOE_ERR_DEVICE.
+ * Other shapes: a general SIMT path. */
 moe_status moe_expert_ffn_q(const moe_layer_desc* desc, const uint16_t* x,
                             int T, int k, const int32_t* expert_offsets,
                             const int32_t* pair_ids, const int32_t* active,
