@@ -293,6 +293,49 @@ moe_status moe_layer_forward(const moe_layer_desc* desc, const uint16_t* x,
                              float* topk_w, float* logits_out, void* ws,
                              size_t ws_bytes, void* stream);
 
+/* ------------------------------------------- pre-norm residual stack ---- */
+
+/* One layer of the 48-layer decode stack ("Avalon": 48 layers of 512
+ * experts, top-10) with the residual add between layers:
+ *   x = bf16(rmsnorm(r)) per row (eps 1e-6, no learned weight),
+ *   r_out = r + MoE(x)            (r_out may alias r: in place)
+ * r fp32 [T x H], 16-byte aligned; the other arguments as in
+ * moe_layer_forward (w_router, bias, blob_index, topk_idx, topk_w,
+ * logits_out or NULL, out_bf16 = bf16 copy of r_out or NULL).  Workspace:
+ * moe_layer_workspace_bytes.  T <= 8: one kernel. */
+moe_status moe_layer_forward_residual(const moe_layer_desc* desc,
+                                      const float* r, int T, int k,
+                                      const uint16_t* w_router,
+                                      const float* bias,
+                                      const int32_t* blob_index, float* r_out,
+                                      uint16_t* out_bf16, int32_t* topk_idx,
+                                      float* topk_w, float* logits_out,
+                                      void* ws, size_t ws_bytes,
+                                      void* stream);
+
+/* The same layer in two halves, for callers that act between routing and
+ * the expert FFN -- the expert-slot cache ("Betelgeuse": resolve on the
+ * device, copy only the misses, then compute; offloaded and resident runs
+ * agree bit for bit):
+ *   moe_layer_route_residual: x = bf16(rmsnorm(r)), logits, top-k ->
+ *     topk_idx [T x k], topk_w [T x k] (and logits_out or NULL).
+ *   moe_layer_ffn_residual: r_out = r + sum_j topk_w * FFN_{topk_idx}(x)
+ *     with expert e read from pool + blob_index[e] * stride.
+ * route then ffn on the same stream and workspace gives bit-for-bit the
+ * result of moe_layer_forward_residual with the same blob contents. */
+moe_status moe_layer_route_residual(const moe_layer_desc* desc,
+                                    const float* r, int T, int k,
+                                    const uint16_t* w_router,
+                                    const float* bias, int32_t* topk_idx,
+                                    float* topk_w, float* logits_out,
+                                    void* ws, size_t ws_bytes, void* stream);
+moe_status moe_layer_ffn_residual(const moe_layer_desc* desc, const float* r,
+                                  int T, int k, const int32_t* topk_idx,
+                                  const float* topk_w,
+                                  const int32_t* blob_index, float* r_out,
+                                  uint16_t* out_bf16, void* ws,
+                                  size_t ws_bytes, void* stream);
+
 /* Synchronise `stream`, read the FFN/grouping workspace's device error word
  * into *host_err (host pointer, may be NULL) and clear it.  Returns
  * MOE_ERR_DEVICE if it was set, MOE_OK otherwise. */

@@ -75,6 +75,13 @@ _SIGS = {
                                              c_int]),
     "moe_layer_forward": (c_int, [_P, _P, c_int, c_int, _P, _P, _P, _P, _P,
                                   _P, _P, _P, _P, _P, c_size_t, _P]),
+    "moe_layer_forward_residual": (c_int, [_P, _P, c_int, c_int, _P, _P, _P,
+                                           _P, _P, _P, _P, _P, _P, c_size_t,
+                                           _P]),
+    "moe_layer_route_residual": (c_int, [_P, _P, c_int, c_int, _P, _P, _P,
+                                         _P, _P, _P, c_size_t, _P]),
+    "moe_layer_ffn_residual": (c_int, [_P, _P, c_int, c_int, _P, _P, _P, _P,
+                                       _P, _P, c_size_t, _P]),
     "moe_get_device_status": (c_int, [_P, _P, _P]),
     "moe_status_string": (ctypes.c_char_p, [c_int]),
 }
@@ -247,6 +254,31 @@ def moe_layer_forward(desc, x, T, k, w_router, bias, blob_index, residual,
         _ptr(desc), _ptr(x), T, k, _ptr(w_router), _ptr(bias),
         _ptr(blob_index), _ptr(residual), _ptr(out), _ptr(out_bf16),
         _ptr(topk_idx), _ptr(topk_w), _ptr(logits_out), _ptr(ws), ws_bytes,
+        _stream(stream)))
+
+
+def moe_layer_forward_residual(desc, r, T, k, w_router, bias, blob_index,
+                               r_out, out_bf16, topk_idx, topk_w, logits_out,
+                               ws, ws_bytes, stream=None):
+    _check("moe_layer_forward_residual", lib.moe_layer_forward_residual(
+        _ptr(desc), _ptr(r), T, k, _ptr(w_router), _ptr(bias),
+        _ptr(blob_index), _ptr(r_out), _ptr(out_bf16), _ptr(topk_idx),
+        _ptr(topk_w), _ptr(logits_out), _ptr(ws), ws_bytes, _stream(stream)))
+
+
+def moe_layer_route_residual(desc, r, T, k, w_router, bias, topk_idx, topk_w,
+                             logits_out, ws, ws_bytes, stream=None):
+    _check("moe_layer_route_residual", lib.moe_layer_route_residual(
+        _ptr(desc), _ptr(r), T, k, _ptr(w_router), _ptr(bias),
+        _ptr(topk_idx), _ptr(topk_w), _ptr(logits_out), _ptr(ws), ws_bytes,
+        _stream(stream)))
+
+
+def moe_layer_ffn_residual(desc, r, T, k, topk_idx, topk_w, blob_index,
+                           r_out, out_bf16, ws, ws_bytes, stream=None):
+    _check("moe_layer_ffn_residual", lib.moe_layer_ffn_residual(
+        _ptr(desc), _ptr(r), T, k, _ptr(topk_idx), _ptr(topk_w),
+        _ptr(blob_index), _ptr(r_out), _ptr(out_bf16), _ptr(ws), ws_bytes,
         _stream(stream)))
 
 

@@ -62,7 +62,9 @@ moe_status launch_decode_layer(const moe_layer_desc& d, const uint16_t* x,
                                const float* residual, float* out,
                                uint16_t* out_bf16, int32_t* topk_idx,
                                float* topk_w, float* logits, void* ws,
-                               int32_t* err, cudaStream_t s);
+                               int32_t* err, cudaStream_t s, int mode);
+moe_status launch_rmsnorm_bf16(const float* r, int T, int H, uint16_t* x,
+                               cudaStream_t s);
 
 int num_sms() {
   static int cached[64] = {0};
@@ -170,6 +172,7 @@ struct LayerWs {
   int32_t* active;
   int32_t* n_active;
   int32_t* grp;
+  uint16_t* xr;      // bf16 [T][H]: rmsnorm of the residual (T > 8)
   size_t bytes;
 };
 
@@ -187,6 +190,7 @@ static LayerWs carve_layer_ws(void* base, int T, int k, int E, int H, int F) {
   const size_t gr = c.take(group_ws_bytes(T, k, E));
   const size_t fu = c.take(T <= DEC_TMAX ? decode_layer_ws_bytes(T, k, H, F)
                                          : 0);
+  const size_t xr = c.take(T <= DEC_TMAX ? 0 : (size_t)T * H * 2);
   uint8_t* b = static_cast<uint8_t*>(base);
   w.fused = base ? static_cast<void*>(b + fu) : nullptr;
   w.logits = base ? reinterpret_cast<float*>(b + lo) : nullptr;
@@ -195,6 +199,7 @@ static LayerWs carve_layer_ws(void* base, int T, int k, int E, int H, int F) {
   w.active = base ? reinterpret_cast<int32_t*>(b + ac) : nullptr;
   w.n_active = base ? reinterpret_cast<int32_t*>(b + na) : nullptr;
   w.grp = base ? reinterpret_cast<int32_t*>(b + gr) : nullptr;
+  w.xr = base ? reinterpret_cast<uint16_t*>(b + xr) : nullptr;
   w.bytes = c.off;
   return w;
 }
@@ -432,7 +437,7 @@ extern "C" moe_status moe_layer_forward(
   if (decode_layer_supported(*desc, T, k))
     return launch_decode_layer(*desc, x, nullptr, T, k, w_router, bias,
                                blob_index, residual, out, out_bf16, topk_idx,
-                               topk_w, logits, w.fused, w.ffn.err, s);
+                               topk_w, logits, w.fused, w.ffn.err, s, DL_FULL);
   st = launch_route(x, T, desc->H, w_router, desc->E, bias, k, topk_idx,
                     topk_w, logits, w.ffn.err, s);
   if (st != MOE_OK) return st;
@@ -445,6 +450,109 @@ extern "C" moe_status moe_layer_forward(
   return run_down(*desc, T, k, w.offsets, w.pair_ids, w.active, w.n_active,
                   blob_index, w.ffn, nullptr, topk_w, residual, out, out_bf16,
                   s, true);
+}
+
+// ------------------------------------------------ pre-norm residual stack
+// One layer of the residual stack: x = bf16(rmsnorm(r)), r_out = r + MoE(x),
+// as one call or as its routing and FFN halves.
+
+static moe_status check_residual_args(const moe_layer_desc* desc,
+                                      const float* r, int T, int k,
+                                      void* ws, size_t ws_bytes,
+                                      LayerWs* w) {
+  moe_status st = check_desc(desc);
+  if (st != MOE_OK) return st;
+  if (!r) return MOE_ERR_INVALID;
+  if (T <= 0 || k < 1 || k > 32 || k > desc->E) return MOE_ERR_SHAPE;
+  if (desc->H % 8 || ((uintptr_t)r % 16)) return MOE_ERR_INVALID;
+  if (!ws) return MOE_ERR_WORKSPACE;
+  *w = carve_layer_ws(ws, T, k, desc->E, desc->H, desc->F);
+  if (ws_bytes < w->bytes) return MOE_ERR_WORKSPACE;
+  return MOE_OK;
+}
+
+extern "C" moe_status moe_layer_forward_residual(
+    const moe_layer_desc* desc, const float* r, int T, int k,
+    const uint16_t* w_router, const float* bias, const int32_t* blob_index,
+    float* r_out, uint16_t* out_bf16, int32_t* topk_idx, float* topk_w,
+    float* logits_out, void* ws, size_t ws_bytes, void* stream) {
+  LayerWs w;
+  moe_status st = check_residual_args(desc, r, T, k, ws, ws_bytes, &w);
+  if (st != MOE_OK) return st;
+  if (!w_router || !r_out || !topk_idx || !topk_w) return MOE_ERR_INVALID;
+  if ((uintptr_t)w_router % 16) return MOE_ERR_INVALID;
+  cudaStream_t s = (cudaStream_t)stream;
+  float* logits = logits_out ? logits_out : w.logits;
+  if (decode_layer_supported(*desc, T, k))
+    return launch_decode_layer(*desc, nullptr, r, T, k, w_router, bias,
+                               blob_index, r, r_out, out_bf16, topk_idx,
+                               topk_w, logits, w.fused, w.ffn.err, s, DL_FULL);
+  st = launch_rmsnorm_bf16(r, T, desc->H, w.xr, s);
+  if (st != MOE_OK) return st;
+  st = launch_route(w.xr, T, desc->H, w_router, desc->E, bias, k, topk_idx,
+                    topk_w, logits, w.ffn.err, s);
+  if (st != MOE_OK) return st;
+  st = launch_group(topk_idx, T, k, desc->E, w.offsets, w.pair_ids, w.active,
+                    w.n_active, w.grp, w.ffn.err, s);
+  if (st != MOE_OK) return st;
+  st = run_up(*desc, w.xr, T, k, w.offsets, w.pair_ids, w.active, w.n_active,
+              blob_index, w.ffn, s, true);
+  if (st != MOE_OK) return st;
+  return run_down(*desc, T, k, w.offsets, w.pair_ids, w.active, w.n_active,
+                  blob_index, w.ffn, nullptr, topk_w, r, r_out, out_bf16, s,
+                  true);
+}
+
+extern "C" moe_status moe_layer_route_residual(
+    const moe_layer_desc* desc, const float* r, int T, int k,
+    const uint16_t* w_router, const float* bias, int32_t* topk_idx,
+    float* topk_w, float* logits_out, void* ws, size_t ws_bytes,
+    void* stream) {
+  LayerWs w;
+  moe_status st = check_residual_args(desc, r, T, k, ws, ws_bytes, &w);
+  if (st != MOE_OK) return st;
+  if (!w_router || !topk_idx || !topk_w) return MOE_ERR_INVALID;
+  if ((uintptr_t)w_router % 16) return MOE_ERR_INVALID;
+  cudaStream_t s = (cudaStream_t)stream;
+  float* logits = logits_out ? logits_out : w.logits;
+  if (decode_layer_supported(*desc, T, k))
+    return launch_decode_layer(*desc, nullptr, r, T, k, w_router, bias,
+                               nullptr, nullptr, nullptr, nullptr, topk_idx,
+                               topk_w, logits, w.fused, w.ffn.err, s,
+                               DL_ROUTE);
+  st = launch_rmsnorm_bf16(r, T, desc->H, w.xr, s);
+  if (st != MOE_OK) return st;
+  return launch_route(w.xr, T, desc->H, w_router, desc->E, bias, k, topk_idx,
+                      topk_w, logits, w.ffn.err, s);
+}
+
+extern "C" moe_status moe_layer_ffn_residual(
+    const moe_layer_desc* desc, const float* r, int T, int k,
+    const int32_t* topk_idx, const float* topk_w, const int32_t* blob_index,
+    float* r_out, uint16_t* out_bf16, void* ws, size_t ws_bytes,
+    void* stream) {
+  LayerWs w;
+  moe_status st = check_residual_args(desc, r, T, k, ws, ws_bytes, &w);
+  if (st != MOE_OK) return st;
+  if (!r_out || !topk_idx || !topk_w) return MOE_ERR_INVALID;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (decode_layer_supported(*desc, T, k))
+    return launch_decode_layer(*desc, nullptr, r, T, k, nullptr, nullptr,
+                               blob_index, r, r_out, out_bf16,
+                               const_cast<int32_t*>(topk_idx),
+                               const_cast<float*>(topk_w), w.logits, w.fused,
+                               w.ffn.err, s, DL_FFN);
+  st = launch_rmsnorm_bf16(r, T, desc->H, w.xr, s);
+  if (st != MOE_OK) return st;
+  st = launch_group(topk_idx, T, k, desc->E, w.offsets, w.pair_ids, w.active,
+                    w.n_active, w.grp, w.ffn.err, s);
+  if (st != MOE_OK) return st;
+  st = run_up(*desc, w.xr, T, k, w.offsets, w.pair_ids, w.active, w.n_active,
+              blob_index, w.ffn, s, true);
+  if (st != MOE_OK) return st;
+  return run_down(*desc, T, k, w.offsets, w.pair_ids, w.active, w.n_active,
+                  blob_index, w.ffn, nullptr, topk_w, r, r_out, out_bf16, s,
+                  true);
 }
 
 extern "C" moe_status moe_get_device_status(void* ws, int32_t* host_err,

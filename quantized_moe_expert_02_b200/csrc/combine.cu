@@ -52,6 +52,12 @@ moe_status launch_combine(const float* y, const float* w, int T, int k,
   return launch_status();
 }
 
+moe_status launch_rmsnorm_bf16(const float* r, int T, int H, uint16_t* x,
+                               cudaStream_t s) {
+  rmsnorm_bf16_kernel<<<T, 256, 0, s>>>(r, H, x);
+  return launch_status();
+}
+
 }  // namespace moe
 
 using namespace moe;
@@ -70,6 +76,5 @@ extern "C" moe_status moe_rmsnorm_bf16(const float* r, int T, int H,
                                        uint16_t* x_out, void* stream) {
   if (!r || !x_out) return MOE_ERR_INVALID;
   if (T <= 0 || H <= 0) return MOE_ERR_SHAPE;
-  rmsnorm_bf16_kernel<<<T, 256, 0, (cudaStream_t)stream>>>(r, H, x_out);
-  return launch_status();
+  return launch_rmsnorm_bf16(r, T, H, x_out, (cudaStream_t)stream);
 }

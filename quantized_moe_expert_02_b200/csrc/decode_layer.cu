@@ -73,7 +73,10 @@ struct LayerParams {
   int32_t* bar;            // ws [2]: grid barrier, exit counter
   int32_t* up_done;        // ws [MAXP]: finished up units per expert
   int32_t* err;
+  int mode;                // DL_FULL, DL_ROUTE (P0-P1 top-k only) or
+                           // DL_FFN (top-k read from topk_idx/topk_w)
 };
+
 
 struct Smem {  // offsets into dynamic shared memory
   int slot_bytes, ring, frag, red, misc, total;
@@ -246,11 +249,12 @@ __global__ void __launch_bounds__(LAYER_THREADS, 1)
   if (blockIdx.x == 0)
     for (int i = tid; i < T * k; i += LAYER_THREADS) p.hmax[i] = 0u;
   __syncthreads();
-  // router rows of this block: four warps per row, each a quarter of H;
+  // router rows of this block (not in DL_FFN): four warps per row, each a
+  // quarter of H;
   // a lane issues all its loads of the row first (up to RCH 16-byte
   // chunks), then accumulates in fp32; lane sums by a fixed butterfly and
   // the quarters in fixed order (deterministic)
-  {
+  if (p.mode != DL_FFN) {
     constexpr int RQ = 4, RCH = 4;
     float* part = reinterpret_cast<float*>(smem + L.red);   // [rows][RQ][T]
     const int e0 = (int)((int64_t)E * blockIdx.x / G);
@@ -383,7 +387,14 @@ __global__ void __launch_bounds__(LAYER_THREADS, 1)
         reinterpret_cast<uint2*>(frag)[i] = wv;
       }
     }
-    if (warp < T) {
+    if (warp < T && p.mode == DL_FFN) {
+      // the caller's top-k (as a DL_ROUTE launch wrote it)
+      const int t = warp;
+      if (lane < k) {
+        M.tk_idx[t * k + lane] = p.topk_idx[t * k + lane];
+        M.tk_w[t * k + lane] = p.topk_w[t * k + lane];
+      }
+    } else if (warp < T) {
       // top-k of token t: lane-local candidates in registers, one
       // redux.sync arg-max per round, ties to the lowest expert index;
       // the weights exp(l_j - l_0) / sum are computed by lanes j < k
@@ -440,7 +451,7 @@ __global__ void __launch_bounds__(LAYER_THREADS, 1)
     }
     named_bar_sync(BAR_ALL, CW * 32);
     // grouping: rank of pair q = #{r : (e_r, r) < (e_q, q)}
-    const int P = T * k;
+    const int P = p.mode == DL_ROUTE ? 0 : T * k;   // DL_ROUTE: no units
     if (tid < P) {
       const int eq = M.tk_idx[tid];
       int rank = 0;
@@ -770,8 +781,9 @@ __global__ void __launch_bounds__(LAYER_THREADS, 1)
 
   grid_barrier(p, 2);
 
-  // P5: combine, then the exit count that re-arms the grid barrier
-  {
+  // P5: combine (not in DL_ROUTE), then the exit count that re-arms the
+  // grid barrier
+  if (p.mode != DL_ROUTE) {
     const int64_t n = (int64_t)T * H;
     const int64_t i0 = n * blockIdx.x / G, i1 = n * (blockIdx.x + 1) / G;
     for (int64_t i = i0 + tid; i < i1; i += CW * 32) {
@@ -826,8 +838,9 @@ moe_status launch_decode_layer(const moe_layer_desc& d, const uint16_t* x,
                                const float* residual, float* out,
                                uint16_t* out_bf16, int32_t* topk_idx,
                                float* topk_w, float* logits, void* ws,
-                               int32_t* err, cudaStream_t s) {
+                               int32_t* err, cudaStream_t s, int mode) {
   LayerParams p;
+  p.mode = mode;
   p.pool = d.pool;
   p.stride = d.blob_stride;
   p.blob_index = blob_index;

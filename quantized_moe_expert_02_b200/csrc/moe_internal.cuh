@@ -107,6 +107,13 @@ constexpr int DEC_TMAX = 8;     // tokens per decode call (two N tiles)
 constexpr int NSPLIT_MAX = 4;   // K split of the up/gate units
 constexpr int BF_NT = 2;        // N tiles (4 tokens each) of the B layouts
 
+// Modes of one launch of the one-kernel decode layer.  DL_ROUTE then
+// DL_FFN computes exactly what DL_FULL does (same router partition, same
+// top-k and weights, same FFN), so a caller can act between routing and
+// the FFN (the expert-slot cache fills its misses there) without changing
+// a bit of the result.
+constexpr int DL_FULL = 0, DL_ROUTE = 1, DL_FFN = 2;
+
 struct FfnWs {
   int32_t* err;       // [4]  error word, route counter, spare
   int32_t* up_cnt;    // [P * F/32]   arrival counters, 32-row up tiles

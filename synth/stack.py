@@ -1,0 +1,172 @@
+"""Drivers of the multi-layer decode workloads through the library's C ABI:
+the all-resident residual stack and the same stack over an expert-slot
+pool.  No arithmetic of the layer happens here -- every layer runs in the
+library; this module only owns buffers, builds the device pools with the
+seeded generator, and moves missed expert blobs (one copy per expert).
+
+Step semantics (the 48-layer workloads): step s starts from the residual
+r = x_s (the seeded bf16 activations of step s, widened to fp32); each
+layer l then does r <- r + MoE_l(bf16(rmsnorm(r))) with its own router and
+Zipf(1.1) popularity bias.  Steps are independent except through the slot
+pool's state.
+"""
+from __future__ import annotations
+
+from typing import Dict, List, Optional, Sequence, Tuple
+
+import numpy as np
+
+import synth
+from synth.pools import build_pool, dev, layer_desc
+
+
+class Stack:
+    """L resident layers of one shape, with per-layer routers and biases."""
+
+    def __init__(self, L: int, shape: synth.LayerShape = synth.BIG,
+                 seed: int = 0, T: int = 3, zipf: bool = True,
+                 build_pools: bool = True):
+        import torch
+        import quantized_moe_expert_02_b200 as moe
+        self.torch, self.moe = torch, moe
+        self.L, self.shape, self.seed, self.T = L, shape, seed, T
+        self.pools = [build_pool(shape, seed, l) for l in range(L)] \
+            if build_pools else []
+        self.descs = [layer_desc(shape, p) for p in self.pools]
+        self.wr = [dev(synth.gen_router(seed, l, shape.E, shape.H))
+                   for l in range(L)]
+        self.bias_np = [synth.gen_zipf_bias(seed, l, shape.E)[0] if zipf
+                        else None for l in range(L)]
+        self.ranks = [synth.gen_zipf_bias(seed, l, shape.E)[1]
+                      for l in range(L)]
+        self.bias = [dev(b) if b is not None else None for b in self.bias_np]
+        k, E, H, F = shape.k, shape.E, shape.H, shape.F
+        self.ws_bytes = moe.moe_layer_workspace_bytes(T, k, E, H, F)
+        self.ws = torch.zeros(self.ws_bytes, dtype=torch.uint8, device="cuda")
+        self.idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
+        self.w = torch.empty((T, k), device="cuda")
+
+    # ------------------------------------------------------------ inputs --
+    def x0(self, step: int):
+        """Residual at the stack's input for step s: x_s widened to fp32."""
+        xb = synth.gen_x(self.seed, self.T, self.shape.H, step)
+        return dev(synth.bf16_bits_to_f32(xb).copy())
+
+    # ----------------------------------------------------------- resident --
+    def layer(self, l: int, r, record: Optional[List] = None):
+        """One resident layer, in place (one launch for T <= 8)."""
+        shp = self.shape
+        self.moe.moe_layer_forward_residual(
+            self.descs[l], r, self.T, shp.k, self.wr[l], self.bias[l], None,
+            r, None, self.idx, self.w, None, self.ws, self.ws_bytes)
+        if record is not None:
+            record.append(self.idx.clone())
+
+    def run_resident(self, r, layers: Optional[Sequence[int]] = None,
+                     record: Optional[List] = None):
+        for l in (range(self.L) if layers is None else layers):
+            self.layer(l, r, record)
+        return r
+
+
+def hottest(stack: Stack, l: int, n: int) -> np.ndarray:
+    return synth.hottest_experts(stack.ranks[l], n)
+
+
+class SlotPool:
+    """The expert-slot pool of the slot-cache workload: per-layer
+    partitions of a device pool of blobs, their slot tables, and a pinned
+    host store of the blobs that may be copied in.
+
+    The pool starts filled with each layer's hottest experts (slot i holds
+    the (i+1)-th hottest); misses are copied from `store`, a pinned host
+    tensor with one blob per (layer, expert) key in `store_index`.
+    """
+
+    def __init__(self, stack: Stack, capacities: Sequence[int],
+                 store_keys: Sequence[Tuple[int, int]]):
+        torch, moe, shp = stack.torch, stack.moe, stack.shape
+        self.stack, self.torch, self.moe = stack, torch, moe
+        self.caps = [int(c) for c in capacities]
+        self.base = np.concatenate([[0], np.cumsum(self.caps)])[:-1]
+        n_slots = int(sum(self.caps))
+        stride = shp.blob_stride
+        self.stride = stride
+        self.blob = shp.blob_bytes
+        self.pool = torch.empty(n_slots * stride, dtype=torch.uint8,
+                                device="cuda")
+        E = shp.E
+        self.table, self.owner, self.last = [], [], []
+        for l, cap in enumerate(self.caps):
+            hot = hottest(stack, l, cap)
+            tab = torch.full((E,), -1, dtype=torch.int32, device="cuda")
+            own = torch.full((cap,), -1, dtype=torch.int32, device="cuda")
+            for s, e in enumerate(hot):
+                tab[int(e)] = s
+                own[s] = int(e)
+                dst = (int(self.base[l]) + s) * stride
+                src = int(e) * stride
+                self.pool[dst:dst + self.blob].copy_(
+                    stack.pools[l][src:src + self.blob])
+            self.table.append(tab)
+            self.owner.append(own)
+            self.last.append(torch.zeros(cap, dtype=torch.int32,
+                                         device="cuda"))
+        self.descs = [layer_desc(shp, self.pool) for _ in self.caps]
+        # pinned host store, filled from the resident pools
+        keys = sorted(set((int(l), int(e)) for l, e in store_keys))
+        self.store_index: Dict[Tuple[int, int], int] = {
+            key: i for i, key in enumerate(keys)}
+        self.store = torch.empty((max(1, len(keys)), self.blob),
+                                 dtype=torch.uint8).pin_memory()
+        for (l, e), i in self.store_index.items():
+            src = e * stride
+            self.store[i].copy_(stack.pools[l][src:src + self.blob])
+        torch.cuda.synchronize()
+        P = stack.T * shp.k
+        self.blob_index = torch.full((E,), -1, dtype=torch.int32,
+                                     device="cuda")
+        self.mexp = torch.empty(P, dtype=torch.int32, device="cuda")
+        self.mslot = torch.empty(P, dtype=torch.int32, device="cuda")
+        self.nmiss = torch.zeros(1, dtype=torch.int32, device="cuda")
+        self.err = torch.zeros(1, dtype=torch.int32, device="cuda")
+        self.h_n = torch.zeros(1 + 2 * P, dtype=torch.int32).pin_memory()
+        self.misses = 0
+
+    def layer(self, l: int, r, stamp: int, log: Optional[List] = None):
+        """One layer through the slot pool, in place."""
+        st, torch, moe, shp = self.stack, self.torch, self.moe, \
+            self.stack.shape
+        T, k, E = st.T, shp.k, shp.E
+        moe.moe_layer_route_residual(self.descs[l], r, T, k, st.wr[l],
+                                     st.bias[l], st.idx, st.w, None, st.ws,
+                                     st.ws_bytes)
+        moe.moe_slot_resolve(st.idx, T, k, E, self.table[l], self.owner[l],
+                             self.last[l], self.caps[l], int(self.base[l]),
+                             stamp, self.blob_index, self.mexp, self.mslot,
+                             self.nmiss, self.err)
+        # the miss list to the host, then one copy per missed expert
+        P = T * k
+        self.h_n[0:1].copy_(self.nmiss, non_blocking=True)
+        self.h_n[1:1 + P].copy_(self.mexp, non_blocking=True)
+        self.h_n[1 + P:].copy_(self.mslot, non_blocking=True)
+        torch.cuda.current_stream().synchronize()
+        n = int(self.h_n[0])
+        me = self.h_n[1:1 + n].tolist()
+        ms = self.h_n[1 + P:1 + P + n].tolist()
+        for e, s in zip(me, ms):
+            i = self.store_index[(l, e)]
+            dst = (int(self.base[l]) + s) * self.stride
+            self.pool[dst:dst + self.blob].copy_(self.store[i],
+                                                 non_blocking=True)
+        self.misses += n
+        if log is not None:
+            log.append((l, stamp, me, ms))
+        moe.moe_layer_ffn_residual(self.descs[l], r, T, k, st.idx, st.w,
+                                   self.blob_index, r, None, st.ws,
+                                   st.ws_bytes)
+
+    def run(self, r, stamp: int, log: Optional[List] = None):
+        for l in range(len(self.caps)):
+            self.layer(l, r, stamp, log)
+        return r
