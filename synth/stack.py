@@ -80,11 +80,14 @@ class SlotPool:
 
     The pool starts filled with each layer's hottest experts (slot i holds
     the (i+1)-th hottest); misses are copied from `store`, a pinned host
-    tensor with one blob per (layer, expert) key in `store_index`.
+    tensor with one blob per (layer, expert) key in `store_index`.  With
+    store_keys=None the misses are copied from the stack's resident pools
+    instead (device to device) and their keys collected in `seen_keys`:
+    a discovery run that tells which blobs a host store must hold.
     """
 
     def __init__(self, stack: Stack, capacities: Sequence[int],
-                 store_keys: Sequence[Tuple[int, int]]):
+                 store_keys: Optional[Sequence[Tuple[int, int]]]):
         torch, moe, shp = stack.torch, stack.moe, stack.shape
         self.stack, self.torch, self.moe = stack, torch, moe
         self.caps = [int(c) for c in capacities]
@@ -114,7 +117,10 @@ class SlotPool:
                                          device="cuda"))
         self.descs = [layer_desc(shp, self.pool) for _ in self.caps]
         # pinned host store, filled from the resident pools
-        keys = sorted(set((int(l), int(e)) for l, e in store_keys))
+        self.device_source = store_keys is None
+        self.seen_keys = set()
+        keys = [] if store_keys is None else \
+            sorted(set((int(l), int(e)) for l, e in store_keys))
         self.store_index: Dict[Tuple[int, int], int] = {
             key: i for i, key in enumerate(keys)}
         self.store = torch.empty((max(1, len(keys)), self.blob),
@@ -155,10 +161,16 @@ class SlotPool:
         me = self.h_n[1:1 + n].tolist()
         ms = self.h_n[1 + P:1 + P + n].tolist()
         for e, s in zip(me, ms):
-            i = self.store_index[(l, e)]
             dst = (int(self.base[l]) + s) * self.stride
-            self.pool[dst:dst + self.blob].copy_(self.store[i],
-                                                 non_blocking=True)
+            if self.device_source:
+                self.seen_keys.add((l, e))
+                src = e * self.stride
+                self.pool[dst:dst + self.blob].copy_(
+                    st.pools[l][src:src + self.blob], non_blocking=True)
+            else:
+                i = self.store_index[(l, e)]
+                self.pool[dst:dst + self.blob].copy_(self.store[i],
+                                                     non_blocking=True)
         self.misses += n
         if log is not None:
             log.append((l, stamp, me, ms))
