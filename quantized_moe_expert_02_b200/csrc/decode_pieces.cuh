@@ -27,6 +27,11 @@ __device__ __forceinline__ void piece_sb3(const uint8_t* tp,
   const uint32_t hi[4] = {HV.x, HV.y, HV.z, HV.w};
   int32_t S[2][2] = {{0, 0}, {0, 0}};
   const int32_t zero[4] = {0, 0, 0, 0};
+  // (2s+1) of the eight 32-blocks as bytes: even blocks, odd blocks
+  const uint32_t mge = (SC.x & 0x0F0F0F0Fu) * 2u + 0x01010101u;
+  const uint32_t mgo = ((SC.x >> 4) & 0x0F0F0F0Fu) * 2u + 0x01010101u;
+  const uint32_t m8e = (SC.y & 0x0F0F0F0Fu) * 2u + 0x01010101u;
+  const uint32_t m8o = ((SC.y >> 4) & 0x0F0F0F0Fu) * 2u + 0x01010101u;
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
     const uint32_t LO = lo[j], HH = hi[j >> 1];
@@ -39,8 +44,10 @@ __device__ __forceinline__ void piece_sb3(const uint8_t* tp,
     a[1] = prmt(SB3_TAB0, SB3_TAB1, sa >> 16);
     a[2] = prmt(SB3_TAB0, SB3_TAB1, sb);
     a[3] = prmt(SB3_TAB0, SB3_TAB1, sb >> 16);
-    const int mg = (int)((SC.x >> (4 * j)) & 15u) * 2 + 1;
-    const int mg8 = (int)((SC.y >> (4 * j)) & 15u) * 2 + 1;
+    // byte j/2 of the even/odd word, zero-extended (prmt selector 0x444m)
+    const uint32_t bsel = 0x4440u | (uint32_t)(j >> 1);
+    const int mg = (int)prmt((j & 1) ? mgo : mge, 0u, bsel);
+    const int mg8 = (int)prmt((j & 1) ? m8o : m8e, 0u, bsel);
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
       if (nt < NT) {
