@@ -115,7 +115,7 @@ struct Carver {
 
 struct Layout {
   size_t err, up_cnt, dn_cnt, up_part, bfrag, bscale, y_int, h;
-  size_t x16, xscale, tiles, n_tiles, total;
+  size_t x16, xscale, inv, tiles, n_tiles, total;
 };
 
 static Layout ffn_layout(int T, int k, int H, int F) {
@@ -134,6 +134,7 @@ static Layout ffn_layout(int T, int k, int H, int F) {
   L.h = c.take(P * F * 4);
   L.x16 = c.take(dec ? 0 : P * H * 2);
   L.xscale = c.take(dec ? 0 : P * 4);
+  L.inv = c.take(dec ? 0 : P * 4);
   L.tiles = c.take(dec ? 0 : pf_max_tiles(P) * 16);
   L.n_tiles = c.take(64);
   L.total = c.off;
@@ -154,6 +155,7 @@ FfnWs carve_ffn_ws(void* base, int T, int k, int H, int F) {
   w.h = reinterpret_cast<float*>(b + L.h);
   w.x16 = reinterpret_cast<__half*>(b + L.x16);
   w.xscale = reinterpret_cast<float*>(b + L.xscale);
+  w.inv = reinterpret_cast<int32_t*>(b + L.inv);
   w.tiles = reinterpret_cast<int4*>(b + L.tiles);
   w.n_tiles = reinterpret_cast<int32_t*>(b + L.n_tiles);
   w.logits = nullptr;

@@ -22,6 +22,54 @@ __global__ void combine_kernel(const float* __restrict__ y,
   }
 }
 
+// The same sum, four columns per thread: the k rows' float4 loads are all
+// issued before the multiply-adds, which run in the same order (j
+// ascending, then the residual), so the result is bit-identical to the
+// one-column form.  H a multiple of 4, 16-byte aligned y/residual/out.
+__global__ void __launch_bounds__(256)
+    combine4_kernel(const float4* __restrict__ y, const float* __restrict__ w,
+                    int T, int k, int H4, const float4* residual,
+                    float4* out, uint2* __restrict__ out_bf16) {
+  const int64_t n = (int64_t)T * H4;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t t = i / H4;
+    const int h = (int)(i - t * H4);
+    const float* wt = w + t * k;
+    const float4* yt = y + t * k * H4 + h;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j0 = 0; j0 < k; j0 += 8) {
+      float4 v[8];
+#pragma unroll
+      for (int jj = 0; jj < 8; ++jj)
+        if (j0 + jj < k) v[jj] = __ldcs(yt + (int64_t)(j0 + jj) * H4);
+#pragma unroll
+      for (int jj = 0; jj < 8; ++jj)
+        if (j0 + jj < k) {
+          const float wj = __ldg(wt + j0 + jj);
+          acc.x = fmaf(wj, v[jj].x, acc.x);
+          acc.y = fmaf(wj, v[jj].y, acc.y);
+          acc.z = fmaf(wj, v[jj].z, acc.z);
+          acc.w = fmaf(wj, v[jj].w, acc.w);
+        }
+    }
+    if (residual) {
+      const float4 r = residual[i];
+      acc.x += r.x;
+      acc.y += r.y;
+      acc.z += r.z;
+      acc.w += r.w;
+    }
+    out[i] = acc;
+    if (out_bf16)
+      out_bf16[i] = make_uint2(
+          (uint32_t)f32_to_bf16_rne(acc.x) |
+              ((uint32_t)f32_to_bf16_rne(acc.y) << 16),
+          (uint32_t)f32_to_bf16_rne(acc.z) |
+              ((uint32_t)f32_to_bf16_rne(acc.w) << 16));
+  }
+}
+
 // x = bf16(r / sqrt(mean(r^2) + eps)), one block per row.
 __global__ void __launch_bounds__(256)
     rmsnorm_bf16_kernel(const float* __restrict__ r, int H,
@@ -44,11 +92,36 @@ __global__ void __launch_bounds__(256)
 moe_status launch_combine(const float* y, const float* w, int T, int k,
                           int H, const float* residual, float* out,
                           uint16_t* out_bf16, cudaStream_t s) {
-  const int64_t n = (int64_t)T * H;
+  auto a16 = [](const void* q) {
+    return (reinterpret_cast<uintptr_t>(q) & 15) == 0;
+  };
+  const bool vec = H % 4 == 0 && a16(y) && a16(out) &&
+                   (!residual || a16(residual)) &&
+                   (!out_bf16 || (reinterpret_cast<uintptr_t>(out_bf16) & 7) == 0);
+  const int64_t n = (int64_t)T * (vec ? H / 4 : H);
+  // one wave of resident blocks, striding over the elements
+  static int occ[2] = {0, 0};
+  int& o = occ[vec ? 1 : 0];
+  if (!o) {
+    int b = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+            &b,
+            vec ? reinterpret_cast<const void*>(&combine4_kernel)
+                : reinterpret_cast<const void*>(&combine_kernel),
+            256, 0) != cudaSuccess || b <= 0)
+      b = 2;
+    o = b;
+  }
   int64_t g = (n + 255) / 256;
-  if (g > (int64_t)num_sms() * 16) g = (int64_t)num_sms() * 16;
-  combine_kernel<<<(int)g, 256, 0, s>>>(y, w, T, k, H, residual, out,
-                                        out_bf16);
+  if (g > (int64_t)num_sms() * o) g = (int64_t)num_sms() * o;
+  if (vec)
+    combine4_kernel<<<(int)g, 256, 0, s>>>(
+        reinterpret_cast<const float4*>(y), w, T, k, H / 4,
+        reinterpret_cast<const float4*>(residual),
+        reinterpret_cast<float4*>(out), reinterpret_cast<uint2*>(out_bf16));
+  else
+    combine_kernel<<<(int)g, 256, 0, s>>>(y, w, T, k, H, residual, out,
+                                          out_bf16);
   return launch_status();
 }
 

@@ -7,7 +7,10 @@
 // up/gate units (one per slot), then -- without waiting for the up phase to
 // finish -- the down units (four per slot), so the expert stream does not
 // stop at the phase boundaries; warp 17 publishes finished up units to the
-// other blocks.  Only the warps that use a slot wait on it and release it.
+// other blocks; warps 18 and 19 finish the up units of the two up groups
+// (reduction, SwiGLU, h stores), so that the compute warps go on to their
+// next unit at once.  Only the warps that use a slot wait on it and
+// release it.
 //
 // Phases (grid barriers marked ||):
 //   P0  router logits: the E rows are split over the blocks; x staged in
@@ -18,7 +21,8 @@
 //       of the T*k pairs by expert -- all in shared memory; meanwhile the
 //       other warps turn x into int8 hi/lo B fragments (per-token 2^-sigma)
 //   P2  up/gate units (expert, 16 rows of F, all of H), two groups of eight
-//       warps taking alternate units, three tiles per warp:
+//       warps taking alternate units, three tiles per warp, partial sums
+//       -> shared memory; the group's epilogue warp reduces them,
 //       h = silu(g) * u of each of the expert's tokens -> global,
 //       |h| max per pair -> global; each finished unit counts towards its
 //       expert's completion counter
@@ -38,13 +42,15 @@ namespace moe {
 namespace {
 
 constexpr int CW = 16;                      // compute warps
-constexpr int LAYER_THREADS = (CW + 2) * 32;
+constexpr int LAYER_THREADS = (CW + 4) * 32;
 constexpr int PRODUCER = CW;                // warp index of the producer
 constexpr int SIGNALER = CW + 1;            // publishes finished up units
+constexpr int UPEPI = CW + 2;               // up epilogue warps: 18, 19
 constexpr int NSLOT = 4;                    // ring slots
 constexpr int MAXP = 96;                    // max pairs (T*k) per call
 constexpr int BAR_ALL = 1;                  // named barrier: all 16 warps
-constexpr int BAR_UP = 2;                   // 2, 3: up groups
+constexpr int BAR_RDY = 2;                  // 2, 3: up partials written
+constexpr int BAR_FREE = 9;                 // 9, 10: up partials read
 constexpr int BAR_DN = 4;                   // 4..7: down groups
 constexpr int BAR_XF = 8;                   // warps that build x fragments
 constexpr int UPG = 2, UPW = CW / UPG;      // up: 2 groups of 8 warps
@@ -86,12 +92,10 @@ __host__ __device__ inline int dn_unit_bytes(int F) {
   return (F / B32_TILE_COLS) * B32_TILE_BYTES;
 }
 // Reduction buffers: an up group holds [UPW][32 lanes][NT][2 rows][2]
-// floats (double-buffered when NT == 1: then one group barrier per unit
-// suffices), a down group [DNW][32][NT][2] (double-buffered).
+// floats, a down group [DNW][32][NT][2] (double-buffered).
 __host__ __device__ inline int red_up_floats(int NT) {
   return UPW * 32 * NT * 4;
 }
-__host__ __device__ inline int red_up_bufs(int NT) { return NT == 1 ? 2 : 1; }
 __host__ __device__ inline int red_dn_floats(int NT) {
   return DNW * 32 * NT * 2;
 }
@@ -104,7 +108,7 @@ __host__ __device__ inline Smem smem_layout(int fmt_ug, int H, int F, int T) {
   const int NT = (T + 3) / 4;
   const int xfrag = (H / 32) * NT * 64 * 4;
   const int hfrag = 2 * (F / 32) * NT * 64 * 4;
-  const int red_up = UPG * red_up_bufs(NT) * red_up_floats(NT) * 4;
+  const int red_up = UPG * red_up_floats(NT) * 4;
   const int red_dn = DNG * 2 * red_dn_floats(NT) * 4;
   L.slot_bytes = slot;
   L.ring = 0;
@@ -489,8 +493,12 @@ __global__ void __launch_bounds__(LAYER_THREADS, 1)
   const int nrt_f = F / 16, nrt_h = H / 16;
   // up units: (u, rt) over U x F/16; down units: (u, rt) over U x H/16
   const int nu_all = U * nrt_f, nd_all = U * nrt_h;
-  const int u0 = (int)((int64_t)nu_all * blockIdx.x / G);
-  const int u1 = (int)((int64_t)nu_all * (blockIdx.x + 1) / G);
+  // up units are dealt round-robin (unit b + i*G is this block's i-th), so
+  // the experts' up units finish in expert order across the grid and a
+  // down unit rarely waits; down units are contiguous ranges (at most two
+  // experts per block)
+  const int b0 = blockIdx.x;
+  const int n_up = nu_all > b0 ? (nu_all - 1 - b0) / G + 1 : 0;
   const int d0 = (int)((int64_t)nd_all * blockIdx.x / G);
   const int d1 = (int)((int64_t)nd_all * (blockIdx.x + 1) / G);
   const int dnb = dn_unit_bytes(F);
@@ -507,7 +515,8 @@ __global__ void __launch_bounds__(LAYER_THREADS, 1)
           mbar_wait(&M.empty[s], ((slot_i / NSLOT) - 1) & 1, p.err);
         return s;
       };
-      for (int v = u0; v < u1; ++v, ++i) {
+      for (; i < n_up; ++i) {
+        const int v = b0 + i * G;
         const int s = acquire(i);
         const int u = v / nrt_f, rt = v % nrt_f;
         const uint8_t* b = expert_base(p, M.active[u]);
@@ -543,29 +552,97 @@ __global__ void __launch_bounds__(LAYER_THREADS, 1)
   // Publishes this block's finished up units to the per-expert counters
   // (gpu-scope release), so that the compute warps never wait on a fence.
   if (warp == SIGNALER) {
-    if (lane == 0 && u1 > u0) {
-      const int ua = u0 / nrt_f, ub = (u1 - 1) / nrt_f;
-      int pub[4] = {0, 0, 0, 0};
-      int left = u1 - u0;
+    if (n_up > 0) {
+      // lane l watches experts l, l + 32, l + 64 (U <= MAXP)
+      int pub[MAXP / 32];
+#pragma unroll
+      for (int i = 0; i < MAXP / 32; ++i) pub[i] = 0;
+      int left = n_up;
       const uint64_t t0 = globaltimer();
-      bool gave_up = false;
-      while (left > 0 && !gave_up) {
-        for (int u = ua; u <= ub && u - ua < 4; ++u) {
-          const int d = *reinterpret_cast<volatile int32_t*>(&M.up_fin[u]);
-          if (d > pub[u - ua]) {
-            fence_acq_rel();
-            atomicAdd(p.up_done + u, d - pub[u - ua]);
-            left -= d - pub[u - ua];
-            pub[u - ua] = d;
+      while (left > 0) {
+        int got = 0;
+#pragma unroll
+        for (int i = 0; i < MAXP / 32; ++i) {
+          const int u = lane + 32 * i;
+          if (u < U) {
+            const int d = *reinterpret_cast<volatile int32_t*>(&M.up_fin[u]);
+            if (d > pub[i]) {
+              fence_acq_rel();
+              atomicAdd(p.up_done + u, d - pub[i]);
+              got += d - pub[i];
+              pub[i] = d;
+            }
           }
         }
+        left -= __reduce_add_sync(0xffffffffu, (unsigned)got);
         if (left > 0) {
           __nanosleep(64);
-          if (globaltimer() - t0 > 500000000ull) {
-            set_err(p.err, MOE_ERR_TIMEOUT);
-            gave_up = true;
+          if (__any_sync(0xffffffffu, globaltimer() - t0 > 500000000ull)) {
+            if (lane == 0) set_err(p.err, MOE_ERR_TIMEOUT);
+            break;
           }
         }
+      }
+    }
+    return;
+  }
+
+  // ------------------------------------------------ up epilogue warps --
+  // Warp UPEPI + ug, for each unit of up group ug: the group's partial
+  // sums (eight warps) -> u, g of the unit's 16 rows for each of the
+  // expert's pairs (lane o + 32i: pair slot o / 16, row o % 16); the buffer
+  // is released before h = silu(g) * u goes to global memory, |h| max per
+  // pair to hmax, and the unit is counted for the signaler.
+  if (warp >= UPEPI) {
+    const int ug = warp - UPEPI;
+    const float* rb = red + ug * red_up_floats(NT);
+    constexpr int OPL = TM / 2;   // outputs per lane: TM pairs x 16 rows
+    for (int i = ug; i < n_up; i += UPG) {
+      const int v = b0 + i * G;
+      const int u = v / nrt_f, rt = v % nrt_f;
+      const int pb = M.off[u], Tu = M.off[u + 1] - pb;
+      named_bar_sync(BAR_RDY + ug, (UPW + 1) * 32);
+      float su[OPL], sg[OPL];
+      int pp[OPL];
+#pragma unroll
+      for (int i = 0; i < OPL; ++i) {
+        const int o = lane + 32 * i, slot = o >> 4, rho = o & 15;
+        su[i] = 0.f;
+        sg[i] = 0.f;
+        pp[i] = -1;
+        if (slot < Tu) {
+          pp[i] = M.sorted[pb + slot];
+          const int t = pp[i] / k;
+          const int Ln = 4 * (rho & 7) + (t & 3), nt = t >> 2, hh = rho >> 3;
+#pragma unroll
+          for (int w = 0; w < UPW; ++w) {
+            su[i] += rb[(w * 32 + Ln) * NT * 4 + (nt * 2 + hh) * 2 + 0];
+            sg[i] += rb[(w * 32 + Ln) * NT * 4 + (nt * 2 + hh) * 2 + 1];
+          }
+        }
+      }
+      named_bar_arrive(BAR_FREE + ug, (UPW + 1) * 32);
+#pragma unroll
+      for (int i = 0; i < OPL; ++i) {
+        const int rho = lane & 15;
+        float hv = 0.f;
+        if (pp[i] >= 0) {
+          hv = __fdividef(sg[i], 1.0f + __expf(-sg[i])) * su[i];
+          p.h[(int64_t)pp[i] * F + 16 * rt + rho] = hv;
+        }
+        float m = fabsf(hv);
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1)
+          m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if (rho == 0 && pp[i] >= 0)
+          atomicMax(p.hmax + pp[i], __float_as_uint(m));
+      }
+      // the unit's h / hmax writes, then its count; the signaler releases
+      // them at gpu scope
+      __syncwarp();
+      if (lane == 0) {
+        __threadfence_block();
+        atomicAdd(&M.up_fin[u], 1);
       }
     }
     return;
@@ -575,28 +652,19 @@ __global__ void __launch_bounds__(LAYER_THREADS, 1)
   const int c = lane & 3;
   int slot_i = 0;
 
-  // P2: up/gate + SwiGLU.  Group ug takes units v with (v-u0) % 2 == ug.
+  // P2: up/gate partial sums.  Group ug takes this block's units i with
+  // i % 2 == ug; its epilogue warp finishes them (one partial-sum buffer
+  // per group: written after the epilogue warp has read the previous
+  // unit's).
   {
     const int ug = warp / UPW, wg = warp % UPW;
-    const int gtid = tid - ug * UPW * 32;
-    const int nbuf = red_up_bufs(NT);
-    const int rfl = red_up_floats(NT);
+    float* rb = red + ug * red_up_floats(NT);
     float xs2[2];
     xs2[0] = M.xsc[c];
     xs2[1] = M.xsc[4 + c];
     int mine = 0;
-    int prev_u = -1;      // expert of this group's previous unit
-    auto signal = [&](int u) {
-      // one finished unit of expert u: the group's barrier before this made
-      // the group's h / hmax writes visible to this thread; the signaler
-      // warp releases them at gpu scope
-      if (gtid == 0 && u >= 0) {
-        __threadfence_block();
-        atomicAdd(&M.up_fin[u], 1);
-      }
-    };
-    for (int v = u0; v < u1; ++v, ++slot_i) {
-      if (((v - u0) & 1) != ug) continue;     // the other group's unit
+    for (int i = 0; i < n_up; ++i, ++slot_i) {
+      if ((i & 1) != ug) continue;            // the other group's unit
       const int s = slot_i % NSLOT;
       mbar_wait(&M.full[s], (slot_i / NSLOT) & 1, p.err);
       const uint8_t* unit = ring + s * L.slot_bytes;
@@ -616,7 +684,7 @@ __global__ void __launch_bounds__(LAYER_THREADS, 1)
       }
       __syncwarp();
       if (lane == 0) mbar_arrive_n(&M.empty[s], CW / UPW);
-      float* rb = red + (ug * nbuf + (mine % nbuf)) * rfl;
+      if (mine > 0) named_bar_sync(BAR_FREE + ug, (UPW + 1) * 32);
       float* rw = rb + (wg * 32 + lane) * NT * 4;
       for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -624,45 +692,10 @@ __global__ void __launch_bounds__(LAYER_THREADS, 1)
           rw[(nt * 2 + hh) * 2 + 0] = au[nt][hh];
           rw[(nt * 2 + hh) * 2 + 1] = ag[nt][hh];
         }
-      named_bar_sync(BAR_UP + ug, UPW * 32);
-      if (nbuf == 2) signal(prev_u);     // epilogue of the previous unit
-      {
-        const int u = v / nrt_f, rt = v % nrt_f;
-        const int pb = M.off[u], Tu = M.off[u + 1] - pb;
-        const int slot = gtid >> 4, rho = gtid & 15;     // gtid < 256
-        float hv = 0.f;
-        int pp = -1;
-        if (slot < Tu) {
-          pp = M.sorted[pb + slot];
-          const int t = pp / k;
-          const int Ln = 4 * (rho & 7) + (t & 3), nt = t >> 2, hh = rho >> 3;
-          float su = 0.f, sg = 0.f;
-#pragma unroll
-          for (int w = 0; w < UPW; ++w) {
-            su += rb[(w * 32 + Ln) * NT * 4 + (nt * 2 + hh) * 2 + 0];
-            sg += rb[(w * 32 + Ln) * NT * 4 + (nt * 2 + hh) * 2 + 1];
-          }
-          hv = sg / (1.0f + expf(-sg)) * su;
-          p.h[(int64_t)pp * F + 16 * rt + rho] = hv;
-        }
-        float m = fabsf(hv);
-#pragma unroll
-        for (int o = 8; o > 0; o >>= 1)
-          m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        if (rho == 0 && pp >= 0) atomicMax(p.hmax + pp, __float_as_uint(m));
-      }
-      if (nbuf == 1) {
-        named_bar_sync(BAR_UP + ug, UPW * 32);
-        signal(v / nrt_f);
-      } else {
-        prev_u = v / nrt_f;
-      }
+      named_bar_arrive(BAR_RDY + ug, (UPW + 1) * 32);
       ++mine;
     }
-    if (nbuf == 2 && prev_u >= 0) {
-      named_bar_sync(BAR_UP + ug, UPW * 32);
-      signal(prev_u);
-    }
+    if (mine > 0) named_bar_sync(BAR_FREE + ug, (UPW + 1) * 32);
   }
 
   // P3: B fragments of h for this block's down experts (at most two),

@@ -129,6 +129,7 @@ struct FfnWs {
   // grouped row order
   __half* x16;        // [T*k][H] activations as fp16, grouped row order
   float* xscale;      // [T*k]    2^sigma per grouped row
+  int32_t* inv;       // [T*k]    grouped row of each pair
   int4* tiles;        // unit list: {expert, first grouped row, rows, 0}
   int32_t* n_tiles;
   size_t bytes;
@@ -208,6 +209,21 @@ __device__ __forceinline__ bool mbar_try_wait(void* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// The same test, but a thread whose phase is not complete is suspended
+// (issuing nothing) until the phase completes or about `ns` nanoseconds
+// pass.
+__device__ __forceinline__ bool mbar_try_wait_sleep(void* bar, uint32_t parity,
+                                                    uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n"
+      " mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+      " selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
 // Wait for the phase of `parity` to complete; give up after 0.5 s of
 // %globaltimer, set MOE_ERR_TIMEOUT and return false.  Once any wait of the
 // launch has given up, later waits return false at once.
@@ -217,7 +233,7 @@ __device__ __forceinline__ bool mbar_wait(void* bar, uint32_t parity,
   if (err && *reinterpret_cast<volatile int32_t*>(err) == MOE_ERR_TIMEOUT)
     return false;
   const uint64_t t0 = globaltimer();
-  while (!mbar_try_wait(bar, parity)) {
+  while (!mbar_try_wait_sleep(bar, parity, 20000u)) {
     if (globaltimer() - t0 > 500000000ull) {
       set_err(err, MOE_ERR_TIMEOUT);
       return false;
@@ -239,6 +255,12 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src,
 
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+// Arrive on named barrier `id` without waiting (the barrier's other
+// participants wait with bar.sync); this thread's earlier memory accesses
+// are performed for them when the barrier completes.
+__device__ __forceinline__ void named_bar_arrive(int id, int nthreads) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 __device__ __forceinline__ void grid_dep_wait() {

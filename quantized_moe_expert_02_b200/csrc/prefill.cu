@@ -684,17 +684,27 @@ __global__ void __launch_bounds__(1024)
   }
 }
 
-// Grouped row r = x[pair_ids[r] / k] as fp16, scaled by a per-row power of
-// two 2^-sigma that keeps every value below 2^15 (sigma = 0 unless
-// max|x_t| >= 2^15); xscale[r] = 2^sigma.  H a multiple of 8.
+// inv[pair_ids[r]] = r: the grouped row of every pair (pair_ids is a
+// permutation of 0 .. P-1, as the grouping produces it).
+__global__ void pf_inv_kernel(const int32_t* __restrict__ pair_ids, int P,
+                              int32_t* __restrict__ inv) {
+  const int r = blockIdx.x * blockDim.x + threadIdx.x;
+  if (r < P) inv[pair_ids[r]] = r;
+}
+
+// One block per token t: x[t] as fp16, scaled by a power of two 2^-sigma
+// that keeps every value below 2^15 (sigma = 0 unless max|x_t| >= 2^15),
+// written to the grouped rows of the token's k pairs; xscale of those rows
+// = 2^sigma.  H a multiple of 8.
 __global__ void __launch_bounds__(256)
-    pf_xg_kernel(const uint16_t* __restrict__ x, int H,
-                 const int32_t* __restrict__ pair_ids, int k,
-                 __half* __restrict__ xg, float* __restrict__ xscale) {
+    pf_xg_kernel(const uint16_t* __restrict__ x, int H, int k,
+                 const int32_t* __restrict__ inv, __half* __restrict__ xg,
+                 float* __restrict__ xscale) {
   __shared__ float red[8];
-  const int64_t r = blockIdx.x;
-  const uint4* xr =
-      reinterpret_cast<const uint4*>(x + (int64_t)(pair_ids[r] / k) * H);
+  __shared__ int32_t rows[32];
+  const int64_t t = blockIdx.x;
+  if (threadIdx.x < k) rows[threadIdx.x] = inv[t * k + threadIdx.x];
+  const uint4* xr = reinterpret_cast<const uint4*>(x + t * H);
   const int nch = H / 8;
   float m = 0.f;
   for (int c = threadIdx.x; c < nch; c += blockDim.x) {
@@ -713,20 +723,21 @@ __global__ void __launch_bounds__(256)
   for (int w = 1; w < (int)(blockDim.x >> 5); ++w) m = fmaxf(m, red[w]);
   int sigma = 0;
   if (m >= 32768.f && m <= 3.0e38f) sigma = ilogbf(m) - 14;
-  const float inv = ldexpf(1.f, -sigma);
-  if (threadIdx.x == 0) xscale[r] = ldexpf(1.f, sigma);
-  uint4* o = reinterpret_cast<uint4*>(xg + r * H);
+  const float inv_s = ldexpf(1.f, -sigma);
+  if (threadIdx.x < k) xscale[rows[threadIdx.x]] = ldexpf(1.f, sigma);
   for (int c = threadIdx.x; c < nch; c += blockDim.x) {
     const uint4 v = __ldg(xr + c);
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
     uint32_t h[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const __half2 t = __floats2half2_rn(__uint_as_float(w[i] << 16) * inv,
-                                          __uint_as_float(w[i] & 0xFFFF0000u) * inv);
-      h[i] = *reinterpret_cast<const uint32_t*>(&t);
+      const __half2 q = __floats2half2_rn(__uint_as_float(w[i] << 16) * inv_s,
+                                          __uint_as_float(w[i] & 0xFFFF0000u) * inv_s);
+      h[i] = *reinterpret_cast<const uint32_t*>(&q);
     }
-    o[c] = make_uint4(h[0], h[1], h[2], h[3]);
+    const uint4 hv = make_uint4(h[0], h[1], h[2], h[3]);
+    for (int j = 0; j < k; ++j)
+      reinterpret_cast<uint4*>(xg + (int64_t)rows[j] * H)[c] = hv;
   }
 }
 
@@ -808,8 +819,9 @@ moe_status launch_pf_up(const moe_layer_desc& d, const uint16_t* x, int T,
   PfMaps map;
   moe_status st = encode_maps(&map, w.x16, (uint64_t)d.H, (uint64_t)P);
   if (st != MOE_OK) return st;
-  pf_xg_kernel<<<(unsigned)P, 256, 0, s>>>(x, d.H, pair_ids, k, w.x16,
-                                           w.xscale);
+  pf_inv_kernel<<<(unsigned)((P + 255) / 256), 256, 0, s>>>(pair_ids, (int)P,
+                                                           w.inv);
+  pf_xg_kernel<<<T, 256, 0, s>>>(x, d.H, k, w.inv, w.x16, w.xscale);
   pf_plan_kernel<<<1, 1024, 0, s>>>(offsets, d.E, w.tiles, w.n_tiles);
   st = launch_status();
   if (st != MOE_OK) return st;
