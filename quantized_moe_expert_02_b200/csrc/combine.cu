@@ -22,29 +22,29 @@ __global__ void combine_kernel(const float* __restrict__ y,
   }
 }
 
-// The same sum, four columns per thread: the k rows' float4 loads are all
-// issued before the multiply-adds, which run in the same order (j
-// ascending, then the residual), so the result is bit-identical to the
-// one-column form.  H a multiple of 4, 16-byte aligned y/residual/out.
+// The same sum, one block per token and four columns per thread: four of
+// the k rows' float4 loads are issued before their multiply-adds, which
+// run in the same order (j ascending, then the residual), so the result
+// is bit-identical to the one-column form.  H a multiple of 4, 16-byte
+// aligned y/residual/out.
 __global__ void __launch_bounds__(256)
-    combine4_kernel(const float4* __restrict__ y, const float* __restrict__ w,
-                    int T, int k, int H4, const float4* residual,
-                    float4* out, uint2* __restrict__ out_bf16) {
-  const int64_t n = (int64_t)T * H4;
-  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t t = i / H4;
-    const int h = (int)(i - t * H4);
-    const float* wt = w + t * k;
-    const float4* yt = y + t * k * H4 + h;
+    combine_row_kernel(const float4* __restrict__ y,
+                       const float* __restrict__ w, int k, int H4,
+                       const float4* residual, float4* out,
+                       uint2* __restrict__ out_bf16) {
+  constexpr int CH = 4;
+  const int64_t t = blockIdx.x;
+  const float* wt = w + t * k;
+  const float4* yt = y + t * k * H4;
+  for (int h = threadIdx.x; h < H4; h += blockDim.x) {
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int j0 = 0; j0 < k; j0 += 8) {
-      float4 v[8];
+    for (int j0 = 0; j0 < k; j0 += CH) {
+      float4 v[CH];
 #pragma unroll
-      for (int jj = 0; jj < 8; ++jj)
-        if (j0 + jj < k) v[jj] = __ldcs(yt + (int64_t)(j0 + jj) * H4);
+      for (int jj = 0; jj < CH; ++jj)
+        if (j0 + jj < k) v[jj] = __ldcs(yt + (int64_t)(j0 + jj) * H4 + h);
 #pragma unroll
-      for (int jj = 0; jj < 8; ++jj)
+      for (int jj = 0; jj < CH; ++jj)
         if (j0 + jj < k) {
           const float wj = __ldg(wt + j0 + jj);
           acc.x = fmaf(wj, v[jj].x, acc.x);
@@ -53,6 +53,7 @@ __global__ void __launch_bounds__(256)
           acc.w = fmaf(wj, v[jj].w, acc.w);
         }
     }
+    const int64_t i = t * H4 + h;
     if (residual) {
       const float4 r = residual[i];
       acc.x += r.x;
@@ -98,30 +99,18 @@ moe_status launch_combine(const float* y, const float* w, int T, int k,
   const bool vec = H % 4 == 0 && a16(y) && a16(out) &&
                    (!residual || a16(residual)) &&
                    (!out_bf16 || (reinterpret_cast<uintptr_t>(out_bf16) & 7) == 0);
-  const int64_t n = (int64_t)T * (vec ? H / 4 : H);
-  // one wave of resident blocks, striding over the elements
-  static int occ[2] = {0, 0};
-  int& o = occ[vec ? 1 : 0];
-  if (!o) {
-    int b = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-            &b,
-            vec ? reinterpret_cast<const void*>(&combine4_kernel)
-                : reinterpret_cast<const void*>(&combine_kernel),
-            256, 0) != cudaSuccess || b <= 0)
-      b = 2;
-    o = b;
-  }
-  int64_t g = (n + 255) / 256;
-  if (g > (int64_t)num_sms() * o) g = (int64_t)num_sms() * o;
-  if (vec)
-    combine4_kernel<<<(int)g, 256, 0, s>>>(
-        reinterpret_cast<const float4*>(y), w, T, k, H / 4,
+  if (vec) {
+    combine_row_kernel<<<T, 256, 0, s>>>(
+        reinterpret_cast<const float4*>(y), w, k, H / 4,
         reinterpret_cast<const float4*>(residual),
         reinterpret_cast<float4*>(out), reinterpret_cast<uint2*>(out_bf16));
-  else
+  } else {
+    const int64_t n = (int64_t)T * H;
+    int64_t g = (n + 255) / 256;
+    if (g > (int64_t)num_sms() * 8) g = (int64_t)num_sms() * 8;
     combine_kernel<<<(int)g, 256, 0, s>>>(y, w, T, k, H, residual, out,
                                           out_bf16);
+  }
   return launch_status();
 }
 

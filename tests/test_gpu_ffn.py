@@ -135,3 +135,37 @@ def test_bad_blob_index_sets_error_word():
     moe.moe_expert_ffn_q(desc, dev(x), T, shape.k, off, pairs, act, na, bi, y,
                          ws.t, ws.nbytes)
     assert moe.moe_get_device_status(ws.t) == moe.MOE_ERR_DEVICE
+
+
+@pytest.mark.parametrize("T,k,H", [(7, 10, 3072), (5, 3, 20), (3, 2, 6)])
+def test_combine_paths_bit_identical(T, k, H):
+    """moe_combine on 16-byte aligned rows (four columns per thread) and on
+    misaligned views (one column per thread) gives the same bits, equal to
+    the oracle's weighted sum; residual and bf16 output included."""
+    g = torch.Generator().manual_seed(T * 100 + H)
+    yh = torch.randn((T * k * H + 4,), generator=g)
+    wh = torch.rand((T, k), generator=g)
+    rh = torch.randn((T * H + 4,), generator=g)
+    y_al = yh[:T * k * H].cuda().view(T * k, H)
+    r_al = rh[:T * H].cuda().view(T, H)
+    ybuf = torch.empty(T * k * H + 1, device="cuda")
+    ybuf[1:].copy_(yh[:T * k * H])
+    rbuf = torch.empty(T * H + 1, device="cuda")
+    rbuf[1:].copy_(rh[:T * H])
+    wd = wh.cuda()
+    outs = []
+    for y, r, off in ((y_al, r_al, 0), (ybuf[1:].view(T * k, H),
+                                        rbuf[1:].view(T, H), 1)):
+        ob = torch.empty(T * H + 1, device="cuda")
+        out = ob[off:off + T * H].view(T, H)
+        bb = torch.empty(T * H + 1, dtype=torch.int16, device="cuda")
+        outb = bb[off:off + T * H].view(T, H)
+        moe.moe_combine(y, wd, T, k, H, r, out, outb)
+        torch.cuda.synchronize()
+        outs.append((out.clone(), outb.clone()))
+    assert torch.equal(outs[0][0], outs[1][0])
+    assert torch.equal(outs[0][1], outs[1][1])
+    ref = o.combine(yh[:T * k * H].view(T * k, H).double().numpy(),
+                    wh.double().numpy(),
+                    rh[:T * H].view(T, H).double().numpy())
+    assert row_max_rel(outs[0][0].cpu().numpy(), ref) <= 1e-5
