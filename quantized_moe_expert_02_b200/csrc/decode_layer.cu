@@ -146,6 +146,25 @@ __device__ __forceinline__ int ld_acquire(const int32_t* p) {
 __device__ __forceinline__ void fence_acq_rel() {
   asm volatile("fence.acq_rel.gpu;" ::: "memory");
 }
+__device__ __forceinline__ void red_release_add(int32_t* p, int v) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v)
+               : "memory");
+}
+// Spin until *cnt >= target (acquire); gives up after 0.5 s of
+// %globaltimer (MOE_ERR_TIMEOUT, or at once when an earlier wait of this
+// launch gave up).  The timer is read every 64 polls.
+__device__ __forceinline__ void spin_until(const int32_t* cnt, int target,
+                                           int32_t* err) {
+  if (ld_acquire(cnt) >= target) return;
+  if (*reinterpret_cast<volatile int32_t*>(err) == MOE_ERR_TIMEOUT) return;
+  const uint64_t t0 = globaltimer();
+  for (int it = 1; ld_acquire(cnt) < target; ++it) {
+    if ((it & 63) == 0 && globaltimer() - t0 > 500000000ull) {
+      set_err(err, MOE_ERR_TIMEOUT);
+      return;
+    }
+  }
+}
 
 // Grid barrier among the compute warps of all blocks: barrier number `n`
 // (1, 2, 3) completes when the counter reaches n * gridDim.x.  Bounded:
@@ -153,23 +172,22 @@ __device__ __forceinline__ void fence_acq_rel() {
 __device__ void grid_barrier(const LayerParams& p, int n) {
   named_bar_sync(BAR_ALL, CW * 32);
   if (threadIdx.x == 0) {
-    fence_acq_rel();
-    atomicAdd(p.bar, 1);
-    const int target = n * (int)gridDim.x;
-    if (ld_acquire(p.bar) < target) {
-      const bool gave_up =
-          *reinterpret_cast<volatile int32_t*>(p.err) == MOE_ERR_TIMEOUT;
-      const uint64_t t0 = globaltimer();
-      while (!gave_up && ld_acquire(p.bar) < target) {
-        if (globaltimer() - t0 > 500000000ull) {
-          set_err(p.err, MOE_ERR_TIMEOUT);
-          break;
-        }
-        __nanosleep(32);
-      }
-    }
-    fence_acq_rel();
+    // the block's writes (ordered before this thread by the bar.sync) are
+    // released with the arrival
+    red_release_add(p.bar, 1);
+    spin_until(p.bar, n * (int)gridDim.x, p.err);
   }
+  named_bar_sync(BAR_ALL, CW * 32);
+}
+// The same barrier in two halves: the arrival (called by one thread after
+// a __syncthreads that orders the block's writes before it; its release
+// may take a while, so it is made by a warp with nothing else to do),
+// other work, then the wait.
+__device__ void grid_arrive(const LayerParams& p) {
+  red_release_add(p.bar, 1);
+}
+__device__ void grid_wait(const LayerParams& p, int n) {
+  if (threadIdx.x == 0) spin_until(p.bar, n * (int)gridDim.x, p.err);
   named_bar_sync(BAR_ALL, CW * 32);
 }
 
@@ -234,6 +252,29 @@ __global__ void __launch_bounds__(LAYER_THREADS, 1)
   }
   if (tid < DEC_TMAX) M.xmax[tid] = 0u;
   for (int i = tid; i < MAXP; i += LAYER_THREADS) M.up_fin[i] = 0;
+  // router rows of this block (not in DL_FFN): four warps per row, each a
+  // quarter of H; the first row chunk of every warp is loaded before x is
+  // staged, so that the two loads overlap
+  constexpr int RQ = 4, RCH = 4;
+  const bool route = p.mode != DL_FFN;
+  const int e0 = (int)((int64_t)E * blockIdx.x / G);
+  const int e1 = (int)((int64_t)E * (blockIdx.x + 1) / G);
+  const int nrow = e1 - e0;
+  const int nch = H / 8, qch = (nch + RQ - 1) / RQ;
+  uint4 wpre[RCH];
+  {
+    const int r = warp / RQ, q = warp % RQ;
+    const uint4* row =
+        reinterpret_cast<const uint4*>(p.wr + (int64_t)(e0 + r) * H);
+#pragma unroll
+    for (int i = 0; i < RCH; ++i) {
+      const int ch = q * qch + lane + 32 * i;
+      wpre[i] = (route && warp < CW && r < nrow && ch < (q + 1) * qch &&
+                 ch < nch)
+                    ? __ldg(row + ch)
+                    : make_uint4(0, 0, 0, 0);
+    }
+  }
   uint16_t* xs = reinterpret_cast<uint16_t*>(ring);   // [T][H] bf16
   if (p.x) {
     for (int i = tid; i < T * H / 8; i += LAYER_THREADS)
@@ -253,18 +294,11 @@ __global__ void __launch_bounds__(LAYER_THREADS, 1)
   if (blockIdx.x == 0)
     for (int i = tid; i < T * k; i += LAYER_THREADS) p.hmax[i] = 0u;
   __syncthreads();
-  // router rows of this block (not in DL_FFN): four warps per row, each a
-  // quarter of H;
   // a lane issues all its loads of the row first (up to RCH 16-byte
   // chunks), then accumulates in fp32; lane sums by a fixed butterfly and
   // the quarters in fixed order (deterministic)
-  if (p.mode != DL_FFN) {
-    constexpr int RQ = 4, RCH = 4;
+  if (route) {
     float* part = reinterpret_cast<float*>(smem + L.red);   // [rows][RQ][T]
-    const int e0 = (int)((int64_t)E * blockIdx.x / G);
-    const int e1 = (int)((int64_t)E * (blockIdx.x + 1) / G);
-    const int nrow = e1 - e0;
-    const int nch = H / 8, qch = (nch + RQ - 1) / RQ;
     for (int base = 0; base < nrow; base += CW / RQ) {
       const int r = base + warp / RQ, q = warp % RQ;
       if (warp < CW && r < nrow) {
@@ -275,11 +309,13 @@ __global__ void __launch_bounds__(LAYER_THREADS, 1)
         for (int t = 0; t < TM; ++t) acc[t] = 0.f;
         for (int c0 = q * qch; c0 < (q + 1) * qch && c0 < nch; c0 += 32 * RCH) {
           uint4 w[RCH];
+          const bool pre = base == 0 && c0 == q * qch;
 #pragma unroll
           for (int i = 0; i < RCH; ++i) {
             const int ch = c0 + lane + 32 * i;
-            w[i] = (ch < (q + 1) * qch && ch < nch) ? __ldg(row + ch)
-                                                   : make_uint4(0, 0, 0, 0);
+            w[i] = pre ? wpre[i]
+                       : (ch < (q + 1) * qch && ch < nch) ? __ldg(row + ch)
+                                                          : make_uint4(0, 0, 0, 0);
           }
 #pragma unroll
           for (int i = 0; i < RCH; ++i) {
@@ -325,18 +361,15 @@ __global__ void __launch_bounds__(LAYER_THREADS, 1)
   __syncthreads();
 
   // ------------------------------------------------------------- P0|P1 --
-  if (warp < CW) grid_barrier(p, 1);
-
-  // ---------------------------------------------------------------- P1 --
+  if (warp == SIGNALER && lane == 0) grid_arrive(p);
   if (warp < CW) {
-    if (warp >= T) {
-      // the warps without a top-k: per-token activation scale, then the
-      // int8 hi/lo B fragments of x
-      const int xt = tid - T * 32, xn = (CW - T) * 32;
+    if (p.mode != DL_ROUTE) {
+      // per-token activation scale, then the int8 hi/lo B fragments of x
+      // (all compute warps, while the other blocks finish their logits)
+      const int xt = tid, xn = CW * 32;
       float m[TM];
 #pragma unroll
       for (int t = 0; t < TM; ++t) m[t] = 0.f;
-      const int nch = H / 8;
       for (int i = xt; i < T * nch; i += xn) {
         const int t = i / nch;
         const uint4 v = reinterpret_cast<const uint4*>(xs)[i];
@@ -391,6 +424,11 @@ __global__ void __launch_bounds__(LAYER_THREADS, 1)
         reinterpret_cast<uint2*>(frag)[i] = wv;
       }
     }
+    grid_wait(p, 1);
+  }
+
+  // ---------------------------------------------------------------- P1 --
+  if (warp < CW) {
     if (warp < T && p.mode == DL_FFN) {
       // the caller's top-k (as a DL_ROUTE launch wrote it)
       const int t = warp;
@@ -707,22 +745,7 @@ __global__ void __launch_bounds__(LAYER_THREADS, 1)
   const int hwords = (F / 32) * NT * 64;      // words per expert
   {
     // wait until every up unit of this block's down experts is done
-    if (tid < nexp) {
-      const int32_t* cnt = p.up_done + uf + tid;
-      if (ld_acquire(cnt) < nrt_f) {
-        const bool gave_up =
-            *reinterpret_cast<volatile int32_t*>(p.err) == MOE_ERR_TIMEOUT;
-        const uint64_t t0 = globaltimer();
-        while (!gave_up && ld_acquire(cnt) < nrt_f) {
-          if (globaltimer() - t0 > 500000000ull) {
-            set_err(p.err, MOE_ERR_TIMEOUT);
-            break;
-          }
-          __nanosleep(32);
-        }
-      }
-      fence_acq_rel();
-    }
+    if (tid < nexp) spin_until(p.up_done + uf + tid, nrt_f, p.err);
     named_bar_sync(BAR_ALL, CW * 32);
     if (tid < 16) {
       const int b = tid >> 3, sl = tid & 7;
@@ -780,6 +803,7 @@ __global__ void __launch_bounds__(LAYER_THREADS, 1)
       float acc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
       if (have && b >= 0 && b < nexp) {
         const uint8_t* unit = ring + s * L.slot_bytes + dg * dnb;
+#pragma unroll 4
         for (int kt = kt0; kt < kt1; ++kt)
           piece_b32<FDN>(unit + kt * B32_TILE_BYTES,
                          frag + b * hwords + (2 * kt) * NT * 64, NT,

@@ -108,9 +108,12 @@ __device__ __forceinline__ void piece_b32(const uint8_t* tp,
       if (nt < NT) {
         const uint2 b = *reinterpret_cast<const uint2*>(
             bfb + (bl * bnt + nt) * 64 + 2 * lane);
-        int32_t d[4];
+        // the two table halves as independent products (exact int32 sum)
+        int32_t d[4], e[4];
         mma_s8(d, a1, b.x, b.y, zero);
-        mma_s8(d, a2, b.x, b.y, d);
+        mma_s8(e, a2, b.x, b.y, zero);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) d[q] += e[q];
         const float c = cs[bl * cs_stride + 4 * nt];
         acc[nt][0] = fmaf((float)(d[0] * 256 + d[1]), d0 * c, acc[nt][0]);
         acc[nt][1] = fmaf((float)(d[2] * 256 + d[3]), d8 * c, acc[nt][1]);
