@@ -745,7 +745,7 @@ def run_stack(args) -> None:
     print(json.dumps(line), flush=True)
 
 
-PF_LAUNCHES_PER_STEP = 10   # route 2, group 3, x16 + plan + up, down, combine
+PF_LAUNCHES_PER_STEP = 11   # route 2, group 3, pair rows + x16 + plan + up, down, combine
 
 
 def run_prefill(args) -> None:
