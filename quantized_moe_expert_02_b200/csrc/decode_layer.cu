@@ -537,8 +537,33 @@ __global__ void __launch_bounds__(LAYER_THREADS, 1)
   // experts per block)
   const int b0 = blockIdx.x;
   const int n_up = nu_all > b0 ? (nu_all - 1 - b0) / G + 1 : 0;
-  const int d0 = (int)((int64_t)nd_all * blockIdx.x / G);
-  const int d1 = (int)((int64_t)nd_all * (blockIdx.x + 1) / G);
+  // Down ranges are dealt in reverse block order and sized so that each
+  // block's work is about even, counting an up unit as four down units
+  // (their bytes) and the extra up unit of the first nu_all % G blocks as
+  // eight: those blocks also take the last experts' down units, whose up
+  // units are the last to finish, so they wait for them before their down
+  // phase.  Plain even split when that weighting does not fit (ranges must
+  // stay within two experts).
+  int d0, d1;
+  {
+    const int q_up = nu_all / G, extra = nu_all % G;
+    const int64_t ctot = 4LL * q_up * G + 8LL * extra + nd_all;
+    const bool weighted = (4LL * q_up + 8) * G <= ctot &&
+                          (ctot + G - 1) / G - 4LL * q_up <= nrt_h;
+    if (weighted) {
+      auto before = [&](int pos) -> int {   // down units of positions < pos
+        const int64_t up = 4LL * pos * q_up +
+                           8LL * (pos > G - extra ? pos - (G - extra) : 0);
+        return (int)(((int64_t)pos * ctot - (int64_t)G * up) / G);
+      };
+      const int pos = G - 1 - b0;
+      d0 = before(pos);
+      d1 = before(pos + 1);
+    } else {
+      d0 = (int)((int64_t)nd_all * b0 / G);
+      d1 = (int)((int64_t)nd_all * (b0 + 1) / G);
+    }
+  }
   const int dnb = dn_unit_bytes(F);
   int dps = L.slot_bytes / dnb;                // down units per slot
   if (dps > DNG) dps = DNG;
