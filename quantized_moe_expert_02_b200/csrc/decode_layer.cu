@@ -252,6 +252,10 @@ __global__ void __launch_bounds__(LAYER_THREADS, 1)
   }
   if (tid < DEC_TMAX) M.xmax[tid] = 0u;
   for (int i = tid; i < MAXP; i += LAYER_THREADS) M.up_fin[i] = 0;
+  // launched as a programmatic dependent of the previous kernel on the
+  // stream: nothing in global memory is touched before that kernel is
+  // complete and its writes are visible
+  grid_dep_wait();
   // router rows of this block (not in DL_FFN): four warps per row, each a
   // quarter of H; the first row chunk of every warp is loaded before x is
   // staged, so that the two loads overlap
@@ -862,6 +866,9 @@ __global__ void __launch_bounds__(LAYER_THREADS, 1)
   }
 
   grid_barrier(p, 2);
+  // the next kernel on the stream may start its launch (it waits for this
+  // one to finish before it reads or writes global memory)
+  grid_dep_launch();
 
   // P5: combine (not in DL_ROUTE), then the exit count that re-arms the
   // grid barrier
@@ -981,11 +988,13 @@ moe_status launch_decode_layer(const moe_layer_desc& d, const uint16_t* x,
   cfg.blockDim = dim3(LAYER_THREADS);
   cfg.dynamicSmemBytes = (size_t)L.total;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeCooperative;
   attr[0].val.cooperative = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   MOE_CUDA_TRY(cudaLaunchKernelEx(&cfg, kern, p));
   return MOE_OK;
 }
