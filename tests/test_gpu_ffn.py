@@ -73,9 +73,18 @@ def test_expert_ffn_vs_oracle(shape, T):
     assert row_max_rel(out2.cpu().numpy(), ref_out) <= TOL
 
 
+# 1024 experts top-8 (the wide top-k of the one-kernel layer: 32 keys per
+# lane), SB3 up/gate and NL4 down at a small hidden size
+WIDE = synth.LayerShape(H=512, F=256, E=1024, k=8,
+                        fmt_up_gate=synth.SB3_256, fmt_down=synth.NL4_B32,
+                        d_up_gate=(0.002, 0.01), d_down=(0.002, 0.01))
+
+
 @pytest.mark.parametrize("shape,T,zipf", [
     (synth.TINY, 8, False), (synth.BIG, 1, False), (synth.BIG, 3, False),
     (synth.BIG, 3, True), (synth.TINY, 16, False),
+    (synth.BIG, 2, False), (synth.BIG, 5, False), (synth.BIG, 8, True),
+    (WIDE, 3, False), (WIDE, 7, True),
 ])
 def test_layer_forward_vs_oracle(shape, T, zipf):
     pool = pool_for(shape)
