@@ -296,14 +296,16 @@ class Layers:
         self.bufs[T] = b
         return b
 
-    def step(self, T: int, i: int, x=None):
-        """One decode layer through the C ABI (5 kernels)."""
+    def step(self, T: int, i: int, x=None, out=None):
+        """One decode layer through the C ABI (one launch)."""
         b, shp = self.buffers(T), synth.BIG
         l = i % self.L
         xx = b["xs"][i % self.n_x] if x is None else x
         self.moe.moe_layer_forward(self.descs[l], xx, T, shp.k, self.wr[l],
-                                   None, None, None, b["out"], None, b["idx"],
-                                   b["w"], None, b["ws"], b["ws_bytes"])
+                                   None, None, None,
+                                   b["out"] if out is None else out, None,
+                                   b["idx"], b["w"], None, b["ws"],
+                                   b["ws_bytes"])
 
     def unique_experts(self, T: int, i: int) -> int:
         """Distinct experts of step i (untimed: routing only)."""
@@ -331,6 +333,137 @@ def graph_time(steps: int, warmup: int, fn, per_graph: int) -> float:
         with torch.cuda.graph(g):
             for i in range(n):
                 fn(warmup + i)
+        graphs.append((g, reps))
+    for g, _ in graphs:
+        g.replay()
+    torch.cuda.synchronize()
+    s = torch.cuda.current_stream()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    for g, reps in graphs:
+        for _ in range(reps):
+            g.replay()
+    e1.record(s)
+    e1.synchronize()
+    ms = e0.elapsed_time(e1)
+    del graphs
+    return ms
+
+
+def prefill_e2e_time(pf, steps: int, warmup: int) -> float:
+    """Device time (ms) per prefill step end to end through the C ABI:
+    every step copies its x (9536 x 3072 bf16) from pinned host memory and
+    its output (fp32) back to pinned host memory, on two copy streams
+    beside the layer launches (x of step i+1 goes up while step i computes,
+    the output of step i comes back while step i+1 computes)."""
+    import torch
+    H = synth.BIG.H
+    xh = [torch.from_numpy(synth.gen_x(0, pf.T, H, s).view(np.int16))
+          .pin_memory() for s in range(2)]
+    oh = [torch.empty((pf.T, H), dtype=torch.float32).pin_memory()
+          for _ in range(2)]
+    xd = [torch.empty((pf.T, H), dtype=torch.int16, device="cuda")
+          for _ in range(2)]
+    od = [torch.empty((pf.T, H), device="cuda") for _ in range(2)]
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
+    cur = torch.cuda.current_stream()
+
+    def run(n: int):
+        up.wait_stream(cur)
+        down.wait_stream(cur)
+        ev_in, ev_k, ev_out = {}, {}, {}
+        for j in range(n):
+            b = j % 2
+            with torch.cuda.stream(up):
+                if j >= 2:
+                    up.wait_event(ev_k[j - 2])
+                xd[b].copy_(xh[b], non_blocking=True)
+                ev_in[j] = torch.cuda.Event()
+                ev_in[j].record(up)
+            cur.wait_event(ev_in[j])
+            if j >= 2:
+                cur.wait_event(ev_out[j - 2])
+            pf.step(x=xd[b], out=od[b])
+            ev_k[j] = torch.cuda.Event()
+            ev_k[j].record(cur)
+            with torch.cuda.stream(down):
+                down.wait_event(ev_k[j])
+                oh[b].copy_(od[b], non_blocking=True)
+                ev_out[j] = torch.cuda.Event()
+                ev_out[j].record(down)
+        cur.wait_stream(up)
+        cur.wait_stream(down)
+
+    run(warmup)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(cur)
+    run(steps)
+    e1.record(cur)
+    e1.synchronize()
+    return e0.elapsed_time(e1) / steps
+
+
+def e2e_time(lay, T: int, steps: int, warmup: int) -> float:
+    """Device time (ms) of `steps` decode steps end to end through the C
+    ABI: every step copies its x from pinned host memory to the device and
+    its output back to pinned host memory.  The copies run on two copy
+    streams beside the layer launches (x of step i+1 goes up while step i
+    computes; the output of step i comes back while step i+1 computes),
+    with double-buffered device x and output.  Replayed from CUDA graphs of
+    32 steps."""
+    import torch
+    H = synth.BIG.H
+    nh = lay.L * 4
+    xh = [torch.from_numpy(synth.gen_x(0, T, H, s).view(np.int16))
+          .pin_memory() for s in range(nh)]
+    oh = [torch.empty((T, H), dtype=torch.float32).pin_memory()
+          for _ in range(nh)]
+    xd = [torch.empty((T, H), dtype=torch.int16, device="cuda")
+          for _ in range(2)]
+    od = [torch.empty((T, H), device="cuda") for _ in range(2)]
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
+
+    def body(i0: int, n: int):
+        cur = torch.cuda.current_stream()
+        up.wait_stream(cur)
+        down.wait_stream(cur)
+        ev_in, ev_k, ev_out = {}, {}, {}
+        for j in range(n):
+            i, b = i0 + j, j % 2
+            with torch.cuda.stream(up):
+                if j >= 2:
+                    up.wait_event(ev_k[j - 2])      # step j-2 read xd[b]
+                xd[b].copy_(xh[i % nh], non_blocking=True)
+                ev_in[j] = torch.cuda.Event()
+                ev_in[j].record(up)
+            cur.wait_event(ev_in[j])
+            if j >= 2:
+                cur.wait_event(ev_out[j - 2])       # od[b] is back on host
+            lay.step(T, i, x=xd[b], out=od[b])
+            ev_k[j] = torch.cuda.Event()
+            ev_k[j].record(cur)
+            with torch.cuda.stream(down):
+                down.wait_event(ev_k[j])
+                oh[i % nh].copy_(od[b], non_blocking=True)
+                ev_out[j] = torch.cuda.Event()
+                ev_out[j].record(down)
+        cur.wait_stream(up)
+        cur.wait_stream(down)
+
+    body(0, max(warmup, 2))
+    torch.cuda.synchronize()
+    G = min(32, steps)
+    full, rem = divmod(steps, G)
+    graphs = []
+    for n, reps in ((G, full), (rem, 1 if rem else 0)):
+        if not reps:
+            continue
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            body(warmup, n)
         graphs.append((g, reps))
     for g, _ in graphs:
         g.replay()
@@ -428,12 +561,13 @@ class Prefill:
                                device="cuda")
         self.y = torch.empty((T * k, H), device="cuda")
 
-    def step(self, x=None):
+    def step(self, x=None, out=None):
         shp = synth.BIG
         self.moe.moe_layer_forward(self.desc, self.x if x is None else x,
                                    self.T, shp.k, self.wr, self.bias, None,
-                                   None, self.out, None, self.idx, self.w,
-                                   self.lg, self.ws, self.ws_bytes)
+                                   None, self.out if out is None else out,
+                                   None, self.idx, self.w, self.lg, self.ws,
+                                   self.ws_bytes)
 
     def piece_fns(self):
         moe, shp, T = self.moe, synth.BIG, self.T
@@ -560,20 +694,7 @@ def run_ours(args) -> None:
         hbm, tf, src = peaks()
         kt = kernel_timing(lay, T, 64, 4)
         k_gbs = bytes_step / (kt * 1e-3) / 1e9
-        # end to end: x from pinned host memory in, the output back to
-        # pinned host memory, every step, through the C ABI
-        bufs = lay.buffers(T)
-        xh = [torch.from_numpy(synth.gen_x(0, T, 3072, s).view(np.int16))
-              .pin_memory() for s in range(lay.L * 4)]
-        xd = torch.empty((T, 3072), dtype=torch.int16, device="cuda")
-        oh = [torch.empty((T, 3072), dtype=torch.float32).pin_memory()
-              for _ in range(lay.L * 4)]
-
-        def e2e_step(i):
-            xd.copy_(xh[i % len(xh)], non_blocking=True)
-            lay.step(T, i, x=xd)
-            oh[i % len(oh)].copy_(bufs["out"], non_blocking=True)
-        ms_e2e = graph_time(K, W, e2e_step, per_graph=lay.L * 4)
+        ms_e2e = e2e_time(lay, T, K, W)
         t1, _ = decode_measure(lay, 1, K, W)
         line = {
             "metric": METRIC, "value": tok_s, "unit": "tokens/s",
@@ -787,17 +908,7 @@ def run_prefill(args) -> None:
         m = prefill_measure(pf, max(3, min(K, 10)), 2)
         fl = prefill_flops(pf.T)
         up_ms = m["parts_ms"]["up"]
-        # end to end: x in from pinned host memory, out back, every step
-        xh = torch.from_numpy(synth.gen_x(0, pf.T, 3072, 0).view(np.int16)) \
-            .pin_memory()
-        xd = torch.empty((pf.T, 3072), dtype=torch.int16, device="cuda")
-        oh = torch.empty((pf.T, 3072), dtype=torch.float32).pin_memory()
-
-        def e2e():
-            xd.copy_(xh, non_blocking=True)
-            pf.step(x=xd)
-            oh.copy_(pf.out, non_blocking=True)
-        ms_e2e = events_time(e2e, max(3, min(K, 10)), 2)
+        ms_e2e = prefill_e2e_time(pf, max(3, min(K, 10)), 2)
         line = {
             "metric": METRIC, "value": pf.T * K * world / (ms / 1e3),
             "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W,
