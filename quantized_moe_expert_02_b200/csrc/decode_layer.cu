@@ -308,9 +308,10 @@ __global__ void __launch_bounds__(LAYER_THREADS, 1)
       if (warp < CW && r < nrow) {
         const uint4* row =
             reinterpret_cast<const uint4*>(p.wr + (int64_t)(e0 + r) * H);
-        float acc[TM];
+        float acc[TM], xm[TM];   // xm: max |x_t| over this quarter (row 0)
 #pragma unroll
-        for (int t = 0; t < TM; ++t) acc[t] = 0.f;
+        for (int t = 0; t < TM; ++t) acc[t] = xm[t] = 0.f;
+        const bool track = base == 0 && r == 0;
         for (int c0 = q * qch; c0 < (q + 1) * qch && c0 < nch; c0 += 32 * RCH) {
           uint4 w[RCH];
           const bool pre = base == 0 && c0 == q * qch;
@@ -340,6 +341,15 @@ __global__ void __launch_bounds__(LAYER_THREADS, 1)
                            __uint_as_float(xw[qq] & 0xFFFF0000u), a);
                 }
                 acc[t] = a;
+                if (track) {
+                  float m = xm[t];
+#pragma unroll
+                  for (int qq = 0; qq < 4; ++qq)
+                    m = fmaxf(m, fmaxf(fabsf(__uint_as_float(xw[qq] << 16)),
+                                       fabsf(__uint_as_float(xw[qq] &
+                                                             0xFFFF0000u))));
+                  xm[t] = m;
+                }
               }
             }
           }
@@ -350,6 +360,13 @@ __global__ void __launch_bounds__(LAYER_THREADS, 1)
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
           if (lane == 0 && t < T) part[(r * RQ + q) * DEC_TMAX + t] = a;
+          if (track) {
+            float m = xm[t];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1)
+              m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+            if (lane == 0 && t < T) atomicMax(&M.xmax[t], __float_as_uint(m));
+          }
         }
       }
     }
@@ -367,9 +384,8 @@ __global__ void __launch_bounds__(LAYER_THREADS, 1)
   // ------------------------------------------------------------- P0|P1 --
   if (warp == SIGNALER && lane == 0) grid_arrive(p);
   if (warp < CW) {
-    if (p.mode != DL_ROUTE) {
-      // per-token activation scale, then the int8 hi/lo B fragments of x
-      // (all compute warps, while the other blocks finish their logits)
+    if (p.mode != DL_ROUTE && !(route && nrow > 0)) {
+      // max |x_t| (the router's row-0 warps found it when they ran)
       const int xt = tid, xn = CW * 32;
       float m[TM];
 #pragma unroll
@@ -396,7 +412,16 @@ __global__ void __launch_bounds__(LAYER_THREADS, 1)
           a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
         if (lane == 0 && t < T) atomicMax(&M.xmax[t], __float_as_uint(a));
       }
-      named_bar_sync(BAR_XF, xn);
+    }
+    grid_wait(p, 1);
+  }
+
+  // ---------------------------------------------------------------- P1 --
+  if (warp < CW) {
+    if (warp >= T && p.mode != DL_ROUTE) {
+      // the warps without a top-k: per-token activation scale, then the
+      // int8 hi/lo B fragments of x
+      const int xt = tid - T * 32, xn = (CW - T) * 32;
       if (xt < T) {
         const int sg = pow2_sigma(__uint_as_float(M.xmax[xt]));
         M.xsig[xt] = sg;
@@ -428,11 +453,6 @@ __global__ void __launch_bounds__(LAYER_THREADS, 1)
         reinterpret_cast<uint2*>(frag)[i] = wv;
       }
     }
-    grid_wait(p, 1);
-  }
-
-  // ---------------------------------------------------------------- P1 --
-  if (warp < CW) {
     if (warp < T && p.mode == DL_FFN) {
       // the caller's top-k (as a DL_ROUTE launch wrote it)
       const int t = warp;
