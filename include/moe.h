@@ -277,14 +277,17 @@ moe_status moe_rmsnorm_bf16(const float* r, int T, int H, uint16_t* x_out,
 /* Workspace of moe_layer_forward. */
 size_t moe_layer_workspace_bytes(int T, int k, int E, int H, int F);
 
-/* One whole MoE layer: moe_route_topk, moe_group_tokens, then the fused
- * expert FFN + combine, on one stream (the decode kernels when T <= 8 and
- * T*k is at most the SM count, the general path otherwise).  The grouping
- * lives in the workspace.  w_router bf16 [E x H]; bias fp32 [E] or NULL;
- * blob_index as in moe_expert_ffn_q; residual/out/out_bf16 as in
- * moe_combine; topk_idx int32 [T x k], topk_w fp32 [T x k] and logits_out
- * fp32 [T x E] (or NULL) receive the routing.  The decode kernels are
- * chained with programmatic dependent launch. */
+/* One whole MoE layer on one stream: routing, grouping, expert FFN and
+ * the weighted combine.  T <= 8 (with T*k at most the SM count and
+ * E <= 1024): one cooperative kernel does all of it; it is launched as a
+ * programmatic dependent of the work before it on the stream and touches
+ * no global memory until that work has completed, so stream order holds as
+ * usual.  Otherwise: moe_route_topk, moe_group_tokens, then the expert FFN
+ * (the tensor-core prefill path when T > 8 and the shapes allow it) and
+ * the combine.  The grouping lives in the workspace.  w_router bf16
+ * [E x H]; bias fp32 [E] or NULL; blob_index as in moe_expert_ffn_q;
+ * residual/out/out_bf16 as in moe_combine; topk_idx int32 [T x k], topk_w
+ * fp32 [T x k] and logits_out fp32 [T x E] (or NULL) receive the routing. */
 moe_status moe_layer_forward(const moe_layer_desc* desc, const uint16_t* x,
                              int T, int k, const uint16_t* w_router,
                              const float* bias, const int32_t* blob_index,
