@@ -654,6 +654,23 @@ def run_profile(args) -> None:
     print("profile run done", flush=True)
 
 
+def max_over_ranks(ms: float, dist, device: str) -> float:
+    """The job's time: the largest of the ranks' device times (every rank
+    calls this at the same point; a no-op for one process)."""
+    if dist is None:
+        return ms
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(units_per_rank: float, world: int, ms: float) -> float:
+    """Whole-job throughput: the units all ranks processed (replicas, so
+    each did the same) over the job's time in ms."""
+    return units_per_rank * world / (ms / 1e3)
+
+
 def run_ours(args) -> None:
     import torch
     rank = int(os.environ.get("RANK", "0"))
@@ -682,11 +699,8 @@ def run_ours(args) -> None:
     clk.start()
     ms = graph_time(K, W, lambda i: lay.step(T, i), per_graph=lay.L * 4)
     clocks = clk.stop()
-    if dist:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    tok_s = T * K * world / (ms / 1e3)
+    ms = max_over_ranks(ms, dist, "cuda")
+    tok_s = job_rate(T * K, world, ms)
     bytes_step = WR_BYTES + u_avg * BLOB + T * 3072 * 6
 
     line = None
@@ -902,10 +916,7 @@ def run_prefill(args) -> None:
     clk.start()
     ms = events_time(pf.step, K, 0) * K
     clocks = clk.stop()
-    if dist:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, dist, "cuda")
     line = None
     if rank == 0:
         hbm, tf, src = peaks()
@@ -914,7 +925,7 @@ def run_prefill(args) -> None:
         up_ms = m["parts_ms"]["up"]
         ms_e2e = prefill_e2e_time(pf, max(3, min(K, 10)), 2)
         line = {
-            "metric": METRIC, "value": pf.T * K * world / (ms / 1e3),
+            "metric": METRIC, "value": job_rate(pf.T * K, world, ms),
             "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W,
             "ms_per_step": ms / K, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None,
