@@ -87,7 +87,8 @@ class SlotPool:
     """
 
     def __init__(self, stack: Stack, capacities: Sequence[int],
-                 store_keys: Optional[Sequence[Tuple[int, int]]]):
+                 store_keys: Optional[Sequence[Tuple[int, int]]],
+                 copy_streams: int = 2):
         torch, moe, shp = stack.torch, stack.moe, stack.shape
         self.stack, self.torch, self.moe = stack, torch, moe
         self.caps = [int(c) for c in capacities]
@@ -138,6 +139,9 @@ class SlotPool:
         self.err = torch.zeros(1, dtype=torch.int32, device="cuda")
         self.h_n = torch.zeros(1 + 2 * P, dtype=torch.int32).pin_memory()
         self.misses = 0
+        # host-store copies are spread over these streams (half a blob per
+        # copy), so that more than one copy engine moves them
+        self.copy_streams = [torch.cuda.Stream() for _ in range(copy_streams)]
 
     def layer(self, l: int, r, stamp: int, log: Optional[List] = None):
         """One layer through the slot pool, in place."""
@@ -160,6 +164,12 @@ class SlotPool:
         n = int(self.h_n[0])
         me = self.h_n[1:1 + n].tolist()
         ms = self.h_n[1 + P:1 + P + n].tolist()
+        cur = torch.cuda.current_stream()
+        side = self.copy_streams if (n and not self.device_source) else []
+        for cs in side:
+            cs.wait_stream(cur)
+        half = (self.blob // 2 + 255) // 256 * 256
+        j = 0
         for e, s in zip(me, ms):
             dst = (int(self.base[l]) + s) * self.stride
             if self.device_source:
@@ -169,8 +179,13 @@ class SlotPool:
                     st.pools[l][src:src + self.blob], non_blocking=True)
             else:
                 i = self.store_index[(l, e)]
-                self.pool[dst:dst + self.blob].copy_(self.store[i],
-                                                     non_blocking=True)
+                for a, b in ((0, half), (half, self.blob)):
+                    with torch.cuda.stream(side[j % len(side)]):
+                        self.pool[dst + a:dst + b].copy_(self.store[i][a:b],
+                                                         non_blocking=True)
+                    j += 1
+        for cs in side:
+            cur.wait_stream(cs)
         self.misses += n
         if log is not None:
             log.append((l, stamp, me, ms))
