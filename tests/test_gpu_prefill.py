@@ -218,3 +218,33 @@ def test_prefill_layer_full_size_sampled():
     ref = o.moe_layer(xs, o.bf16_to_f64(wr), bias, k, src,
                       topk_idx=got_idx[toks])
     assert row_max_rel(got[toks], ref["out"]) <= TOL
+
+
+def test_prefill_past_int32_elements_sampled():
+    """70,000 tokens x top-10: y_pairs holds 700,000 x 3072 > 2^31 fp32
+    elements and x_g 4.3 GB, so every pair/row index of the prefill path
+    needs 64-bit arithmetic.  Sampled tokens against the oracle; the last
+    token's rows sit past element 2^31."""
+    shape = synth.BIG
+    T = 70000
+    k, E, H = shape.k, shape.E, shape.H
+    assert T * k * H > 2 ** 31
+    desc = layer_desc(shape, pool_for(shape))
+    x, wr, bias = route_inputs(shape, 0, 0, T, step=9, zipf=True)
+    ws = Ws(moe.moe_layer_workspace_bytes(T, k, E, H, shape.F))
+    idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, k), device="cuda")
+    out = torch.empty((T, H), device="cuda")
+    moe.moe_layer_forward(desc, dev(x), T, k, dev(wr), dev(bias), None, None,
+                          out, None, idx, w, None, ws.t, ws.nbytes)
+    assert moe.moe_get_device_status(ws.t) == 0
+    toks = [0, T // 2, T - 2, T - 1]
+    got_idx = idx[toks].cpu().numpy()
+    src = oracle_experts(shape, 0, 0)
+    ref = o.moe_layer(o.bf16_to_f64(x[toks]), o.bf16_to_f64(wr), bias, k,
+                      src, topk_idx=got_idx)
+    got = out[toks].cpu().numpy()
+    assert np.isfinite(got).all()
+    assert row_max_rel(got, ref["out"]) <= TOL
+    del ws
+    torch.cuda.empty_cache()
