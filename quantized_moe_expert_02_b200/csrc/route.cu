@@ -120,8 +120,8 @@ __global__ void __launch_bounds__(128)
   float* my = sl + (size_t)warp * E;
   for (int e = lane; e < E; e += 32) my[e] = logits[(int64_t)t * E + e];
   __syncwarp();
-  float sel_v[32];
-  int sel_i[32];
+  float my_v = 0.f;   // lane r keeps round r's winner
+  int my_i = 0;
   for (int r = 0; r < k; ++r) {
     float bv = -FLT_MAX;
     int bi = 0x7fffffff;
@@ -135,20 +135,18 @@ __global__ void __launch_bounds__(128)
       const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
       if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
     }
-    sel_v[r] = bv;
-    sel_i[r] = bi;
+    if (lane == r) { my_v = bv; my_i = bi; }
     if (lane == 0 && bi < E) my[bi] = -INFINITY;
     __syncwarp();
   }
-  if (lane == 0) {
-    const float m = sel_v[0];
-    float ex[32];
-    float s = 0.f;
-    for (int r = 0; r < k; ++r) { ex[r] = expf(sel_v[r] - m); s += ex[r]; }
-    for (int r = 0; r < k; ++r) {
-      topk_idx[(int64_t)t * k + r] = sel_i[r];
-      topk_w[(int64_t)t * k + r] = ex[r] / s;
-    }
+  // weights: exp(l_r - l_0) summed in round order, as a serial loop would
+  const float m = __shfl_sync(0xffffffffu, my_v, 0);
+  const float ex = lane < k ? expf(my_v - m) : 0.f;
+  float s = 0.f;
+  for (int r = 0; r < k; ++r) s += __shfl_sync(0xffffffffu, ex, r);
+  if (lane < k) {
+    topk_idx[(int64_t)t * k + lane] = my_i;
+    topk_w[(int64_t)t * k + lane] = ex / s;
   }
 }
 
