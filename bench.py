@@ -412,8 +412,8 @@ def e2e_time(lay, T: int, steps: int, warmup: int) -> float:
     its output back to pinned host memory.  The copies run on two copy
     streams beside the layer launches (x of step i+1 goes up while step i
     computes; the output of step i comes back while step i+1 computes),
-    with double-buffered device x and output.  Replayed from CUDA graphs of
-    32 steps."""
+    with triple-buffered device x and output, so a launch waits only on
+    copies two steps back.  Replayed from CUDA graphs of 32 steps."""
     import torch
     H = synth.BIG.H
     nh = lay.L * 4
@@ -421,9 +421,10 @@ def e2e_time(lay, T: int, steps: int, warmup: int) -> float:
           .pin_memory() for s in range(nh)]
     oh = [torch.empty((T, H), dtype=torch.float32).pin_memory()
           for _ in range(nh)]
+    NB = 3
     xd = [torch.empty((T, H), dtype=torch.int16, device="cuda")
-          for _ in range(2)]
-    od = [torch.empty((T, H), device="cuda") for _ in range(2)]
+          for _ in range(NB)]
+    od = [torch.empty((T, H), device="cuda") for _ in range(NB)]
     up, down = torch.cuda.Stream(), torch.cuda.Stream()
 
     def body(i0: int, n: int):
@@ -432,16 +433,16 @@ def e2e_time(lay, T: int, steps: int, warmup: int) -> float:
         down.wait_stream(cur)
         ev_in, ev_k, ev_out = {}, {}, {}
         for j in range(n):
-            i, b = i0 + j, j % 2
+            i, b = i0 + j, j % NB
             with torch.cuda.stream(up):
-                if j >= 2:
-                    up.wait_event(ev_k[j - 2])      # step j-2 read xd[b]
+                if j >= NB:
+                    up.wait_event(ev_k[j - NB])     # step j-NB read xd[b]
                 xd[b].copy_(xh[i % nh], non_blocking=True)
                 ev_in[j] = torch.cuda.Event()
                 ev_in[j].record(up)
             cur.wait_event(ev_in[j])
-            if j >= 2:
-                cur.wait_event(ev_out[j - 2])       # od[b] is back on host
+            if j >= NB:
+                cur.wait_event(ev_out[j - NB])      # od[b] is back on host
             lay.step(T, i, x=xd[b], out=od[b])
             ev_k[j] = torch.cuda.Event()
             ev_k[j].record(cur)
@@ -453,7 +454,7 @@ def e2e_time(lay, T: int, steps: int, warmup: int) -> float:
         cur.wait_stream(up)
         cur.wait_stream(down)
 
-    body(0, max(warmup, 2))
+    body(0, max(warmup, NB))
     torch.cuda.synchronize()
     G = min(32, steps)
     full, rem = divmod(steps, G)
