@@ -44,12 +44,17 @@ KERNEL_SOURCES = ["quantized_moe_expert_02_b200/csrc/decode_layer.cu",
                   "quantized_moe_expert_02_b200/csrc/moe_internal.cuh"]
 
 
-def captured_traffic(alg_bytes_per_launch: float):
-    """DRAM traffic per launch from the committed ncu capture of the decode
-    kernel, scaled from the captured launch's algorithmic bytes to the
-    bench's average launch; None when the kernel sources changed since."""
+PF_KERNEL_SOURCES = ["quantized_moe_expert_02_b200/csrc/prefill.cu",
+                     "quantized_moe_expert_02_b200/csrc/tc_ptx.cuh",
+                     "quantized_moe_expert_02_b200/csrc/moe_internal.cuh"]
+
+
+def profile_values(name: str, sources):
+    """The `key: value` lines of a committed ncu summary under profiles/,
+    or None when it is missing or the kernel sources changed since it was
+    taken (its source_sha is the sha256 of the sources' digest lines)."""
     import hashlib
-    prof = os.path.join(ROOT, "profiles", "decode_layer_t3.md")
+    prof = os.path.join(ROOT, "profiles", name)
     if not os.path.exists(prof):
         return None
     vals = {}
@@ -58,15 +63,32 @@ def captured_traffic(alg_bytes_per_launch: float):
             k, v = line.split(":", 1)
             vals[k.strip()] = v.strip()
     digests = []
-    for f in KERNEL_SOURCES:
+    for f in sources:
         digests.append(hashlib.sha256(open(os.path.join(ROOT, f), "rb")
                                       .read()).hexdigest() + "  " + f)
     sha = hashlib.sha256(("\n".join(digests) + "\n").encode()).hexdigest()
     if vals.get("source_sha") != sha[:16]:
         return None
+    return vals
+
+
+def captured_traffic(alg_bytes_per_launch: float):
+    """DRAM traffic per launch from the committed ncu capture of the decode
+    kernel, scaled from the captured launch's algorithmic bytes to the
+    bench's average launch; None when the kernel sources changed since."""
+    vals = profile_values("decode_layer_t3.md", KERNEL_SOURCES)
+    if vals is None:
+        return None
     t = float(vals["traffic_bytes_per_launch"])
     a = float(vals["algorithmic_bytes_of_captured_launch"])
     return t * alg_bytes_per_launch / a
+
+
+def captured_traffic_prefill():
+    """DRAM traffic of one up/gate launch of the prefill chunk from the
+    committed ncu capture (same workload); None when stale."""
+    vals = profile_values("pf_gemm_prefill_9536.md", PF_KERNEL_SOURCES)
+    return None if vals is None else float(vals["traffic_bytes_per_launch"])
 
 
 def peaks():
@@ -943,7 +965,7 @@ def run_prefill(args) -> None:
                 "kernel": "pf_gemm_kernel<up, SB3> (up/gate + SwiGLU)",
                 "achieved": m["up_tflops"], "peak": tf, "unit": "TFLOP/s",
                 "frac": m["up_tflops"] / tf, "peak_source": src,
-                "traffic": None,
+                "traffic": captured_traffic_prefill(),
                 "algorithmic_flops_per_launch": fl["up"],
                 "avg_launch_ms": up_ms},
             "prefill": m,
