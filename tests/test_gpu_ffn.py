@@ -80,11 +80,18 @@ WIDE = synth.LayerShape(H=512, F=256, E=1024, k=8,
                         d_up_gate=(0.002, 0.01), d_down=(0.002, 0.01))
 
 
+# 1024 experts top-20: 8 tokens make 160 pairs, more than the SM count and
+# the one-kernel layer's pair limit, so the layer takes the general path
+WIDE20 = synth.LayerShape(H=512, F=256, E=1024, k=20,
+                          fmt_up_gate=synth.SB3_256, fmt_down=synth.NL4_B32,
+                          d_up_gate=(0.002, 0.01), d_down=(0.002, 0.01))
+
+
 @pytest.mark.parametrize("shape,T,zipf", [
     (synth.TINY, 8, False), (synth.BIG, 1, False), (synth.BIG, 3, False),
     (synth.BIG, 3, True), (synth.TINY, 16, False),
     (synth.BIG, 2, False), (synth.BIG, 5, False), (synth.BIG, 8, True),
-    (WIDE, 3, False), (WIDE, 7, True),
+    (WIDE, 3, False), (WIDE, 7, True), (WIDE20, 8, False),
 ])
 def test_layer_forward_vs_oracle(shape, T, zipf):
     pool = pool_for(shape)
