@@ -1,8 +1,10 @@
 """Drivers of the multi-layer decode workloads through the library's C ABI:
 the all-resident residual stack and the same stack over an expert-slot
-pool.  No arithmetic of the layer happens here -- every layer runs in the
-library; this module only owns buffers, builds the device pools with the
-seeded generator, and moves missed expert blobs (one copy per expert).
+pool (misses handled by a host round trip per layer, or in-stream through
+the library's doorbell and stager).  No arithmetic of the layer happens
+here -- every layer runs in the library; this module only owns buffers,
+builds the device pools with the seeded generator, and moves missed expert
+blobs (one copy per expert).
 
 Step semantics (the 48-layer workloads): step s starts from the residual
 r = x_s (the seeded bf16 activations of step s, widened to fp32); each
@@ -100,22 +102,7 @@ class SlotPool:
         self.pool = torch.empty(n_slots * stride, dtype=torch.uint8,
                                 device="cuda")
         E = shp.E
-        self.table, self.owner, self.last = [], [], []
-        for l, cap in enumerate(self.caps):
-            hot = hottest(stack, l, cap)
-            tab = torch.full((E,), -1, dtype=torch.int32, device="cuda")
-            own = torch.full((cap,), -1, dtype=torch.int32, device="cuda")
-            for s, e in enumerate(hot):
-                tab[int(e)] = s
-                own[s] = int(e)
-                dst = (int(self.base[l]) + s) * stride
-                src = int(e) * stride
-                self.pool[dst:dst + self.blob].copy_(
-                    stack.pools[l][src:src + self.blob])
-            self.table.append(tab)
-            self.owner.append(own)
-            self.last.append(torch.zeros(cap, dtype=torch.int32,
-                                         device="cuda"))
+        self.reset()
         self.descs = [layer_desc(shp, self.pool) for _ in self.caps]
         # pinned host store, filled from the resident pools
         self.device_source = store_keys is None
@@ -142,6 +129,28 @@ class SlotPool:
         # host-store copies are spread over these streams (half a blob per
         # copy), so that more than one copy engine moves them
         self.copy_streams = [torch.cuda.Stream() for _ in range(copy_streams)]
+
+    def reset(self) -> None:
+        """The starting state: each layer's slots hold its hottest experts,
+        every last-use stamp is zero."""
+        torch, st, E = self.torch, self.stack, self.stack.shape.E
+        self.table, self.owner, self.last = [], [], []
+        for l, cap in enumerate(self.caps):
+            hot = hottest(st, l, cap)
+            tab = torch.full((E,), -1, dtype=torch.int32, device="cuda")
+            own = torch.full((cap,), -1, dtype=torch.int32, device="cuda")
+            for s, e in enumerate(hot):
+                tab[int(e)] = s
+                own[s] = int(e)
+                dst = (int(self.base[l]) + s) * self.stride
+                src = int(e) * self.stride
+                self.pool[dst:dst + self.blob].copy_(
+                    st.pools[l][src:src + self.blob])
+            self.table.append(tab)
+            self.owner.append(own)
+            self.last.append(torch.zeros(cap, dtype=torch.int32,
+                                         device="cuda"))
+        self.misses = 0
 
     def layer(self, l: int, r, stamp: int, log: Optional[List] = None):
         """One layer through the slot pool, in place."""
@@ -196,4 +205,58 @@ class SlotPool:
     def run(self, r, stamp: int, log: Optional[List] = None):
         for l in range(len(self.caps)):
             self.layer(l, r, stamp, log)
+        return r
+
+    # ----------------------------------------- in-stream doorbell mode --
+    def start_stager(self, timeout_us: int = 2_000_000) -> None:
+        """Miss handling without a host round trip per layer: the layer's
+        misses go to a mapped pinned mailbox (moe_miss_post), the library's
+        stager thread copies them from the host store, and the stream waits
+        on the device (moe_wait_done) before the FFN."""
+        torch, moe = self.torch, self.moe
+        assert not self.device_source, "the doorbell mode needs a host store"
+        L, E = len(self.caps), self.stack.shape.E
+        self.mailbox = torch.zeros(moe.moe_mailbox_bytes(),
+                                   dtype=torch.uint8).pin_memory()
+        self.sync = torch.zeros(2, dtype=torch.int32, device="cuda")
+        table = [0] * (L * E)
+        for (l, e), i in self.store_index.items():
+            table[l * E + e] = self.store[i].data_ptr()
+        self.timeout_us = int(timeout_us)
+        torch.cuda.synchronize()
+        self.stager = moe.moe_stager_create(
+            self.mailbox, self.pool, self.stride, self.blob, table, L, E,
+            self.copy_streams)
+
+    def stop_stager(self) -> Tuple[int, int, int]:
+        """Stops the stager; returns (status, requests, blobs copied)."""
+        self.torch.cuda.synchronize()
+        st, req, cop = self.moe.moe_stager_stats(self.stager)
+        st2 = self.moe.moe_stager_destroy(self.stager)
+        self.stager = None
+        return (st or st2), req, cop
+
+    def layer_doorbell(self, l: int, r, stamp: int) -> None:
+        """One layer through the slot pool, in place, with no host sync."""
+        st, moe, shp = self.stack, self.moe, self.stack.shape
+        T, k, E = st.T, shp.k, shp.E
+        moe.moe_layer_route_residual(self.descs[l], r, T, k, st.wr[l],
+                                     st.bias[l], st.idx, st.w, None, st.ws,
+                                     st.ws_bytes)
+        moe.moe_slot_resolve(st.idx, T, k, E, self.table[l], self.owner[l],
+                             self.last[l], self.caps[l], int(self.base[l]),
+                             stamp, self.blob_index, self.mexp, self.mslot,
+                             self.nmiss, self.err)
+        moe.moe_miss_post(self.nmiss, self.mexp, self.mslot, T * k, l,
+                          int(self.base[l]), self.mailbox, self.sync,
+                          self.err)
+        moe.moe_wait_done(self.mailbox, self.sync, self.timeout_us,
+                          self.err)
+        moe.moe_layer_ffn_residual(self.descs[l], r, T, k, st.idx, st.w,
+                                   self.blob_index, r, None, st.ws,
+                                   st.ws_bytes)
+
+    def run_doorbell(self, r, stamp: int):
+        for l in range(len(self.caps)):
+            self.layer_doorbell(l, r, stamp)
         return r

@@ -6,7 +6,10 @@
   routing, matches the fp64 oracle within 2e-3.
 * Running the stack through a small slot pool -- misses copied from a
   pinned host store, one copy per expert -- gives output bit-identical to
-  the all-resident run, and the miss lists equal the oracle's LRU replay.
+  the all-resident run, and the miss lists equal the oracle's LRU replay;
+  the same holds with the misses handled in-stream (doorbell + stager).
+* A device wait on a done word that nothing raises gives up after its
+  bound with MOE_ERR_TIMEOUT, and the device stays usable.
 """
 import numpy as np
 import pytest
@@ -109,3 +112,79 @@ def test_slot_cache_bit_exact_vs_resident():
     assert moe.moe_get_device_status(st.ws) == 0
     assert log == expect
     assert pool.misses == sum(len(m) for _, _, m, _ in expect)
+
+
+def _replay_misses(st, routing, L, steps, cap):
+    replay = [o.SlotCache(st.shape.E, cap, list(hottest(st, l, cap)))
+              for l in range(L)]
+    expect, keys = [], set()
+    for s in range(steps):
+        for l in range(L):
+            _, miss, victims = replay[l].resolve(routing[s][l], s + 1)
+            expect.append((l, s + 1, miss, victims))
+            keys.update((l, e) for e in miss)
+    return expect, keys
+
+
+def test_slot_cache_doorbell_bit_exact_vs_resident():
+    L, steps, cap = 3, 8, 32
+    st = stack_for(L)
+    resident, routing = [], []
+    for s in range(steps):
+        rec = []
+        resident.append(st.run_resident(st.x0(s), record=rec).clone())
+        routing.append([i.cpu().numpy() for i in rec])
+    expect, keys = _replay_misses(st, routing, L, steps, cap)
+    assert keys
+    pool = SlotPool(st, [cap] * L, sorted(keys))
+    pool.start_stager()
+    try:
+        outs = [pool.run_doorbell(st.x0(s), s + 1).clone()
+                for s in range(steps)]
+    finally:
+        status, requests, copies = pool.stop_stager()
+    for s in range(steps):
+        assert torch.equal(outs[s], resident[s]), s
+    assert status == 0
+    assert int(pool.err.item()) == 0
+    assert moe.moe_get_device_status(st.ws) == 0
+    n_miss = sum(len(m) for _, _, m, _ in expect)
+    assert copies == n_miss
+    assert requests == sum(1 for _, _, m, _ in expect if m)
+    # every layer posted one request; the last one is done
+    sync = pool.sync.cpu().numpy()
+    done = int(pool.mailbox[12:16].view(torch.int32).item())
+    assert sync[0] == L * steps
+    assert max(int(sync[1]), done) == L * steps
+
+
+def test_wait_done_times_out_and_device_stays_usable():
+    mb = torch.zeros(moe.moe_mailbox_bytes(), dtype=torch.uint8).pin_memory()
+    sync = torch.tensor([1, 0], dtype=torch.int32, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    moe.moe_wait_done(mb, sync, 2000, err)      # request 1 is never done
+    torch.cuda.synchronize()
+    assert int(err.item()) == moe.MOE_ERR_TIMEOUT
+    # the same wait passes at once on a done request: device word ...
+    err.zero_()
+    sync[1] = 1
+    moe.moe_wait_done(mb, sync, 2000, err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    # ... or the mailbox's done word, written by the host
+    sync[0] = 2
+    mb[12:16].view(torch.int32)[0] = 2
+    moe.moe_wait_done(mb, sync, 2000, err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    # a mailbox that is not pinned host memory is an argument error
+    with pytest.raises(moe.MoeError):
+        moe.moe_wait_done(sync, sync, 2000, err)
+    # a miss count out of range is a device error, not a post
+    n = torch.tensor([99], dtype=torch.int32, device="cuda")
+    lst = torch.zeros(30, dtype=torch.int32, device="cuda")
+    moe.moe_miss_post(n, lst, lst, 30, 0, 0, mb, sync, err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == moe.MOE_ERR_DEVICE
+    assert int(mb[:4].view(torch.int32).item()) == 0   # nothing posted
+    assert int(sync[1].item()) == 3                   # marked done at once
