@@ -866,23 +866,27 @@ def run_stack(args) -> None:
     slot_ms = e0.elapsed_time(e1)
     slot_wall = time.perf_counter() - t0
     bit_exact = all(torch.equal(a, b) for a, b in zip(outs, ref[:S4]))
-    # the same steps with the misses handled in-stream: doorbell + stager
-    # thread, no host sync per layer
+    host_misses = pool.misses
+    # the same steps with the misses pulled from the pinned host store by
+    # the library on the stream itself: no host sync per layer
     pool.reset()
-    pool.start_stager()
+    pool.start_staging()
     outs = []
+    for s in range(min(S4, W)):          # untimed: the launch path warm
+        r.copy_(xs[s])
+        pool.run_staged(r, s + 1)
+    pool.reset()
     torch.cuda.synchronize()
     e0.record()
     for s in range(S4):
         r.copy_(xs[s])
-        pool.run_doorbell(r, s + 1)
+        pool.run_staged(r, s + 1)
         outs.append(r.clone())
     e1.record()
     e1.synchronize()
     db_ms = e0.elapsed_time(e1)
-    db_status, db_req, db_copies = pool.stop_stager()
     db_exact = all(torch.equal(a, b) for a, b in zip(outs, ref[:S4])) and \
-        int(pool.err.item()) == 0 and db_status == 0
+        int(pool.err.item()) == 0
     del outs
     hbm, tf, src = peaks()
     gbs = bytes_step / (ms / S * 1e-3) / 1e9
@@ -910,20 +914,19 @@ def run_stack(args) -> None:
             "tokens_per_s": T * S4 / (slot_ms / 1e3),
             "ms_per_step": slot_ms / max(1, S4), "wall_s": slot_wall,
             "capacities": "240 (layers 0-4), 92 (5-31), 60 (32-47)",
-            "misses": pool.misses,
-            "miss_rate": pool.misses / float(np.sum(uniq[:S4])),
-            "h2d_bytes": pool.misses * shp.blob_bytes,
+            "misses": host_misses,
+            "miss_rate": host_misses / float(np.sum(uniq[:S4])),
+            "h2d_bytes": host_misses * shp.blob_bytes,
             "host_store_blobs": len(keys),
             "host_store_build_s": store_s,
             "bit_exact_vs_resident": bit_exact},
-        "slot_cache_doorbell": {
+        "slot_cache_in_stream": {
             "steps": S4,
             "tokens_per_s": T * S4 / (db_ms / 1e3),
             "ms_per_step": db_ms / max(1, S4),
-            "how": ("per layer: route, resolve, miss post to a mapped "
-                    "mailbox, bounded device wait, FFN; the library's stager "
-                    "thread copies the misses; no host sync per layer"),
-            "requests": db_req, "blobs_copied": db_copies,
+            "how": ("per layer on one stream: route, resolve, a kernel that "
+                    "pulls each missed blob from the pinned host store over "
+                    "PCIe into its slot, FFN; no host sync per layer"),
             "bit_exact_vs_resident": db_exact},
         "setup_s": setup_s,
         "gpu_launches": L * S,

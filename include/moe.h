@@ -193,66 +193,36 @@ moe_status moe_slot_resolve(const int32_t* topk_idx, int T, int k, int E,
 
 /* ---------------------------------------- in-stream expert staging ---- */
 
-/* Miss handling without a host round trip per layer ("Betelgeuse": the
- * decode stream rings a mapped host doorbell only when a layer misses, and
- * a host pager fills the slots).  Per layer, on the compute stream:
- *   moe_slot_resolve -> moe_miss_post -> moe_wait_done -> the expert FFN
- * and, on the host, one stager (moe_stager_create) that copies the missed
- * blobs.  Every call below is asynchronous and can be captured in a CUDA
- * graph (except the stager calls, which are host-only).
- *   mailbox  mapped pinned host memory of moe_mailbox_bytes() bytes, zeroed
- *            before first use (cudaHostAlloc / torch pin_memory); holds the
- *            posted request, its miss list and the stager's done word
- *   sync     uint32 [2] device memory, zeroed before first use: the last
- *            request number and the done word of requests without misses
- * A request with misses is served in order by the stager, which waits for
- * its copies on the host and then writes the done word: nothing it does
- * uses a compute queue, where it could sit behind the launches the wait
- * holds up.  A request without misses is done at once.  At most 1024
- * misses per request.  A wrong mailbox or sync pointer is MOE_ERR_INVALID
- * (checked on the host). */
-size_t moe_mailbox_bytes(void);
+/* Miss handling without a host round trip per layer ("Betelgeuse": a VRAM
+ * slot pool whose misses a pager fills while the decode stream waits).
+ * The host copies of the blobs sit in pinned host memory, so the GPU pulls
+ * the misses itself; per layer, on one stream (capturable in a graph):
+ *   moe_slot_resolve -> moe_stage_misses -> the expert FFN
+ * No host thread, flag or second stream is involved. */
 
-/* Post this layer's misses (moe_slot_resolve's n_miss / miss_expert /
- * miss_slot, device pointers; P = T*k entries at most) as request
- * number sync[0] + 1 for layer `layer`; the stager copies blob (layer, e)
- * into pool slot slot_base + miss_slot[i].  A miss count outside [0, P]
- * sets MOE_ERR_DEVICE in err (device, may be NULL) and posts nothing. */
-moe_status moe_miss_post(const int32_t* n_miss, const int32_t* miss_expert,
-                         const int32_t* miss_slot, int P, int layer,
-                         int slot_base, void* mailbox, uint32_t* sync,
-                         int32_t* err, void* stream);
+/* Build the device table of host blob addresses once: host_blob[i] (host
+ * pointers, i = layer * E + e, NULL = not stored) must be 16-byte aligned
+ * mapped pinned host memory (cudaHostAlloc, torch pin_memory), else
+ * MOE_ERR_INVALID; table is uint64 [n] device memory.  Synchronises
+ * `stream`. */
+moe_status moe_stage_table(const void* const* host_blob, int n,
+                           uint64_t* table, void* stream);
 
-/* Hold the stream until the last posted request is done (its blobs are in
- * the pool).  Bounded: after timeout_us microseconds of %globaltimer the
- * kernel gives up, sets MOE_ERR_TIMEOUT in err (device word, required) and
- * the stream goes on, so a missing stager never hangs the device. */
-moe_status moe_wait_done(void* mailbox, const uint32_t* sync,
-                         uint32_t timeout_us, int32_t* err, void* stream);
-
-/* Start the host pager (one thread).  It polls the mailbox; for each
- * request it issues one cudaMemcpyAsync per half blob from
- * host_blob[layer * E + e] (host pointers, pinned, NULL = not stored:
- * MOE_ERR_CAPACITY in the stager status) to pool + slot * blob_stride on
- * copy_streams (cudaStream_t, round robin), waits for them and writes the
- * done word.  Requests posted before this call are not its own.
- * host_blob is copied; the streams, pool and mailbox stay owned by the
- * caller and must outlive the stager.  *out receives an opaque handle. */
-moe_status moe_stager_create(void** out, void* mailbox,
-                             uint8_t* pool, int64_t blob_stride,
-                             int64_t blob_bytes, const void* const* host_blob,
-                             int L, int E, void* const* copy_streams,
-                             int n_copy_streams);
-
-/* Requests served and blobs copied so far (either pointer may be NULL);
- * returns the stager's first error status, MOE_OK if none. */
-moe_status moe_stager_stats(void* stager, int64_t* requests,
-                            int64_t* copies);
-
-/* Stop and join the thread, wait for its copies, free the handle; returns
- * the stager's first error status.  Any device wait still pending then
- * ends by its timeout. */
-moe_status moe_stager_destroy(void* stager);
+/* Copy this layer's missed blobs (moe_slot_resolve's n_miss / miss_expert /
+ * miss_slot, device, P = T*k entries) from their pinned host copies
+ * table[layer * E + e] into pool slot slot_base + miss_slot[i] (pool has
+ * pool_slots slots of blob_stride bytes; blob_bytes are copied), reading
+ * host memory over PCIe from one kernel on the stream.  A missing host copy
+ * or a slot outside the pool sets MOE_ERR_CAPACITY in err (device word) and
+ * skips that blob; a miss count outside [0, P] sets MOE_ERR_DEVICE.
+ * blob_bytes, blob_stride and pool must be multiples of 16 (bytes), and
+ * 0 <= layer < L. */
+moe_status moe_stage_misses(const int32_t* n_miss, const int32_t* miss_expert,
+                            const int32_t* miss_slot, int P, int layer, int L,
+                            int E, const uint64_t* table, uint8_t* pool,
+                            int slot_base, int64_t pool_slots,
+                            int64_t blob_stride, int64_t blob_bytes,
+                            int32_t* err, void* stream);
 
 /* ------------------------------------------------------- expert FFN ---- */
 

@@ -82,14 +82,10 @@ _SIGS = {
                                          _P, _P, _P, c_size_t, _P]),
     "moe_layer_ffn_residual": (c_int, [_P, _P, c_int, c_int, _P, _P, _P, _P,
                                        _P, _P, c_size_t, _P]),
-    "moe_mailbox_bytes": (c_size_t, []),
-    "moe_miss_post": (c_int, [_P, _P, _P, c_int, c_int, c_int, _P, _P, _P,
-                              _P]),
-    "moe_wait_done": (c_int, [_P, _P, c_uint32, _P, _P]),
-    "moe_stager_create": (c_int, [_P, _P, _P, c_int64, c_int64, _P, c_int,
-                                  c_int, _P, c_int]),
-    "moe_stager_stats": (c_int, [_P, _P, _P]),
-    "moe_stager_destroy": (c_int, [_P]),
+    "moe_stage_table": (c_int, [_P, c_int, _P, _P]),
+    "moe_stage_misses": (c_int, [_P, _P, _P, c_int, c_int, c_int, c_int, _P,
+                                 _P, c_int, c_int64, c_int64, c_int64, _P,
+                                 _P]),
     "moe_get_device_status": (c_int, [_P, _P, _P]),
     "moe_status_string": (ctypes.c_char_p, [c_int]),
 }
@@ -290,49 +286,21 @@ def moe_layer_ffn_residual(desc, r, T, k, topk_idx, topk_w, blob_index,
         _stream(stream)))
 
 
-def moe_mailbox_bytes() -> int:
-    return lib.moe_mailbox_bytes()
+def moe_stage_table(host_blob, table, stream=None):
+    """host_blob: host addresses (0 = not stored), one per table entry."""
+    n = len(host_blob)
+    arr = (c_void_p * n)(*[int(a) or None for a in host_blob])
+    _check("moe_stage_table", lib.moe_stage_table(
+        arr, n, _ptr(table), _stream(stream)))
 
 
-def moe_miss_post(n_miss, miss_expert, miss_slot, P, layer, slot_base,
-                  mailbox, sync, err, stream=None):
-    _check("moe_miss_post", lib.moe_miss_post(
-        _ptr(n_miss), _ptr(miss_expert), _ptr(miss_slot), P, layer,
-        slot_base, _ptr(mailbox), _ptr(sync), _ptr(err), _stream(stream)))
-
-
-def moe_wait_done(mailbox, sync, timeout_us, err, stream=None):
-    _check("moe_wait_done", lib.moe_wait_done(
-        _ptr(mailbox), _ptr(sync), timeout_us, _ptr(err), _stream(stream)))
-
-
-def moe_stager_create(mailbox, pool, blob_stride, blob_bytes, host_blob, L,
-                      E, copy_streams) -> int:
-    """host_blob: L*E host addresses (0 = not stored); copy_streams: torch
-    streams or raw handles.  Returns the opaque handle."""
-    n = L * E
-    if len(host_blob) != n:
-        raise ValueError("host_blob needs L*E entries")
-    table = (c_void_p * n)(*[int(a) or None for a in host_blob])
-    streams = (c_void_p * len(copy_streams))(
-        *[_stream(s) for s in copy_streams])
-    h = c_void_p()
-    _check("moe_stager_create", lib.moe_stager_create(
-        ctypes.byref(h), _ptr(mailbox), _ptr(pool), blob_stride, blob_bytes,
-        table, L, E, streams, len(copy_streams)))
-    return h.value
-
-
-def moe_stager_stats(stager):
-    """(status, requests served, blobs copied)."""
-    r, c = ctypes.c_int64(0), ctypes.c_int64(0)
-    st = lib.moe_stager_stats(stager, ctypes.byref(r), ctypes.byref(c))
-    return st, r.value, c.value
-
-
-def moe_stager_destroy(stager) -> int:
-    """Stops the stager; returns its first error status (0 = none)."""
-    return lib.moe_stager_destroy(stager)
+def moe_stage_misses(n_miss, miss_expert, miss_slot, P, layer, L, E, table,
+                     pool, slot_base, pool_slots, blob_stride, blob_bytes,
+                     err, stream=None):
+    _check("moe_stage_misses", lib.moe_stage_misses(
+        _ptr(n_miss), _ptr(miss_expert), _ptr(miss_slot), P, layer, L, E,
+        _ptr(table), _ptr(pool), slot_base, pool_slots, blob_stride,
+        blob_bytes, _ptr(err), _stream(stream)))
 
 
 def moe_get_device_status(ws, stream=None) -> int:

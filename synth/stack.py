@@ -1,7 +1,7 @@
 """Drivers of the multi-layer decode workloads through the library's C ABI:
 the all-resident residual stack and the same stack over an expert-slot
-pool (misses handled by a host round trip per layer, or in-stream through
-the library's doorbell and stager).  No arithmetic of the layer happens
+pool (misses copied after a host round trip per layer, or pulled from the
+pinned host store by the library on the stream itself).  No arithmetic of the layer happens
 here -- every layer runs in the library; this module only owns buffers,
 builds the device pools with the seeded generator, and moves missed expert
 blobs (one copy per expert).
@@ -207,36 +207,22 @@ class SlotPool:
             self.layer(l, r, stamp, log)
         return r
 
-    # ----------------------------------------- in-stream doorbell mode --
-    def start_stager(self, timeout_us: int = 2_000_000) -> None:
-        """Miss handling without a host round trip per layer: the layer's
-        misses go to a mapped pinned mailbox (moe_miss_post), the library's
-        stager thread copies them from the host store, and the stream waits
-        on the device (moe_wait_done) before the FFN."""
+    # ------------------------------------------- in-stream staging mode --
+    def start_staging(self) -> None:
+        """Miss handling without a host round trip per layer: after the
+        resolve, moe_stage_misses pulls each missed blob from the pinned
+        host store into its slot on the same stream."""
         torch, moe = self.torch, self.moe
-        assert not self.device_source, "the doorbell mode needs a host store"
+        assert not self.device_source, "in-stream staging needs a host store"
         L, E = len(self.caps), self.stack.shape.E
-        self.mailbox = torch.zeros(moe.moe_mailbox_bytes(),
-                                   dtype=torch.uint8).pin_memory()
-        self.sync = torch.zeros(2, dtype=torch.int32, device="cuda")
         table = [0] * (L * E)
         for (l, e), i in self.store_index.items():
             table[l * E + e] = self.store[i].data_ptr()
-        self.timeout_us = int(timeout_us)
-        torch.cuda.synchronize()
-        self.stager = moe.moe_stager_create(
-            self.mailbox, self.pool, self.stride, self.blob, table, L, E,
-            self.copy_streams)
+        self.table_dev = torch.zeros(L * E, dtype=torch.int64, device="cuda")
+        moe.moe_stage_table(table, self.table_dev)
+        self.n_slots = int(sum(self.caps))
 
-    def stop_stager(self) -> Tuple[int, int, int]:
-        """Stops the stager; returns (status, requests, blobs copied)."""
-        self.torch.cuda.synchronize()
-        st, req, cop = self.moe.moe_stager_stats(self.stager)
-        st2 = self.moe.moe_stager_destroy(self.stager)
-        self.stager = None
-        return (st or st2), req, cop
-
-    def layer_doorbell(self, l: int, r, stamp: int) -> None:
+    def layer_staged(self, l: int, r, stamp: int) -> None:
         """One layer through the slot pool, in place, with no host sync."""
         st, moe, shp = self.stack, self.moe, self.stack.shape
         T, k, E = st.T, shp.k, shp.E
@@ -247,16 +233,15 @@ class SlotPool:
                              self.last[l], self.caps[l], int(self.base[l]),
                              stamp, self.blob_index, self.mexp, self.mslot,
                              self.nmiss, self.err)
-        moe.moe_miss_post(self.nmiss, self.mexp, self.mslot, T * k, l,
-                          int(self.base[l]), self.mailbox, self.sync,
-                          self.err)
-        moe.moe_wait_done(self.mailbox, self.sync, self.timeout_us,
-                          self.err)
+        moe.moe_stage_misses(self.nmiss, self.mexp, self.mslot, T * k, l,
+                             len(self.caps), E, self.table_dev, self.pool,
+                             int(self.base[l]), self.n_slots, self.stride,
+                             self.blob, self.err)
         moe.moe_layer_ffn_residual(self.descs[l], r, T, k, st.idx, st.w,
                                    self.blob_index, r, None, st.ws,
                                    st.ws_bytes)
 
-    def run_doorbell(self, r, stamp: int):
+    def run_staged(self, r, stamp: int):
         for l in range(len(self.caps)):
-            self.layer_doorbell(l, r, stamp)
+            self.layer_staged(l, r, stamp)
         return r

@@ -7,9 +7,11 @@
 * Running the stack through a small slot pool -- misses copied from a
   pinned host store, one copy per expert -- gives output bit-identical to
   the all-resident run, and the miss lists equal the oracle's LRU replay;
-  the same holds with the misses handled in-stream (doorbell + stager).
-* A device wait on a done word that nothing raises gives up after its
-  bound with MOE_ERR_TIMEOUT, and the device stays usable.
+  the same holds with the misses pulled from the host store on the stream
+  (no host round trip per layer).
+* The in-stream copy moves blobs byte for byte, rejects host memory that is
+  not mapped pinned memory on the host, and reports a missing host copy or
+  a bad miss count in the device error word.
 """
 import numpy as np
 import pytest
@@ -126,7 +128,7 @@ def _replay_misses(st, routing, L, steps, cap):
     return expect, keys
 
 
-def test_slot_cache_doorbell_bit_exact_vs_resident():
+def test_slot_cache_in_stream_staging_bit_exact_vs_resident():
     L, steps, cap = 3, 8, 32
     st = stack_for(L)
     resident, routing = [], []
@@ -137,54 +139,58 @@ def test_slot_cache_doorbell_bit_exact_vs_resident():
     expect, keys = _replay_misses(st, routing, L, steps, cap)
     assert keys
     pool = SlotPool(st, [cap] * L, sorted(keys))
-    pool.start_stager()
-    try:
-        outs = [pool.run_doorbell(st.x0(s), s + 1).clone()
-                for s in range(steps)]
-    finally:
-        status, requests, copies = pool.stop_stager()
+    pool.start_staging()
+    outs = [pool.run_staged(st.x0(s), s + 1).clone() for s in range(steps)]
     for s in range(steps):
         assert torch.equal(outs[s], resident[s]), s
-    assert status == 0
     assert int(pool.err.item()) == 0
     assert moe.moe_get_device_status(st.ws) == 0
-    n_miss = sum(len(m) for _, _, m, _ in expect)
-    assert copies == n_miss
-    assert requests == sum(1 for _, _, m, _ in expect if m)
-    # every layer posted one request; the last one is done
-    sync = pool.sync.cpu().numpy()
-    done = int(pool.mailbox[12:16].view(torch.int32).item())
-    assert sync[0] == L * steps
-    assert max(int(sync[1]), done) == L * steps
+    # the slot tables end where the host-round-trip run ends
+    ref = SlotPool(st, [cap] * L, sorted(keys))
+    for s in range(steps):
+        ref.run(st.x0(s), s + 1)
+    for l in range(L):
+        assert torch.equal(pool.table[l], ref.table[l])
+        assert torch.equal(pool.owner[l], ref.owner[l])
 
 
-def test_wait_done_times_out_and_device_stays_usable():
-    mb = torch.zeros(moe.moe_mailbox_bytes(), dtype=torch.uint8).pin_memory()
-    sync = torch.tensor([1, 0], dtype=torch.int32, device="cuda")
+def test_stage_misses_copies_and_errors():
+    E, L, blob, stride, slots = 4, 2, 4096 + 256, 4608, 6
+    host = torch.randint(0, 256, (L * E, blob), dtype=torch.uint8)
+    host = host.pin_memory()
+    table_host = [host[i].data_ptr() for i in range(L * E)]
+    table_host[1 * E + 3] = 0                      # (layer 1, expert 3) absent
+    table = torch.zeros(L * E, dtype=torch.int64, device="cuda")
+    moe.moe_stage_table(table_host, table)
+    pool = torch.zeros(slots * stride, dtype=torch.uint8, device="cuda")
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
-    moe.moe_wait_done(mb, sync, 2000, err)      # request 1 is never done
+    mexp = torch.tensor([2, 0, 3], dtype=torch.int32, device="cuda")
+    mslot = torch.tensor([1, 0, 2], dtype=torch.int32, device="cuda")
+    n = torch.tensor([3], dtype=torch.int32, device="cuda")
+    # layer 1, slot base 3: blobs (1,2) -> slot 4, (1,0) -> slot 3, (1,3) absent
+    moe.moe_stage_misses(n, mexp, mslot, 3, 1, L, E, table, pool, 3, slots,
+                         stride, blob, err)
     torch.cuda.synchronize()
-    assert int(err.item()) == moe.MOE_ERR_TIMEOUT
-    # the same wait passes at once on a done request: device word ...
+    assert int(err.item()) == moe.MOE_ERR_CAPACITY
+    got = pool.cpu()
+    assert torch.equal(got[4 * stride:4 * stride + blob], host[1 * E + 2])
+    assert torch.equal(got[3 * stride:3 * stride + blob], host[1 * E + 0])
+    assert int(got[5 * stride:6 * stride].sum()) == 0     # skipped
+    assert int(got[:3 * stride].sum()) == 0               # untouched
+    # a miss count out of range: device error, nothing copied
     err.zero_()
-    sync[1] = 1
-    moe.moe_wait_done(mb, sync, 2000, err)
-    torch.cuda.synchronize()
-    assert int(err.item()) == 0
-    # ... or the mailbox's done word, written by the host
-    sync[0] = 2
-    mb[12:16].view(torch.int32)[0] = 2
-    moe.moe_wait_done(mb, sync, 2000, err)
-    torch.cuda.synchronize()
-    assert int(err.item()) == 0
-    # a mailbox that is not pinned host memory is an argument error
-    with pytest.raises(moe.MoeError):
-        moe.moe_wait_done(sync, sync, 2000, err)
-    # a miss count out of range is a device error, not a post
-    n = torch.tensor([99], dtype=torch.int32, device="cuda")
-    lst = torch.zeros(30, dtype=torch.int32, device="cuda")
-    moe.moe_miss_post(n, lst, lst, 30, 0, 0, mb, sync, err)
+    pool.zero_()
+    n[0] = 7
+    moe.moe_stage_misses(n, mexp, mslot, 3, 0, L, E, table, pool, 0, slots,
+                         stride, blob, err)
     torch.cuda.synchronize()
     assert int(err.item()) == moe.MOE_ERR_DEVICE
-    assert int(mb[:4].view(torch.int32).item()) == 0   # nothing posted
-    assert int(sync[1].item()) == 3                   # marked done at once
+    assert int(pool.sum()) == 0
+    # host memory that is not pinned, and a layer outside the table, are
+    # argument errors found on the host
+    plain = torch.zeros(blob, dtype=torch.uint8)
+    with pytest.raises(moe.MoeError):
+        moe.moe_stage_table([plain.data_ptr()], table)
+    with pytest.raises(moe.MoeError):
+        moe.moe_stage_misses(n, mexp, mslot, 3, L, L, E, table, pool, 0,
+                             slots, stride, blob, err)
