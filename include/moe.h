@@ -180,9 +180,10 @@ moe_status moe_group_tokens_static(const int32_t* topk_idx, int T, int k,
  *               nothing is updated)
  * Victim rule: the slot with the smallest last_use among the slots this
  * call has not used or filled, ties to the lowest slot; the evicted
- * expert's table entry becomes -1.  After the call the caller copies each
- * missed expert's blob into pool + blob_index[e] * stride (one copy per
- * expert) before the FFN runs on the same stream.  Needs T*k <= 1024,
+ * expert's table entry becomes -1.  After the call each missed expert's
+ * blob goes into pool + blob_index[e] * stride (one copy per expert) before
+ * the FFN runs on the same stream: copied by the caller, or pulled from
+ * pinned host memory on the stream by moe_stage_misses.  Needs T*k <= 1024,
  * E <= 8192, n_slots <= 8192. */
 moe_status moe_slot_resolve(const int32_t* topk_idx, int T, int k, int E,
                             int32_t* slot_table, int32_t* slot_owner,
