@@ -45,3 +45,38 @@ def test_host_side_queries_without_gpu():
     assert moe.moe_tensor_bytes(moe.MOE_SB3_256, 16, 100) == 0
     assert moe.moe_ffn_workspace_bytes(3, 10, 3072, 1024) > 0
     assert moe.status_string(moe.MOE_ERR_CAPACITY).startswith("slot")
+
+
+def test_stage_argument_errors_without_gpu():
+    """The in-stream staging calls reject bad arguments on the host, before
+    any CUDA call (fake non-null addresses are never dereferenced)."""
+    f = 4096   # a 16-byte aligned stand-in address
+    lib = moe.lib
+
+    def stage(**kw):
+        a = dict(n_miss=f, miss_expert=f, miss_slot=f, P=30, layer=0, L=48,
+                 E=512, table=f, pool=f, slot_base=0, pool_slots=4644,
+                 blob_stride=4276224, blob_bytes=4276224, err=f, stream=None)
+        a.update(kw)
+        return lib.moe_stage_misses(
+            a["n_miss"], a["miss_expert"], a["miss_slot"], a["P"],
+            a["layer"], a["L"], a["E"], a["table"], a["pool"],
+            a["slot_base"], a["pool_slots"], a["blob_stride"],
+            a["blob_bytes"], a["err"], a["stream"])
+
+    assert stage(n_miss=None) == moe.MOE_ERR_INVALID
+    assert stage(table=None) == moe.MOE_ERR_INVALID
+    assert stage(pool=None) == moe.MOE_ERR_INVALID
+    assert stage(P=0) == moe.MOE_ERR_SHAPE
+    assert stage(layer=48) == moe.MOE_ERR_SHAPE           # layer >= L
+    assert stage(layer=-1) == moe.MOE_ERR_SHAPE
+    assert stage(blob_bytes=4276224 + 8) == moe.MOE_ERR_SHAPE   # not 16n
+    assert stage(blob_stride=4276224 - 16) == moe.MOE_ERR_SHAPE  # < blob
+    assert stage(pool=f + 8) == moe.MOE_ERR_SHAPE           # misaligned
+    assert stage(pool_slots=0) == moe.MOE_ERR_SHAPE
+    table = (ctypes.c_void_p * 1)(None)
+    assert lib.moe_stage_table(table, 0, f, None) == moe.MOE_ERR_INVALID
+    assert lib.moe_stage_table(None, 1, f, None) == moe.MOE_ERR_INVALID
+    # an unaligned host address is refused before it is looked up
+    table[0] = f + 4
+    assert lib.moe_stage_table(table, 1, f, None) == moe.MOE_ERR_INVALID
