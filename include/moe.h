@@ -9,13 +9,15 @@
  * and each expert stored packed as up | gate | down (model card, "Files").
  * The device-side expert-slot lookup follows the "Betelgeuse" post (VRAM
  * slot pool with per-layer capacities, hits resolved on the device, only
- * misses reported).
+ * misses reported); the missed blobs can be pulled from pinned host memory
+ * on the stream itself (moe_stage_misses), with no host round trip.
  *
  * Conventions (every entry point):
  *   - Pointers are DEVICE pointers unless the comment says "host".
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy stream).
  *   - The library never allocates memory, never synchronises the stream
- *     (except moe_get_device_status) and never prints.  Memory is owned by
+ *     (except moe_get_device_status, and moe_stage_table, a once-per-pool
+ *     setup call) and never prints.  Memory is owned by
  *     the caller; workspaces are sized with the *_workspace_bytes queries.
  *   - Argument errors are returned synchronously (MOE_ERR_INVALID /
  *     MOE_ERR_SHAPE / MOE_ERR_WORKSPACE) before anything is launched.  A
