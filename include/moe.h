@@ -105,6 +105,26 @@ moe_status moe_pack_tensor(int fmt, const uint8_t* natural, int rows,
 moe_status moe_dequant(int fmt, const uint8_t* packed, int rows, int cols,
                        float* out, void* stream);
 
+/* Hot-path decoders of moe_dequant_path. */
+typedef enum { MOE_DQ_DECODE = 1, MOE_DQ_PREFILL = 2 } moe_dq_path;
+
+/* Packed tensor -> its weights as one of the layer's hot-path decoders
+ * produces them (the closed forms of moe_qfmt are the reference; model
+ * card, "Files").  A check and debugging export: the FFN kernels never
+ * materialise these tensors.
+ *   path MOE_DQ_DECODE:  out fp32 [rows x cols] row-major, computed by the
+ *        int8 tensor-core tile decoders of the decode kernels (T <= 8),
+ *        fed one-hot activations.  Every weight of these formats is exact
+ *        in fp32, so the result equals the closed form bit for bit.
+ *   path MOE_DQ_PREFILL: out fp16 bits [rows x cols] row-major: the
+ *        operand tiles the prefill grouped GEMM's dequantising warps write
+ *        to shared memory, un-swizzled.  Each value is the round-to-nearest-
+ *        even fp16 of the closed form.  Needs rows % 128 == 0.
+ * packed and out 16-byte aligned (else MOE_ERR_INVALID); shape rules of
+ * moe_pack_tensor (else MOE_ERR_SHAPE). */
+moe_status moe_dequant_path(int fmt, int path, const uint8_t* packed,
+                            int rows, int cols, void* out, void* stream);
+
 /* ---------------------------------------------------------- routing ---- */
 
 /* Router and top-k ("Avalon": 512 experts, 10 active; softmax over all E,
@@ -153,9 +173,10 @@ moe_status moe_group_tokens(const int32_t* topk_idx, int T, int k, int E,
  *   Limits: T*k <= 262144 and E <= 1024, else MOE_ERR_SHAPE.
  *   err  int32 [1] device error word, or NULL to use the array's own word
  *        (cleared at each call; then bad expert ids are not reported).
- *   The first call on each device looks up the array's device address (a
- *   runtime symbol lookup); make that first call before any stream
- *   capture.  Calls that overlap on the GPU (other streams, other host
+ *   The first call in each CUDA context (per device) looks up the array's
+ *   device address (a runtime symbol lookup); make that first call before
+ *   any stream capture.  Do not use the library across a device reset
+ *   (cudaDeviceReset): the array lives in the context that loaded it.  Calls that overlap on the GPU (other streams, other host
  *   threads) share the array and race: serialise them.  Nothing is
  *   allocated or freed by this call. */
 moe_status moe_group_tokens_static(const int32_t* topk_idx, int T, int k,
@@ -194,6 +215,25 @@ moe_status moe_slot_resolve(const int32_t* topk_idx, int T, int k, int E,
                             int32_t* miss_expert, int32_t* miss_slot,
                             int32_t* n_miss, int32_t* err, void* stream);
 
+/* moe_slot_resolve with the stamp kept on the device, so that a decode
+ * step (route -> resolve -> stage -> FFN for every layer) can be captured
+ * once as a CUDA graph and replayed step after step with no host argument
+ * changing ("Betelgeuse": the whole decode pass as one graph replay).
+ *   stamp  uint32 [1] device counter of this partition, 0 before its first
+ *          call: the call stamps with *stamp + 1 and stores that value back
+ *          (unless it reports an error, when nothing is updated).
+ * Resolving each layer once per step with its own counter gives exactly
+ * the stamps (and so the victims) of moe_slot_resolve called with
+ * stamp = step number, steps counted from 1.  Other arguments, limits and
+ * errors as moe_slot_resolve; stamp NULL is MOE_ERR_INVALID. */
+moe_status moe_slot_resolve_dev(const int32_t* topk_idx, int T, int k, int E,
+                                int32_t* slot_table, int32_t* slot_owner,
+                                uint32_t* last_use, int n_slots,
+                                int slot_base, uint32_t* stamp,
+                                int32_t* blob_index, int32_t* miss_expert,
+                                int32_t* miss_slot, int32_t* n_miss,
+                                int32_t* err, void* stream);
+
 /* ---------------------------------------- in-stream expert staging ---- */
 
 /* Miss handling without a host round trip per layer ("Betelgeuse": a VRAM
@@ -213,17 +253,19 @@ moe_status moe_stage_table(const void* const* host_blob, int n,
 
 /* Copy this layer's missed blobs (moe_slot_resolve's n_miss / miss_expert /
  * miss_slot, device, P = T*k entries) from their pinned host copies
- * table[layer * E + e] into pool slot slot_base + miss_slot[i] (pool has
- * pool_slots slots of blob_stride bytes; blob_bytes are copied), reading
- * host memory over PCIe from one kernel on the stream.  A missing host copy
- * or a slot outside the pool sets MOE_ERR_CAPACITY in err (device word) and
- * skips that blob; a miss count outside [0, P] sets MOE_ERR_DEVICE.
- * blob_bytes, blob_stride and pool must be multiples of 16 (bytes), and
- * 0 <= layer < L. */
+ * table[layer * E + e] into pool slot slot_base + miss_slot[i], reading
+ * host memory over PCIe from one kernel on the stream.  The layer's
+ * partition is slots slot_base .. slot_base + n_slots - 1 of a pool of
+ * pool_slots slots of blob_stride bytes; blob_bytes are copied per blob.
+ * A missing host copy, or a miss_slot outside [0, n_slots), sets
+ * MOE_ERR_CAPACITY in err (device word) and skips that blob (so a bad slot
+ * never overwrites another layer's expert); a miss count outside [0, P]
+ * sets MOE_ERR_DEVICE.  blob_bytes, blob_stride and pool must be multiples
+ * of 16 (bytes), 0 <= layer < L and slot_base + n_slots <= pool_slots. */
 moe_status moe_stage_misses(const int32_t* n_miss, const int32_t* miss_expert,
                             const int32_t* miss_slot, int P, int layer, int L,
                             int E, const uint64_t* table, uint8_t* pool,
-                            int slot_base, int64_t pool_slots,
+                            int slot_base, int n_slots, int64_t pool_slots,
                             int64_t blob_stride, int64_t blob_bytes,
                             int32_t* err, void* stream);
 
@@ -317,8 +359,10 @@ size_t moe_layer_workspace_bytes(int T, int k, int E, int H, int F);
  * the weighted combine.  T <= 8 (with T*k at most the SM count and
  * E <= 1024): one cooperative kernel does all of it; it is launched as a
  * programmatic dependent of the work before it on the stream and touches
- * no global memory until that work has completed, so stream order holds as
- * usual.  Otherwise: moe_route_topk, moe_group_tokens, then the expert FFN
+ * no global memory until that work has completed -- except w_router, whose
+ * rows it starts loading at once: w_router must not be written by the work
+ * just before the call on the stream (the same holds for the residual
+ * variants below).  Otherwise: moe_route_topk, moe_group_tokens, then the expert FFN
  * (the tensor-core prefill path when T > 8 and the shapes allow it) and
  * the combine.  The grouping lives in the workspace.  w_router bf16
  * [E x H]; bias fp32 [E] or NULL; blob_index as in moe_expert_ffn_q;

@@ -30,6 +30,9 @@ MOE_Q4_B32 = 1
 MOE_SB3_256 = 2
 MOE_NL4_B32 = 3
 
+MOE_DQ_DECODE = 1
+MOE_DQ_PREFILL = 2
+
 
 class MoeError(RuntimeError):
     def __init__(self, fn: str, code: int):
@@ -49,6 +52,7 @@ _SIGS = {
     "moe_blob_bytes": (c_size_t, [c_int, c_int, c_int, c_int]),
     "moe_pack_tensor": (c_int, [c_int, _P, c_int, c_int, _P, _P]),
     "moe_dequant": (c_int, [c_int, _P, c_int, c_int, _P, _P]),
+    "moe_dequant_path": (c_int, [c_int, c_int, _P, c_int, c_int, _P, _P]),
     "moe_route_topk": (c_int, [_P, c_int, c_int, _P, c_int, _P, c_int, _P,
                                _P, _P, _P]),
     "moe_group_workspace_bytes": (c_size_t, [c_int, c_int, c_int]),
@@ -84,8 +88,11 @@ _SIGS = {
                                        _P, _P, c_size_t, _P]),
     "moe_stage_table": (c_int, [_P, c_int, _P, _P]),
     "moe_stage_misses": (c_int, [_P, _P, _P, c_int, c_int, c_int, c_int, _P,
-                                 _P, c_int, c_int64, c_int64, c_int64, _P,
-                                 _P]),
+                                 _P, c_int, c_int, c_int64, c_int64, c_int64,
+                                 _P, _P]),
+    "moe_slot_resolve_dev": (c_int, [_P, c_int, c_int, c_int, _P, _P, _P,
+                                     c_int, c_int, _P, _P, _P, _P, _P, _P,
+                                     _P]),
     "moe_get_device_status": (c_int, [_P, _P, _P]),
     "moe_status_string": (ctypes.c_char_p, [c_int]),
 }
@@ -154,6 +161,11 @@ def moe_dequant(fmt, packed, rows, cols, out, stream=None):
         fmt, _ptr(packed), rows, cols, _ptr(out), _stream(stream)))
 
 
+def moe_dequant_path(fmt, path, packed, rows, cols, out, stream=None):
+    _check("moe_dequant_path", lib.moe_dequant_path(
+        fmt, path, _ptr(packed), rows, cols, _ptr(out), _stream(stream)))
+
+
 def moe_route_topk(x, T, H, w_router, E, bias, k, topk_idx, topk_w,
                    logits_out, stream=None):
     _check("moe_route_topk", lib.moe_route_topk(
@@ -185,6 +197,16 @@ def moe_slot_resolve(topk_idx, T, k, E, slot_table, slot_owner, last_use,
     _check("moe_slot_resolve", lib.moe_slot_resolve(
         _ptr(topk_idx), T, k, E, _ptr(slot_table), _ptr(slot_owner),
         _ptr(last_use), n_slots, slot_base, stamp, _ptr(blob_index),
+        _ptr(miss_expert), _ptr(miss_slot), _ptr(n_miss), _ptr(err),
+        _stream(stream)))
+
+
+def moe_slot_resolve_dev(topk_idx, T, k, E, slot_table, slot_owner,
+                         last_use, n_slots, slot_base, stamp, blob_index,
+                         miss_expert, miss_slot, n_miss, err, stream=None):
+    _check("moe_slot_resolve_dev", lib.moe_slot_resolve_dev(
+        _ptr(topk_idx), T, k, E, _ptr(slot_table), _ptr(slot_owner),
+        _ptr(last_use), n_slots, slot_base, _ptr(stamp), _ptr(blob_index),
         _ptr(miss_expert), _ptr(miss_slot), _ptr(n_miss), _ptr(err),
         _stream(stream)))
 
@@ -295,11 +317,11 @@ def moe_stage_table(host_blob, table, stream=None):
 
 
 def moe_stage_misses(n_miss, miss_expert, miss_slot, P, layer, L, E, table,
-                     pool, slot_base, pool_slots, blob_stride, blob_bytes,
-                     err, stream=None):
+                     pool, slot_base, n_slots, pool_slots, blob_stride,
+                     blob_bytes, err, stream=None):
     _check("moe_stage_misses", lib.moe_stage_misses(
         _ptr(n_miss), _ptr(miss_expert), _ptr(miss_slot), P, layer, L, E,
-        _ptr(table), _ptr(pool), slot_base, pool_slots, blob_stride,
+        _ptr(table), _ptr(pool), slot_base, n_slots, pool_slots, blob_stride,
         blob_bytes, _ptr(err), _stream(stream)))
 
 

@@ -19,7 +19,8 @@
 //   P1  every block: top-k of every token from the logits (a warp per
 //       token, one redux.sync arg-max per round), softmax weights, grouping
 //       of the T*k pairs by expert -- all in shared memory; meanwhile the
-//       other warps turn x into int8 hi/lo B fragments (per-token 2^-sigma)
+//       other warps turn x into int8 hi/lo B fragments (2^-sigma per token
+//       and 256-column block)
 //   P2  up/gate units (expert, 16 rows of F, all of H), two groups of eight
 //       warps taking alternate units, three tiles per warp, partial sums
 //       -> shared memory; the group's epilogue warp reduces them,
@@ -85,7 +86,7 @@ struct LayerParams {
 
 
 struct Smem {  // offsets into dynamic shared memory
-  int slot_bytes, ring, frag, red, misc, total;
+  int slot_bytes, ring, frag, red, misc, xsc, total;
 };
 
 __host__ __device__ inline int dn_unit_bytes(int F) {
@@ -115,7 +116,9 @@ __host__ __device__ inline Smem smem_layout(int fmt_ug, int H, int F, int T) {
   L.frag = NSLOT * slot;
   L.red = L.frag + ((xfrag > hfrag ? xfrag : hfrag) + 127) / 128 * 128;
   L.misc = L.red + (red_up > red_dn ? red_up : red_dn);
-  L.total = L.misc + 3072;
+  // activation scales: float 2^-sigma, then int sigma, [nxb][DEC_TMAX] each
+  L.xsc = L.misc + 3072;
+  L.total = L.xsc + ((H + XB_COLS - 1) / XB_COLS) * DEC_TMAX * 8;
   return L;
 }
 
@@ -123,9 +126,6 @@ __host__ __device__ inline Smem smem_layout(int fmt_ug, int H, int F, int T) {
 struct Misc {
   uint64_t full[NSLOT];
   uint64_t empty[NSLOT];
-  float xsc[DEC_TMAX];       // 2^-sigma_t (/8 for SB3)
-  int xsig[DEC_TMAX];
-  uint32_t xmax[DEC_TMAX];   // max |x| per token (float bits)
   int32_t tk_idx[MAXP];
   float tk_w[MAXP];
   int32_t sorted[MAXP];      // pair ids sorted by (expert, pair)
@@ -231,6 +231,11 @@ __global__ void __launch_bounds__(LAYER_THREADS, 1)
   uint8_t* ring = smem + L.ring;
   uint32_t* frag = reinterpret_cast<uint32_t*>(smem + L.frag);
   float* red = reinterpret_cast<float*>(smem + L.red);
+  // per (256-column block b, token t) at b * DEC_TMAX + t: 2^-sigma (/8 for
+  // SB3) and sigma of the activations' fixed-point scale
+  float* xsc = reinterpret_cast<float*>(smem + L.xsc);
+  const int nxb = (p.H + XB_COLS - 1) / XB_COLS;
+  int* xsig = reinterpret_cast<int*>(xsc + nxb * DEC_TMAX);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int H = p.H, F = p.F, T = p.T, k = p.k, E = p.E;
@@ -250,15 +255,14 @@ __global__ void __launch_bounds__(LAYER_THREADS, 1)
     }
     fence_mbar_init();
   }
-  if (tid < DEC_TMAX) M.xmax[tid] = 0u;
   for (int i = tid; i < MAXP; i += LAYER_THREADS) M.up_fin[i] = 0;
-  // launched as a programmatic dependent of the previous kernel on the
-  // stream: nothing in global memory is touched before that kernel is
-  // complete and its writes are visible
-  grid_dep_wait();
   // router rows of this block (not in DL_FFN): four warps per row, each a
-  // quarter of H; the first row chunk of every warp is loaded before x is
-  // staged, so that the two loads overlap
+  // quarter of H.  The kernel is launched as a programmatic dependent of
+  // the previous kernel on the stream, and the router weights are the one
+  // input that kernel does not produce: the first row chunk of every warp
+  // is loaded BEFORE the wait for it (griddepcontrol.wait), so that the
+  // load overlaps the end of the previous kernel; nothing else in global
+  // memory is touched before the wait.
   constexpr int RQ = 4, RCH = 4;
   const bool route = p.mode != DL_FFN;
   const int e0 = (int)((int64_t)E * blockIdx.x / G);
@@ -279,6 +283,7 @@ __global__ void __launch_bounds__(LAYER_THREADS, 1)
                     : make_uint4(0, 0, 0, 0);
     }
   }
+  grid_dep_wait();
   uint16_t* xs = reinterpret_cast<uint16_t*>(ring);   // [T][H] bf16
   if (p.x) {
     for (int i = tid; i < T * H / 8; i += LAYER_THREADS)
@@ -308,10 +313,9 @@ __global__ void __launch_bounds__(LAYER_THREADS, 1)
       if (warp < CW && r < nrow) {
         const uint4* row =
             reinterpret_cast<const uint4*>(p.wr + (int64_t)(e0 + r) * H);
-        float acc[TM], xm[TM];   // xm: max |x_t| over this quarter (row 0)
+        float acc[TM];
 #pragma unroll
-        for (int t = 0; t < TM; ++t) acc[t] = xm[t] = 0.f;
-        const bool track = base == 0 && r == 0;
+        for (int t = 0; t < TM; ++t) acc[t] = 0.f;
         for (int c0 = q * qch; c0 < (q + 1) * qch && c0 < nch; c0 += 32 * RCH) {
           uint4 w[RCH];
           const bool pre = base == 0 && c0 == q * qch;
@@ -341,15 +345,6 @@ __global__ void __launch_bounds__(LAYER_THREADS, 1)
                            __uint_as_float(xw[qq] & 0xFFFF0000u), a);
                 }
                 acc[t] = a;
-                if (track) {
-                  float m = xm[t];
-#pragma unroll
-                  for (int qq = 0; qq < 4; ++qq)
-                    m = fmaxf(m, fmaxf(fabsf(__uint_as_float(xw[qq] << 16)),
-                                       fabsf(__uint_as_float(xw[qq] &
-                                                             0xFFFF0000u))));
-                  xm[t] = m;
-                }
               }
             }
           }
@@ -360,13 +355,6 @@ __global__ void __launch_bounds__(LAYER_THREADS, 1)
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
           if (lane == 0 && t < T) part[(r * RQ + q) * DEC_TMAX + t] = a;
-          if (track) {
-            float m = xm[t];
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1)
-              m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-            if (lane == 0 && t < T) atomicMax(&M.xmax[t], __float_as_uint(m));
-          }
         }
       }
     }
@@ -384,35 +372,6 @@ __global__ void __launch_bounds__(LAYER_THREADS, 1)
   // ------------------------------------------------------------- P0|P1 --
   if (warp == SIGNALER && lane == 0) grid_arrive(p);
   if (warp < CW) {
-    if (p.mode != DL_ROUTE && !(route && nrow > 0)) {
-      // max |x_t| (the router's row-0 warps found it when they ran)
-      const int xt = tid, xn = CW * 32;
-      float m[TM];
-#pragma unroll
-      for (int t = 0; t < TM; ++t) m[t] = 0.f;
-      for (int i = xt; i < T * nch; i += xn) {
-        const int t = i / nch;
-        const uint4 v = reinterpret_cast<const uint4*>(xs)[i];
-        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-        float mm = 0.f;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          mm = fmaxf(mm, fabsf(__uint_as_float(w4[q] << 16)));
-          mm = fmaxf(mm, fabsf(__uint_as_float(w4[q] & 0xFFFF0000u)));
-        }
-#pragma unroll
-        for (int tt = 0; tt < TM; ++tt)
-          if (tt == t) m[tt] = fmaxf(m[tt], mm);
-      }
-#pragma unroll
-      for (int t = 0; t < TM; ++t) {
-        float a = m[t];
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1)
-          a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
-        if (lane == 0 && t < T) atomicMax(&M.xmax[t], __float_as_uint(a));
-      }
-    }
     grid_wait(p, 1);
   }
 
@@ -422,10 +381,24 @@ __global__ void __launch_bounds__(LAYER_THREADS, 1)
       // the warps without a top-k: per-token activation scale, then the
       // int8 hi/lo B fragments of x
       const int xt = tid - T * 32, xn = (CW - T) * 32;
-      if (xt < T) {
-        const int sg = pow2_sigma(__uint_as_float(M.xmax[xt]));
-        M.xsig[xt] = sg;
-        M.xsc[xt] = exp2i(-sg) * (FUG == MOE_SB3_256 ? 0.125f : 1.0f);
+      // max |x| per (token, 256-column block): one warp per pair, a lane
+      // per 8 values
+      for (int item = warp - T; item < T * nxb; item += CW - T) {
+        const int t = item / nxb, b = item % nxb;
+        const int ch = b * (XB_COLS / 8) + lane;
+        const float m0 =
+            ch < nch ? absmax8_bf16(reinterpret_cast<const uint4*>(xs)[t * nch + ch])
+                     : 0.f;
+        float m = m0;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+          m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if (lane == 0) {
+          const int sg = pow2_sigma(m);
+          xsig[b * DEC_TMAX + t] = sg;
+          xsc[b * DEC_TMAX + t] =
+              exp2i(-sg) * (FUG == MOE_SB3_256 ? 0.125f : 1.0f);
+        }
       }
       named_bar_sync(BAR_XF, xn);
       const int nent = (H / 32) * NT * 32;
@@ -435,7 +408,7 @@ __global__ void __launch_bounds__(LAYER_THREADS, 1)
         const int t = 4 * nt + (n >> 1);
         uint2 wv = make_uint2(0u, 0u);
         if (t < T) {
-          const float sc = exp2i(M.xsig[t]);
+          const float sc = exp2i(xsig[(32 * blk / XB_COLS) * DEC_TMAX + t]);
           const uint16_t* xr = xs + t * H + 32 * blk + 4 * cq;
           const uint2 a = *reinterpret_cast<const uint2*>(xr);
           const uint2 b = *reinterpret_cast<const uint2*>(xr + 16);
@@ -596,15 +569,18 @@ __global__ void __launch_bounds__(LAYER_THREADS, 1)
   if (warp == PRODUCER) {
     if (lane == 0) {
       int i = 0;
+      bool ok = true;   // false once a wait for a free slot gave up
       auto acquire = [&](int slot_i) {
         const int s = slot_i % NSLOT;
-        if (slot_i >= NSLOT)
-          mbar_wait(&M.empty[s], ((slot_i / NSLOT) - 1) & 1, p.err);
+        if (slot_i >= NSLOT &&
+            !mbar_wait(&M.empty[s], ((slot_i / NSLOT) - 1) & 1, p.err))
+          ok = false;
         return s;
       };
       for (; i < n_up; ++i) {
         const int v = b0 + i * G;
         const int s = acquire(i);
+        if (!ok) break;
         const int u = v / nrt_f, rt = v % nrt_f;
         const uint8_t* b = expert_base(p, M.active[u]);
         if (!b) { mbar_arrive_expect_tx(&M.full[s], 0); continue; }
@@ -614,8 +590,9 @@ __global__ void __launch_bounds__(LAYER_THREADS, 1)
         bulk_g2s(dst, b + (int64_t)rt * nb, nb, &M.full[s]);
         bulk_g2s(dst + nb, b + p.gate_off + (int64_t)rt * nb, nb, &M.full[s]);
       }
-      for (int v = d0; v < d1; v += dps, ++i) {
+      for (int v = d0; ok && v < d1; v += dps, ++i) {
         const int s = acquire(i);
+        if (!ok) break;
         const int n = (d1 - v) < dps ? (d1 - v) : dps;
         uint32_t tot = 0;
         const uint8_t* src[DNG];
@@ -630,6 +607,15 @@ __global__ void __launch_bounds__(LAYER_THREADS, 1)
           if (src[j])
             bulk_g2s(ring + s * L.slot_bytes + j * dnb, src[j], (uint32_t)dnb,
                      &M.full[s]);
+      }
+      // Fills 0 .. i-1 were issued.  None may still be in flight when the
+      // block exits (after a timed-out wait the compute warps stop waiting
+      // for them), so wait -- bounded, and without the early give-up of
+      // mbar_wait -- for the last fill of every slot to land.
+      for (int s = 0; s < NSLOT && s < i; ++s) {
+        const int last = s + ((i - 1 - s) / NSLOT) * NSLOT;
+        if (!mbar_wait_drain(&M.full[s], (last / NSLOT) & 1))
+          set_err(p.err, MOE_ERR_TIMEOUT);
       }
     }
     return;
@@ -746,9 +732,6 @@ __global__ void __launch_bounds__(LAYER_THREADS, 1)
   {
     const int ug = warp / UPW, wg = warp % UPW;
     float* rb = red + ug * red_up_floats(NT);
-    float xs2[2];
-    xs2[0] = M.xsc[c];
-    xs2[1] = M.xsc[4 + c];
     int mine = 0;
     for (int i = 0; i < n_up; ++i, ++slot_i) {
       if ((i & 1) != ug) continue;            // the other group's unit
@@ -761,12 +744,14 @@ __global__ void __launch_bounds__(LAYER_THREADS, 1)
         const int tz = pc / nk, kt = pc % nk;
         const uint8_t* tp = unit + pc * TBU;
         const uint32_t* xf = frag + kt * (TCU / 32) * NT * 64;
+        const float* xb = xsc + (kt * TCU / XB_COLS) * DEC_TMAX;
         if (FUG == MOE_SB3_256) {
+          const float xs2[2] = {xb[c], xb[4 + c]};
           if (tz == 0) piece_sb3(tp, xf, NT, xs2, au, lane, NT);
           else piece_sb3(tp, xf, NT, xs2, ag, lane, NT);
         } else {
-          if (tz == 0) piece_b32<FUG>(tp, xf, NT, M.xsc + c, 0, au, lane, NT);
-          else piece_b32<FUG>(tp, xf, NT, M.xsc + c, 0, ag, lane, NT);
+          if (tz == 0) piece_b32<FUG>(tp, xf, NT, xb + c, 0, au, lane, NT);
+          else piece_b32<FUG>(tp, xf, NT, xb + c, 0, ag, lane, NT);
         }
       }
       __syncwarp();

@@ -122,6 +122,22 @@ __device__ __forceinline__ void piece_b32(const uint8_t* tp,
   }
 }
 
+// Columns of x that share one activation scale in the decode kernels: a
+// large value in one channel coarsens only the other values of its block.
+constexpr int XB_COLS = 256;
+
+// max |v| of 8 bf16 values packed in a 16-byte word.
+__device__ __forceinline__ float absmax8_bf16(const uint4 v) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  float m = 0.f;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    m = fmaxf(m, fabsf(__uint_as_float(w[q] << 16)));
+    m = fmaxf(m, fabsf(__uint_as_float(w[q] & 0xFFFF0000u)));
+  }
+  return m;
+}
+
 // 2^sigma with sigma chosen so that max|v| * 2^sigma < 2^14.
 __device__ __forceinline__ int pow2_sigma(float m) {
   if (!(m > 0.f) || !isfinite(m)) return 0;

@@ -8,7 +8,8 @@
 // alternate units.  A consumer turns the codes of its tile into the int8
 // A fragment of mma.m16n8k32 with byte-table lookups (prmt), and the
 // activations enter as the B fragment split into two int8 halves
-// (v = 256*hi + lo, v = round(a * 2^sigma), |v| < 2^14), so the products
+// (v = 256*hi + lo, v = round(a * 2^sigma), |v| < 2^14, with one sigma per
+// token and 256-column block of x), so the products
 // and their sums over a 32-block are exact integers.  Scales are applied
 // in fp32 per block (per super-block for SB3, whose sub-scales multiply
 // the integer partials).
@@ -85,9 +86,11 @@ __global__ void __launch_bounds__(DEC_THREADS, 1)
   uint32_t* xf = reinterpret_cast<uint32_t*>(smem + UP_STAGES * stage_bytes);
   uint64_t* full = reinterpret_cast<uint64_t*>(xf + nblk * BF_NT * 64);
   uint64_t* empty = full + UP_STAGES;
-  float* xsc = reinterpret_cast<float*>(empty + UP_STAGES);  // [8]
-  int* xsig = reinterpret_cast<int*>(xsc + DEC_TMAX);        // [8]
-  int* flag = xsig + DEC_TMAX;                               // [NGRP]
+  // activation scales per (256-column block, token): [nxb][8]
+  const int nxb = (p.H + XB_COLS - 1) / XB_COLS;
+  float* xsc = reinterpret_cast<float*>(empty + UP_STAGES);
+  int* xsig = reinterpret_cast<int*>(xsc + nxb * DEC_TMAX);
+  int* flag = xsig + nxb * DEC_TMAX;                         // [NGRP]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
@@ -97,18 +100,25 @@ __global__ void __launch_bounds__(DEC_THREADS, 1)
     }
     fence_mbar_init();
   }
-  // per-token scale of the activations (x is an input of this layer)
-  for (int t = warp; t < p.T; t += DEC_THREADS / 32) {
+  // scale of the activations per token and 256-column block (x is an
+  // input of this layer): one warp per (token, block), a lane per 8 values
+  for (int item = warp; item < p.T * nxb; item += DEC_THREADS / 32) {
+    const int t = item / nxb, b = item % nxb;
+    const int h0 = b * XB_COLS + 8 * lane;
     float m = 0.f;
-    for (int h = lane; h < p.H; h += 32)
-      m = fmaxf(m, fabsf(bf16_to_f32(p.x[(int64_t)t * p.H + h])));
+    if (h0 < p.H) {
+      const uint4 v =
+          *reinterpret_cast<const uint4*>(p.x + (int64_t)t * p.H + h0);
+      m = absmax8_bf16(v);
+    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1)
       m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
     if (lane == 0) {
       const int s = pow2_sigma(m);
-      xsig[t] = s;
-      xsc[t] = exp2i(-s) * (FMT == MOE_SB3_256 ? 0.125f : 1.0f);
+      xsig[b * DEC_TMAX + t] = s;
+      xsc[b * DEC_TMAX + t] =
+          exp2i(-s) * (FMT == MOE_SB3_256 ? 0.125f : 1.0f);
     }
   }
   __syncthreads();
@@ -121,7 +131,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 1)
     const int t = 4 * nt + (n >> 1);
     uint32_t word = 0;
     if (t < p.T) {
-      const float sc = exp2i(xsig[t]);
+      const float sc = exp2i(xsig[(32 * blk / XB_COLS) * DEC_TMAX + t]);
       const uint16_t* xr = p.x + (int64_t)t * p.H + 32 * blk + 16 * reg + 4 * c;
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
@@ -172,9 +182,6 @@ __global__ void __launch_bounds__(DEC_THREADS, 1)
   const int gtid = tid - grp * GRP_WARPS * 32;   // 0..127 within the group
   const int tz = wg >> 1, rg = wg & 1;
   const int g = lane >> 2, c = lane & 3;
-  float xs[2];
-  xs[0] = xsc[c];
-  xs[1] = xsc[4 + c];
   for (int i = grp; i < nu; i += NGRP) {
     const int s = i % UP_STAGES;
     mbar_wait(&full[s], (i / UP_STAGES) & 1, p.err);
@@ -186,11 +193,14 @@ __global__ void __launch_bounds__(DEC_THREADS, 1)
     const uint8_t* chunk = stages + s * stage_bytes + wg * chunk_bytes;
     for (int kt = 0; kt < k1 - k0; ++kt) {
       const int blk0 = (k0 + kt) * (TC / 32);
-      if (FMT == MOE_SB3_256)
+      const float* xb = xsc + ((k0 + kt) * TC / XB_COLS) * DEC_TMAX;
+      if (FMT == MOE_SB3_256) {
+        const float xs[2] = {xb[c], xb[4 + c]};
         piece_sb3(chunk + kt * TB, xf + blk0 * BF_NT * 64, NT, xs, acc, lane);
-      else
-        piece_b32<FMT>(chunk + kt * TB, xf + blk0 * BF_NT * 64, NT, xsc + c,
+      } else {
+        piece_b32<FMT>(chunk + kt * TB, xf + blk0 * BF_NT * 64, NT, xb + c,
                        0, acc, lane);
+      }
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
@@ -422,8 +432,9 @@ static size_t up_smem_bytes(int fmt, int H) {
   const int nk = H / TC;
   const int nsplit = nk < NSPLIT_MAX ? nk : NSPLIT_MAX;
   const int kmax = (nk + nsplit - 1) / nsplit;
+  const int nxb = (H + XB_COLS - 1) / XB_COLS;
   return (size_t)UP_STAGES * 4 * kmax * TB + (size_t)(H / 32) * BF_NT * 64 * 4 +
-         2 * UP_STAGES * 8 + 2 * DEC_TMAX * 4 + 64;
+         2 * UP_STAGES * 8 + (size_t)2 * nxb * DEC_TMAX * 4 + 64;
 }
 static size_t dn_smem_bytes(int F) {
   const int nk = F / B32_TILE_COLS, nblk = F / 32;

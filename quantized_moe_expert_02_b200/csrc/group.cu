@@ -168,6 +168,8 @@ moe_status launch_group(const int32_t* idx, int T, int k, int E,
 // capture that the caller does not own, real-time loops that forbid
 // allocation -- this variant keeps its scratch in a fixed array in the
 // library's own device memory instead of a workspace.
+#include <cuda.h>
+
 #include <mutex>
 
 namespace moe {
@@ -184,22 +186,44 @@ constexpr size_t STATIC_GROUP_WORDS =
 
 static __device__ __align__(256) int32_t g_group_scratch[STATIC_GROUP_WORDS];
 
-// Device address of the scratch array on the current device, looked up
-// once per device (the array's name is only a host-side stand-in).
+// Device address of the scratch array in the current context, looked up
+// once per (device, context) with that device current (the array's name is
+// only a host-side stand-in).  A symbol's address belongs to a context: a
+// second context on the device gets its own lookup.
 moe_status group_scratch_address(int32_t** out) {
-  static int32_t* addr[64] = {};
+  using CtxGetCurrent = CUresult (*)(CUcontext*);
+  struct Entry { int dev; CUcontext ctx; int32_t* addr; };
+  static Entry seen[64];
+  static int n_seen = 0;
+  static CtxGetCurrent ctx_get = nullptr;
   static std::mutex mu;
   int dev = 0;
   MOE_CUDA_TRY(cudaGetDevice(&dev));
-  if (dev < 0 || dev >= 64) return MOE_ERR_CUDA;
   std::lock_guard<std::mutex> lock(mu);
-  if (!addr[dev]) {
-    void* p = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&p, g_group_scratch);
-    if (e != cudaSuccess || !p) return MOE_ERR_CUDA;
-    addr[dev] = static_cast<int32_t*>(p);
+  if (!ctx_get) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault,
+                                &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !f)
+      return MOE_ERR_CUDA;
+    ctx_get = reinterpret_cast<CtxGetCurrent>(f);
   }
-  *out = addr[dev];
+  CUcontext ctx = nullptr;
+  if (ctx_get(&ctx) != CUDA_SUCCESS) return MOE_ERR_CUDA;
+  if (ctx)
+    for (int i = 0; i < n_seen; ++i)
+      if (seen[i].dev == dev && seen[i].ctx == ctx) {
+        *out = seen[i].addr;
+        return MOE_OK;
+      }
+  // the lookup makes the device's primary context current if none was
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_group_scratch);
+  if (e != cudaSuccess || !p) return MOE_ERR_CUDA;
+  if (!ctx && (ctx_get(&ctx) != CUDA_SUCCESS || !ctx)) return MOE_ERR_CUDA;
+  if (n_seen < 64) seen[n_seen++] = Entry{dev, ctx, static_cast<int32_t*>(p)};
+  *out = static_cast<int32_t*>(p);
   return MOE_OK;
 }
 

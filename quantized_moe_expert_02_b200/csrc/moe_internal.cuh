@@ -242,6 +242,16 @@ __device__ __forceinline__ bool mbar_wait(void* bar, uint32_t parity,
   return true;
 }
 
+// Wait for the phase of `parity` to complete, bounded by 0.5 s of
+// %globaltimer but without mbar_wait's early return after another wait of
+// the launch gave up: for draining copies that are in flight.
+__device__ __forceinline__ bool mbar_wait_drain(void* bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer();
+  while (!mbar_try_wait_sleep(bar, parity, 20000u))
+    if (globaltimer() - t0 > 500000000ull) return false;
+  return true;
+}
+
 // 1-D bulk copy global -> shared, completion counted on `bar`.  Addresses
 // 16-byte aligned, size a multiple of 16.
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src,

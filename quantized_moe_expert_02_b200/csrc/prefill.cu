@@ -275,6 +275,61 @@ __device__ __forceinline__ void b32_store(const B32Q& q, int g, int p,
     }
 }
 
+// ------------------------------------------------------ tile export --
+// The A operand tiles exactly as the dequant warps of pf_gemm_kernel write
+// them (same loads, same stores, same thread mapping), for one 128-row
+// block and one group of k-steps -- SB3: the four 64-column k-steps of a
+// super-block (group gamma writes k-steps gamma and gamma + 2); Q4/NL4: two
+// k-steps, one per group -- then un-swizzled to fp16 [rows][cols].  Used
+// only by moe_dequant_path, to check these decoders bit for bit.
+template <bool SB3>
+__global__ void __launch_bounds__(256)
+    pf_dequant_export_kernel(const uint8_t* __restrict__ t, int cols,
+                             uint4 tab4, uint16_t* __restrict__ out) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  const uint8_t* smem = smem_raw + (sbase - raw);
+  constexpr int NKS = SB3 ? 4 : 2;   // k-steps of one block
+  const int gamma = threadIdx.x >> 7, tt = threadIdx.x & 127;
+  const int tg = tt & 7, tp_ = (tt >> 3) & 1, tti = tt >> 4;
+  const int m = blockIdx.x, kg = blockIdx.y;
+  const int tcols = SB3 ? SB3_TILE_COLS : B32_TILE_COLS;
+  const int tbytes = SB3 ? SB3_TILE_BYTES : B32_TILE_BYTES;
+  const int64_t trow_stride = (int64_t)(cols / tcols) * tbytes;
+  const uint8_t* ptp = t + (int64_t)(m * (PF_BM / 16) + tti) * trow_stride;
+  const int nks_total = cols / PF_BK;
+  if constexpr (SB3) {
+    Sb3Half q;
+    sb3_load(ptp + (int64_t)kg * SB3_TILE_BYTES, tg, tp_, gamma, q);
+#pragma unroll
+    for (int qh = 0; qh < 2; ++qh)
+      sb3_store(q, tg, tp_, gamma, qh, 16 * tti,
+                sbase + (uint32_t)((gamma + 2 * qh) * PF_A_BYTES));
+  } else {
+    const B32Tab tab = {tab4.x, tab4.y, tab4.z, tab4.w};
+    const int ks = NKS * kg + gamma;
+    if (ks < nks_total) {
+      const B32Q q = b32_load(ptp + (int64_t)ks * B32_TILE_BYTES, tg, tp_);
+#pragma unroll
+      for (int rh = 0; rh < 2; ++rh)
+        b32_store(q, tg, tp_, rh, 16 * tti, tab,
+                  sbase + (uint32_t)(gamma * PF_A_BYTES));
+    }
+  }
+  __syncthreads();
+  // 16-byte chunk ch of row r of k-step q holds columns 8ch .. 8ch+7
+  for (int i = threadIdx.x; i < NKS * PF_BM * 8; i += blockDim.x) {
+    const int q = i / (PF_BM * 8), r = (i / 8) % PF_BM, ch = i % 8;
+    const int ksg = kg * NKS + q;
+    if (ksg >= nks_total) continue;
+    const uint4 v = *reinterpret_cast<const uint4*>(smem + q * PF_A_BYTES +
+                                                    sw128(r, ch));
+    *reinterpret_cast<uint4*>(out + (int64_t)(PF_BM * m + r) * cols +
+                              ksg * PF_BK + 8 * ch) = v;
+  }
+}
+
 // --------------------------------------------------------------- kernel --
 // maps: up: x_g [P][H], down: h16 [P][F], both fp16 in grouped row
 // order, boxes of 64 columns, 128-byte swizzle.
@@ -757,6 +812,33 @@ static void pf_tables(int fmt, uint32_t (&t)[4]) {
   } else {
     t[0] = Q4_TA0; t[1] = Q4_TA1; t[2] = Q4_TB0; t[3] = Q4_TB1;
   }
+}
+
+bool pf_export_supported(int fmt, int rows, int cols) {
+  return rows > 0 && cols > 0 && rows % PF_BM == 0 &&
+         cols % (fmt == MOE_SB3_256 ? SB3_TILE_COLS : B32_TILE_COLS) == 0;
+}
+
+moe_status launch_pf_dequant_export(int fmt, const uint8_t* t, int rows,
+                                    int cols, uint16_t* out, cudaStream_t s) {
+  uint32_t tb[4] = {0u, 0u, 0u, 0u};
+  if (fmt != MOE_SB3_256) pf_tables(fmt, tb);
+  const uint4 tab4 = make_uint4(tb[0], tb[1], tb[2], tb[3]);
+  const bool sb3 = fmt == MOE_SB3_256;
+  const int nks = sb3 ? 4 : 2;
+  const size_t smem = (size_t)nks * PF_A_BYTES + 1024;
+  const void* fn = sb3 ? (const void*)&pf_dequant_export_kernel<true>
+                       : (const void*)&pf_dequant_export_kernel<false>;
+  moe_status st = ensure_smem(fn, smem);
+  if (st != MOE_OK) return st;
+  const dim3 grid(rows / PF_BM, sb3 ? cols / SB3_TILE_COLS
+                                    : (cols / PF_BK + 1) / 2);
+  if (sb3)
+    pf_dequant_export_kernel<true><<<grid, 256, smem, s>>>(t, cols, tab4, out);
+  else
+    pf_dequant_export_kernel<false><<<grid, 256, smem, s>>>(t, cols, tab4,
+                                                            out);
+  return launch_status();
 }
 
 // fp16 [outer][inner] row-major tensor map with the 128-byte swizzle and

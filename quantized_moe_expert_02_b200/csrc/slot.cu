@@ -13,7 +13,8 @@ __global__ void __launch_bounds__(1024)
     slot_resolve_kernel(const int32_t* __restrict__ topk_idx, int P, int E,
                         int32_t* __restrict__ table, int32_t* __restrict__ owner,
                         uint32_t* __restrict__ last_use, int n_slots,
-                        int slot_base, uint32_t stamp,
+                        int slot_base, uint32_t stamp_arg,
+                        uint32_t* stamp_ctr,
                         int32_t* __restrict__ blob_index,
                         int32_t* __restrict__ miss_expert,
                         int32_t* __restrict__ miss_slot,
@@ -25,6 +26,9 @@ __global__ void __launch_bounds__(1024)
   __shared__ int32_t s_nmiss, s_nhit, s_bad;
   __shared__ unsigned long long s_best;
   const int tid = threadIdx.x;
+  // with a device counter, this call's stamp is the counter + 1 (stored
+  // back below, once the call updates the partition)
+  const uint32_t stamp = stamp_ctr ? *stamp_ctr + 1u : stamp_arg;
   for (int e = tid; e < E; e += blockDim.x) chosen[e] = 0;
   for (int s = tid; s < n_slots; s += blockDim.x) used[s] = 0;
   if (tid == 0) { s_nmiss = 0; s_nhit = 0; s_bad = 0; }
@@ -104,6 +108,7 @@ __global__ void __launch_bounds__(1024)
       miss_slot[i] = v;
     }
     *n_miss = nm;
+    if (stamp_ctr) *stamp_ctr = stamp;
   }
   __syncthreads();
   for (int e = tid; e < E; e += blockDim.x)
@@ -116,15 +121,13 @@ __global__ void __launch_bounds__(1024)
 
 using namespace moe;
 
-extern "C" moe_status moe_slot_resolve(const int32_t* topk_idx, int T, int k,
-                                       int E, int32_t* slot_table,
-                                       int32_t* slot_owner,
-                                       uint32_t* last_use, int n_slots,
-                                       int slot_base, uint32_t stamp,
-                                       int32_t* blob_index,
-                                       int32_t* miss_expert,
-                                       int32_t* miss_slot, int32_t* n_miss,
-                                       int32_t* err, void* stream) {
+static moe_status slot_resolve(const int32_t* topk_idx, int T, int k, int E,
+                               int32_t* slot_table, int32_t* slot_owner,
+                               uint32_t* last_use, int n_slots, int slot_base,
+                               uint32_t stamp, uint32_t* stamp_ctr,
+                               int32_t* blob_index, int32_t* miss_expert,
+                               int32_t* miss_slot, int32_t* n_miss,
+                               int32_t* err, void* stream) {
   if (!topk_idx || !slot_table || !slot_owner || !last_use || !blob_index ||
       !miss_expert || !miss_slot || !n_miss || !err)
     return MOE_ERR_INVALID;
@@ -134,6 +137,32 @@ extern "C" moe_status moe_slot_resolve(const int32_t* topk_idx, int T, int k,
     return MOE_ERR_SHAPE;
   slot_resolve_kernel<<<1, 1024, 0, (cudaStream_t)stream>>>(
       topk_idx, T * k, E, slot_table, slot_owner, last_use, n_slots,
-      slot_base, stamp, blob_index, miss_expert, miss_slot, n_miss, err);
+      slot_base, stamp, stamp_ctr, blob_index, miss_expert, miss_slot, n_miss,
+      err);
   return launch_status();
+}
+
+extern "C" moe_status moe_slot_resolve(const int32_t* topk_idx, int T, int k,
+                                       int E, int32_t* slot_table,
+                                       int32_t* slot_owner,
+                                       uint32_t* last_use, int n_slots,
+                                       int slot_base, uint32_t stamp,
+                                       int32_t* blob_index,
+                                       int32_t* miss_expert,
+                                       int32_t* miss_slot, int32_t* n_miss,
+                                       int32_t* err, void* stream) {
+  return slot_resolve(topk_idx, T, k, E, slot_table, slot_owner, last_use,
+                      n_slots, slot_base, stamp, nullptr, blob_index,
+                      miss_expert, miss_slot, n_miss, err, stream);
+}
+
+extern "C" moe_status moe_slot_resolve_dev(
+    const int32_t* topk_idx, int T, int k, int E, int32_t* slot_table,
+    int32_t* slot_owner, uint32_t* last_use, int n_slots, int slot_base,
+    uint32_t* stamp, int32_t* blob_index, int32_t* miss_expert,
+    int32_t* miss_slot, int32_t* n_miss, int32_t* err, void* stream) {
+  if (!stamp) return MOE_ERR_INVALID;
+  return slot_resolve(topk_idx, T, k, E, slot_table, slot_owner, last_use,
+                      n_slots, slot_base, 0u, stamp, blob_index, miss_expert,
+                      miss_slot, n_miss, err, stream);
 }

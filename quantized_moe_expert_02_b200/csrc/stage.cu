@@ -25,7 +25,7 @@ constexpr int STAGE_UNROLL = 4;   // 16-byte loads in flight per thread
 __global__ void __launch_bounds__(STAGE_THREADS)
     stage_misses_kernel(const int32_t* n_miss, const int32_t* miss_expert,
                         const int32_t* miss_slot, int P, int layer, int E,
-                        int slot_base, int64_t pool_slots,
+                        int slot_base, int n_slots, int64_t pool_slots,
                         const uint64_t* table, uint8_t* pool, int64_t stride,
                         int64_t blob_bytes, int32_t* err) {
   const int n = *n_miss;
@@ -48,11 +48,13 @@ __global__ void __launch_bounds__(STAGE_THREADS)
       const int m = (int)(i / words);
       const int64_t w = i % words;
       const int e = miss_expert[m];
-      const int64_t slot = (int64_t)slot_base + miss_slot[m];
+      const int ls = miss_slot[m];   // slot inside the layer's partition
+      const int64_t slot = (int64_t)slot_base + ls;
       const uint64_t src = (e >= 0 && e < E) ? table[(int64_t)layer * E + e]
                                              : 0ull;
-      if (src == 0ull || slot < 0 || slot >= pool_slots) {
-        if (w == 0) set_err(err, MOE_ERR_CAPACITY);   // no host copy
+      // no host copy, or a slot outside the layer's partition: skipped
+      if (src == 0ull || ls < 0 || ls >= n_slots || slot >= pool_slots) {
+        if (w == 0) set_err(err, MOE_ERR_CAPACITY);
         continue;
       }
       v[u] = reinterpret_cast<const uint4*>(src)[w];
@@ -105,20 +107,22 @@ extern "C" moe_status moe_stage_misses(const int32_t* n_miss,
                                        int layer, int L, int E,
                                        const uint64_t* table,
                                        uint8_t* pool, int slot_base,
-                                       int64_t pool_slots,
+                                       int n_slots, int64_t pool_slots,
                                        int64_t blob_stride,
                                        int64_t blob_bytes, int32_t* err,
                                        void* stream) {
   if (!n_miss || !miss_expert || !miss_slot || !table || !pool)
     return MOE_ERR_INVALID;
   if (P < 1 || layer < 0 || layer >= L || E < 1 || slot_base < 0 ||
-      pool_slots < 1 ||
+      n_slots < 1 || pool_slots < 1 ||
+      slot_base + (int64_t)n_slots > pool_slots ||
       blob_bytes < 16 || blob_bytes % 16 || blob_stride % 16 ||
       blob_stride < blob_bytes || reinterpret_cast<uintptr_t>(pool) % 16)
     return MOE_ERR_SHAPE;
   moe::stage_misses_kernel<<<moe::num_sms(), moe::STAGE_THREADS, 0,
                              (cudaStream_t)stream>>>(
-      n_miss, miss_expert, miss_slot, P, layer, E, slot_base, pool_slots,
+      n_miss, miss_expert, miss_slot, P, layer, E, slot_base, n_slots,
+      pool_slots,
       table, pool, blob_stride, blob_bytes, err);
   return moe::launch_status();
 }

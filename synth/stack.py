@@ -102,7 +102,7 @@ class SlotPool:
         self.pool = torch.empty(n_slots * stride, dtype=torch.uint8,
                                 device="cuda")
         E = shp.E
-        self.reset()
+        self._reset_slots()
         self.descs = [layer_desc(shp, self.pool) for _ in self.caps]
         # pinned host store, filled from the resident pools
         self.device_source = store_keys is None
@@ -130,7 +130,7 @@ class SlotPool:
         # copy), so that more than one copy engine moves them
         self.copy_streams = [torch.cuda.Stream() for _ in range(copy_streams)]
 
-    def reset(self) -> None:
+    def _reset_slots(self) -> None:
         """The starting state: each layer's slots hold its hottest experts,
         every last-use stamp is zero."""
         torch, st, E = self.torch, self.stack, self.stack.shape.E
@@ -211,7 +211,10 @@ class SlotPool:
     def start_staging(self) -> None:
         """Miss handling without a host round trip per layer: after the
         resolve, moe_stage_misses pulls each missed blob from the pinned
-        host store into its slot on the same stream."""
+        host store into its slot on the same stream.  The resolve keeps its
+        LRU stamp in a per-layer device counter (moe_slot_resolve_dev), so
+        that no host argument changes from one step to the next and a whole
+        step can be captured once as a CUDA graph."""
         torch, moe = self.torch, self.moe
         assert not self.device_source, "in-stream staging needs a host store"
         L, E = len(self.caps), self.stack.shape.E
@@ -221,27 +224,48 @@ class SlotPool:
         self.table_dev = torch.zeros(L * E, dtype=torch.int64, device="cuda")
         moe.moe_stage_table(table, self.table_dev)
         self.n_slots = int(sum(self.caps))
+        # stamp counters: counter l = number of steps layer l has resolved
+        self.stamps = torch.zeros(L, dtype=torch.int32, device="cuda")
 
-    def layer_staged(self, l: int, r, stamp: int) -> None:
+    def reset(self) -> None:
+        self._reset_slots()
+        if hasattr(self, "stamps"):
+            self.stamps.zero_()
+
+    def layer_staged(self, l: int, r) -> None:
         """One layer through the slot pool, in place, with no host sync."""
         st, moe, shp = self.stack, self.moe, self.stack.shape
         T, k, E = st.T, shp.k, shp.E
         moe.moe_layer_route_residual(self.descs[l], r, T, k, st.wr[l],
                                      st.bias[l], st.idx, st.w, None, st.ws,
                                      st.ws_bytes)
-        moe.moe_slot_resolve(st.idx, T, k, E, self.table[l], self.owner[l],
-                             self.last[l], self.caps[l], int(self.base[l]),
-                             stamp, self.blob_index, self.mexp, self.mslot,
-                             self.nmiss, self.err)
+        moe.moe_slot_resolve_dev(st.idx, T, k, E, self.table[l],
+                                 self.owner[l], self.last[l], self.caps[l],
+                                 int(self.base[l]),
+                                 self.stamps.data_ptr() + 4 * l,
+                                 self.blob_index, self.mexp, self.mslot,
+                                 self.nmiss, self.err)
         moe.moe_stage_misses(self.nmiss, self.mexp, self.mslot, T * k, l,
                              len(self.caps), E, self.table_dev, self.pool,
-                             int(self.base[l]), self.n_slots, self.stride,
-                             self.blob, self.err)
+                             int(self.base[l]), self.caps[l], self.n_slots,
+                             self.stride, self.blob, self.err)
         moe.moe_layer_ffn_residual(self.descs[l], r, T, k, st.idx, st.w,
                                    self.blob_index, r, None, st.ws,
                                    st.ws_bytes)
 
-    def run_staged(self, r, stamp: int):
+    def run_staged(self, r):
+        """One step: every layer in order, in place on r."""
         for l in range(len(self.caps)):
-            self.layer_staged(l, r, stamp)
+            self.layer_staged(l, r)
         return r
+
+    def capture_step(self, x_in, r):
+        """The whole step -- r <- x_in, then route, resolve, pull and FFN of
+        every layer -- captured once as one CUDA graph; each replay runs
+        the next step (the slot state and the stamp counters live on the
+        device).  Returns the graph."""
+        g = self.torch.cuda.CUDAGraph()
+        with self.torch.cuda.graph(g):
+            r.copy_(x_in)
+            self.run_staged(r)
+        return g

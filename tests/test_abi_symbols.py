@@ -55,13 +55,14 @@ def test_stage_argument_errors_without_gpu():
 
     def stage(**kw):
         a = dict(n_miss=f, miss_expert=f, miss_slot=f, P=30, layer=0, L=48,
-                 E=512, table=f, pool=f, slot_base=0, pool_slots=4644,
+                 E=512, table=f, pool=f, slot_base=0, n_slots=240,
+                 pool_slots=4644,
                  blob_stride=4276224, blob_bytes=4276224, err=f, stream=None)
         a.update(kw)
         return lib.moe_stage_misses(
             a["n_miss"], a["miss_expert"], a["miss_slot"], a["P"],
             a["layer"], a["L"], a["E"], a["table"], a["pool"],
-            a["slot_base"], a["pool_slots"], a["blob_stride"],
+            a["slot_base"], a["n_slots"], a["pool_slots"], a["blob_stride"],
             a["blob_bytes"], a["err"], a["stream"])
 
     assert stage(n_miss=None) == moe.MOE_ERR_INVALID
@@ -74,6 +75,11 @@ def test_stage_argument_errors_without_gpu():
     assert stage(blob_stride=4276224 - 16) == moe.MOE_ERR_SHAPE  # < blob
     assert stage(pool=f + 8) == moe.MOE_ERR_SHAPE           # misaligned
     assert stage(pool_slots=0) == moe.MOE_ERR_SHAPE
+    assert stage(n_slots=0) == moe.MOE_ERR_SHAPE
+    # the layer's partition must lie inside the pool
+    assert stage(slot_base=4644 - 59, n_slots=60) == moe.MOE_ERR_SHAPE
+    assert lib.moe_slot_resolve_dev(f, 3, 10, 512, f, f, f, 60, 0, None, f,
+                                    f, f, f, f, None) == moe.MOE_ERR_INVALID
     table = (ctypes.c_void_p * 1)(None)
     assert lib.moe_stage_table(table, 0, f, None) == moe.MOE_ERR_INVALID
     assert lib.moe_stage_table(None, 1, f, None) == moe.MOE_ERR_INVALID

@@ -3,7 +3,7 @@
 Routings are built so that the per-expert token lists cross the 256-row
 unit boundary (exactly 256, 257, 512 rows), hit the 16-row MMA granularity
 (1, 15, 16, 17 rows) and leave experts empty; the full prefill chunk
-(9536 tokens, Zipf-skewed routing) is checked on sampled tokens."""
+(9536 tokens, Zipf-skewed routing) is checked on every row."""
 import numpy as np
 import pytest
 import torch
@@ -184,10 +184,12 @@ def test_prefill_h_overflow_sets_error_word():
     assert st == moe.MOE_ERR_DEVICE
 
 
-def test_prefill_layer_full_size_sampled():
+def test_prefill_layer_full_size_all_rows():
     """The prefill chunk: 9536 tokens, 512 experts top-10, Zipf(1.1)
-    routing bias; whole layer through moe_layer_forward, checked on
-    sampled tokens against the oracle (and run twice: bit-identical)."""
+    routing bias; whole layer through moe_layer_forward, every one of the
+    9536 output rows against the oracle (its expert FFNs run in a pool of
+    spawned worker processes), and run twice: bit-identical."""
+    from oracle_pool import expert_outputs
     shape = synth.BIG
     T = synth.WORKLOADS["prefill"].T
     k, E, H = shape.k, shape.E, shape.H
@@ -210,14 +212,17 @@ def test_prefill_layer_full_size_sampled():
     assert np.array_equal(got_idx, o.topk_select(lg.cpu().numpy(), k))
     got = out.cpu().numpy()
     assert np.isfinite(got).all()
-    # sampled tokens: the first, the last, and four more
-    rng = np.random.default_rng(11)
-    toks = sorted(set([0, T - 1] + list(rng.choice(T, 4, replace=False))))
-    src = oracle_experts(shape, 0, 0)
-    xs = o.bf16_to_f64(x[toks])
-    ref = o.moe_layer(xs, o.bf16_to_f64(wr), bias, k, src,
-                      topk_idx=got_idx[toks])
-    assert row_max_rel(got[toks], ref["out"]) <= TOL
+    del ws, outs
+    # the oracle: routing weights from its fp64 logits on the kernel's
+    # selection, every pair's expert FFN, the weighted combine
+    logits = o.router_logits(o.bf16_to_f64(x), o.bf16_to_f64(wr), bias)
+    p = o.softmax(logits)
+    ps = np.take_along_axis(p, got_idx.astype(np.int64), axis=1)
+    w_ref = ps / ps.sum(axis=1, keepdims=True)
+    y_ref = expert_outputs(shape, 0, 0, x, got_idx)
+    ref = o.combine(y_ref, w_ref)
+    del y_ref
+    assert row_max_rel(got, ref) <= TOL
 
 
 def test_prefill_past_int32_elements_sampled():

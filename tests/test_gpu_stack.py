@@ -8,7 +8,8 @@
   pinned host store, one copy per expert -- gives output bit-identical to
   the all-resident run, and the miss lists equal the oracle's LRU replay;
   the same holds with the misses pulled from the host store on the stream
-  (no host round trip per layer).
+  (no host round trip per layer), eagerly and as one CUDA graph per step,
+  and at the workload's real shape (48 layers, 240 / 92 / 60 slots).
 * The in-stream copy moves blobs byte for byte, rejects host memory that is
   not mapped pinned memory on the host, and reports a missing host copy or
   a bad miss count in the device error word.
@@ -140,18 +141,109 @@ def test_slot_cache_in_stream_staging_bit_exact_vs_resident():
     assert keys
     pool = SlotPool(st, [cap] * L, sorted(keys))
     pool.start_staging()
-    outs = [pool.run_staged(st.x0(s), s + 1).clone() for s in range(steps)]
+    outs = [pool.run_staged(st.x0(s)).clone() for s in range(steps)]
     for s in range(steps):
         assert torch.equal(outs[s], resident[s]), s
     assert int(pool.err.item()) == 0
     assert moe.moe_get_device_status(st.ws) == 0
-    # the slot tables end where the host-round-trip run ends
+    # the slot tables end where the host-round-trip run ends (host stamps
+    # = step numbers; the device counters reach the same values)
     ref = SlotPool(st, [cap] * L, sorted(keys))
     for s in range(steps):
         ref.run(st.x0(s), s + 1)
     for l in range(L):
         assert torch.equal(pool.table[l], ref.table[l])
         assert torch.equal(pool.owner[l], ref.owner[l])
+        assert torch.equal(pool.last[l], ref.last[l])
+    assert pool.stamps.tolist() == [steps] * L
+
+
+def test_slot_cache_step_as_one_graph_bit_exact():
+    """The slot-cache step (route, device-stamped resolve, in-stream pull
+    and FFN of every layer) captured once as one CUDA graph and replayed
+    once per step: bit-identical to the all-resident run on every step,
+    slot state equal to the eager run's."""
+    L, steps, cap = 3, 8, 32
+    st = stack_for(L)
+    resident, routing = [], []
+    for s in range(steps):
+        rec = []
+        resident.append(st.run_resident(st.x0(s), record=rec).clone())
+        routing.append([i.cpu().numpy() for i in rec])
+    expect, keys = _replay_misses(st, routing, L, steps, cap)
+    pool = SlotPool(st, [cap] * L, sorted(keys))
+    pool.start_staging()
+    x_in = st.x0(0)
+    r = torch.empty_like(x_in)
+    # capturing records the launches without running them
+    g = pool.capture_step(x_in, r)
+    torch.cuda.synchronize()
+    assert pool.stamps.tolist() == [0] * L
+    for s in range(steps):
+        x_in.copy_(st.x0(s))
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(r, resident[s]), s
+    assert int(pool.err.item()) == 0
+    assert moe.moe_get_device_status(st.ws) == 0
+    eager = SlotPool(st, [cap] * L, sorted(keys))
+    eager.start_staging()
+    for s in range(steps):
+        eager.run_staged(st.x0(s))
+    for l in range(L):
+        assert torch.equal(pool.table[l], eager.table[l])
+        assert torch.equal(pool.last[l], eager.last[l])
+    del g
+
+
+def test_slot_cache_full_capacities_48_layers():
+    """The slot-cache workload at its real shape: 48 layers, 240 / 92 / 60
+    slots per layer, Zipf-hot initial fill, 3 tokens per step.  Misses
+    copied after a host round trip (from the resident pools) and, in a
+    second pool, pulled in-stream from a pinned host store by one graph
+    replay per step: both bit-identical to the all-resident run on every
+    step; the miss lists and victims equal the oracle's LRU replay."""
+    L, steps = 48, 4
+    st = stack_for(L)
+    caps = [synth.slot_capacity(l) for l in range(L)]
+    assert caps[0] == 240 and caps[5] == 92 and caps[47] == 60
+    resident, routing = [], []
+    for s in range(steps):
+        rec = []
+        resident.append(st.run_resident(st.x0(s), record=rec).clone())
+        routing.append([i.cpu().numpy() for i in rec])
+    replay = [o.SlotCache(st.shape.E, caps[l], list(hottest(st, l, caps[l])))
+              for l in range(L)]
+    expect, keys = [], set()
+    for s in range(steps):
+        for l in range(L):
+            _, miss, victims = replay[l].resolve(routing[s][l], s + 1)
+            expect.append((l, s + 1, miss, victims))
+            keys.update((l, e) for e in miss)
+    assert keys
+    disc = SlotPool(st, caps, None)          # misses copied device to device
+    log = []
+    for s in range(steps):
+        r = disc.run(st.x0(s), s + 1, log)
+        assert torch.equal(r, resident[s]), s
+    assert log == expect
+    assert int(disc.err.item()) == 0
+    del disc
+    torch.cuda.empty_cache()
+    pool = SlotPool(st, caps, sorted(keys))  # pinned host store
+    pool.start_staging()
+    x_in = st.x0(0)
+    r = torch.empty_like(x_in)
+    g = pool.capture_step(x_in, r)
+    for s in range(steps):
+        x_in.copy_(st.x0(s))
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(r, resident[s]), s
+    assert int(pool.err.item()) == 0
+    assert moe.moe_get_device_status(st.ws) == 0
+    del g, pool
+    torch.cuda.empty_cache()
 
 
 def test_stage_misses_copies_and_errors():
@@ -167,9 +259,10 @@ def test_stage_misses_copies_and_errors():
     mexp = torch.tensor([2, 0, 3], dtype=torch.int32, device="cuda")
     mslot = torch.tensor([1, 0, 2], dtype=torch.int32, device="cuda")
     n = torch.tensor([3], dtype=torch.int32, device="cuda")
-    # layer 1, slot base 3: blobs (1,2) -> slot 4, (1,0) -> slot 3, (1,3) absent
-    moe.moe_stage_misses(n, mexp, mslot, 3, 1, L, E, table, pool, 3, slots,
-                         stride, blob, err)
+    # layer 1, partition of 3 slots at base 3: blobs (1,2) -> slot 4,
+    # (1,0) -> slot 3, (1,3) absent
+    moe.moe_stage_misses(n, mexp, mslot, 3, 1, L, E, table, pool, 3, 3,
+                         slots, stride, blob, err)
     torch.cuda.synchronize()
     assert int(err.item()) == moe.MOE_ERR_CAPACITY
     got = pool.cpu()
@@ -181,16 +274,31 @@ def test_stage_misses_copies_and_errors():
     err.zero_()
     pool.zero_()
     n[0] = 7
-    moe.moe_stage_misses(n, mexp, mslot, 3, 0, L, E, table, pool, 0, slots,
-                         stride, blob, err)
+    moe.moe_stage_misses(n, mexp, mslot, 3, 0, L, E, table, pool, 0, 3,
+                         slots, stride, blob, err)
     torch.cuda.synchronize()
     assert int(err.item()) == moe.MOE_ERR_DEVICE
     assert int(pool.sum()) == 0
+    # a victim slot inside the pool but outside the layer's partition (a
+    # corrupted miss list): that blob is skipped, the other one copied
+    err.zero_()
+    n[0] = 2
+    bad = torch.tensor([3, 1, 0], dtype=torch.int32, device="cuda")
+    moe.moe_stage_misses(n, mexp, bad, 3, 0, L, E, table, pool, 0, 3, slots,
+                         stride, blob, err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == moe.MOE_ERR_CAPACITY
+    got = pool.cpu()
+    assert int(got[3 * stride:4 * stride].sum()) == 0     # not overwritten
+    assert torch.equal(got[1 * stride:1 * stride + blob], host[0 * E + 0])
     # host memory that is not pinned, and a layer outside the table, are
     # argument errors found on the host
     plain = torch.zeros(blob, dtype=torch.uint8)
     with pytest.raises(moe.MoeError):
         moe.moe_stage_table([plain.data_ptr()], table)
     with pytest.raises(moe.MoeError):
-        moe.moe_stage_misses(n, mexp, mslot, 3, L, L, E, table, pool, 0,
+        moe.moe_stage_misses(n, mexp, mslot, 3, L, L, E, table, pool, 0, 3,
+                             slots, stride, blob, err)
+    with pytest.raises(moe.MoeError):        # partition past the pool
+        moe.moe_stage_misses(n, mexp, mslot, 3, 0, L, E, table, pool, 4, 3,
                              slots, stride, blob, err)

@@ -49,6 +49,38 @@ def test_static_grouping_matches_workspace_grouping(T, k, E):
         assert np.array_equal(s_pairs, r_pairs)
 
 
+def test_static_grouping_at_capacity_allocates_nothing():
+    """The largest sizes the fixed array holds (T*k = 262144 pairs over
+    E = 1024 experts fill every per-chunk histogram row), against the
+    workspace call; and the device's free memory is the same before and
+    after a call (the call itself allocates nothing)."""
+    T, k, E = 32768, 8, 1024
+    rng = np.random.default_rng(5)
+    idx = np.argsort(rng.random((T, E)), axis=1)[:, :k].astype(np.int32)
+    off, pairs, act, err, _ = run_group(idx, E)
+    assert err == 0
+    d_idx = dev(idx)
+    s_off = torch.full((E + 1,), -9, dtype=torch.int32, device="cuda")
+    s_pairs = torch.full((T * k,), -9, dtype=torch.int32, device="cuda")
+    s_act = torch.full((E,), -9, dtype=torch.int32, device="cuda")
+    na = torch.full((1,), -9, dtype=torch.int32, device="cuda")
+    for _ in range(2):      # the first call has looked the array up
+        moe.moe_group_tokens_static(d_idx, T, k, E, s_off, s_pairs, s_act,
+                                    na, None)
+        torch.cuda.synchronize()
+        free0, _ = torch.cuda.mem_get_info()
+        used0 = torch.cuda.memory_allocated()
+        s_pairs.fill_(-9)
+        moe.moe_group_tokens_static(d_idx, T, k, E, s_off, s_pairs, s_act,
+                                    na, None)
+        torch.cuda.synchronize()
+        assert torch.cuda.mem_get_info()[0] == free0
+        assert torch.cuda.memory_allocated() == used0
+        assert np.array_equal(s_off.cpu().numpy(), off)
+        assert np.array_equal(s_pairs.cpu().numpy(), pairs)
+        assert np.array_equal(s_act.cpu().numpy()[:int(na.item())], act)
+
+
 def test_static_grouping_reports_bad_ids_and_rejects_large_sizes():
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
     idx = np.array([[0, 3], [99, 1]], np.int32)
