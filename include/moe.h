@@ -287,8 +287,13 @@ moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream);
  *   blob_index int32 [E] or NULL (NULL: expert e's blob is blob e); a
  *              negative entry of a chosen expert sets MOE_ERR_DEVICE
  * Needs H, F multiples of 256 (SB3) or 64 (Q4/NL4) and of 16.
- * T <= 8: exact int8 tensor-core decode kernels (activations split into
- *   int8 halves, fp32 scale folds).
+ * T <= 8: int8 tensor-core decode kernels.  The weights enter exactly
+ *   (int8 codes, integer sub-scale folds, fp32 scales); the activations
+ *   are rounded to 15-bit fixed point with one power-of-two scale per
+ *   token and 256-column block (split into two int8 halves), h with one
+ *   per pair; the integer block sums are exact, the scales apply in fp32.
+ *   A bf16 activation keeps every bit when it is at least 2^-6 times the
+ *   largest magnitude of its 256-column block.
  * T > 8 with H, F multiples of 128 (the prefill path): grouped GEMMs on the
  *   5th-generation tensor cores in fp16 with fp32 accumulation.  Each
  *   weight enters as the round-to-nearest fp16 of its exact value, each
