@@ -59,14 +59,29 @@ typedef enum {
  *  MOE_NL4_B32: 32 weights per block, fp16 scale d, 4-bit codes q into the
  *               int8 codebook {-127,-104,-83,-65,-49,-35,-22,-10,1,13,25,
  *               38,53,69,89,113}, w = d * cb[q].             (4.5 bpw)
+ *  MOE_NL3_256: 256-weight super-block, fp16 scale d, eight 4-bit
+ *               sub-scales s_j and eight codebook-shift bits e_j (one per
+ *               32 weights), 3-bit codes q into the non-uniform codebook
+ *               cb3 = {-15,-10,-6,-2,1,5,9,14}:
+ *               w = d * (2*s_j + 1) * (cb3[q] + e_j) / 16.   (3.22 bpw)
+ *               This library's own stand-in for the 3-bit non-linear
+ *               "K" type the model card lists for up/gate (IQ3_K,
+ *               3.44 bpw): the card gives only its name and bit rate, so
+ *               neither this layout nor this codebook follows that type.
  * Natural byte layout of a [rows x cols] tensor (rows of blocks along the
- * columns, planar): codes plane, then (SB3 only) sub-scale plane, then the
+ * columns, planar): codes plane, then (SB3, NL3) sub-scale plane, then the
  * fp16 d plane.  SB3 codes: 96 bytes per super-block, a little-endian bit
  * stream with code i at bit 3i; sub-scale j at bit 4j of a little-endian
- * 32-bit word.  Q4/NL4 codes: weight i of a row in byte i/2, low nibble for
- * even i.  The *packed* layout (same byte count) is the GPU tile layout
+ * 32-bit word.  NL3: the SB3 planes (codes, sub-scale words, d), then a
+ * plane of one byte per super-block whose bit j is e_j.  Q4/NL4 codes:
+ * weight i of a row in byte i/2, low nibble for even i.  The *packed* layout (same byte count) is the GPU tile layout
  * that moe_pack_tensor produces and every compute entry point reads. */
-typedef enum { MOE_Q4_B32 = 1, MOE_SB3_256 = 2, MOE_NL4_B32 = 3 } moe_qfmt;
+typedef enum {
+  MOE_Q4_B32 = 1,
+  MOE_SB3_256 = 2,
+  MOE_NL4_B32 = 3,
+  MOE_NL3_256 = 4
+} moe_qfmt;
 
 /* One MoE layer's experts as the FFN sees them.
  * Expert e's blob starts at pool + blob_index[e] * blob_stride and holds the
@@ -96,7 +111,8 @@ size_t moe_blob_bytes(int fmt_up_gate, int fmt_down, int H, int F);
 /* Natural layout -> packed GPU tile layout (model card, "Files": the expert
  * quant types; the packed layout is this library's own).  `natural` and
  * `packed` are distinct device buffers of moe_tensor_bytes() bytes.
- * Needs rows % 16 == 0, cols % 256 == 0 (SB3) or cols % 64 == 0 (Q4/NL4). */
+ * Needs rows % 16 == 0, cols % 256 == 0 (SB3, NL3) or cols % 64 == 0
+ * (Q4/NL4). */
 moe_status moe_pack_tensor(int fmt, const uint8_t* natural, int rows,
                            int cols, uint8_t* packed, void* stream);
 
@@ -286,7 +302,7 @@ moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream);
  *   expert_offsets/pair_ids/active/n_active: moe_group_tokens' outputs
  *   blob_index int32 [E] or NULL (NULL: expert e's blob is blob e); a
  *              negative entry of a chosen expert sets MOE_ERR_DEVICE
- * Needs H, F multiples of 256 (SB3) or 64 (Q4/NL4) and of 16.
+ * Needs H, F multiples of 256 (SB3, NL3) or 64 (Q4/NL4) and of 16.
  * T <= 8: int8 tensor-core decode kernels.  The weights enter exactly
  *   (int8 codes, integer sub-scale folds, fp32 scales); the activations
  *   are rounded to 15-bit fixed point with one power-of-two scale per

@@ -29,6 +29,10 @@ Readings of points the sources leave open are listed in the repository's
 design notes; the ones that shape arithmetic here are:
   * SB3 value: w = d * (2s+1) * c / 8 with c = 2q - 7 (q the 3-bit code).
   * NL4 value: w = d * cb[q] with the 16-entry int8 codebook below.
+  * NL3 value: w = d * (2s+1) * (cb3[q] + e) / 16 with the 8-entry codebook
+    below and one shift bit e per 32 weights (this repository's own 3-bit
+    non-uniform format; the model card lists such a type, IQ3_K, by name
+    and bit rate only).
   * Q4 value:  w = d * (q - 8).
   * Stacked decode layers use the pre-norm residual r <- r + MoE(x),
     x = bf16(rmsnorm(r)), rmsnorm without a learned weight, eps = 1e-6.
@@ -42,11 +46,15 @@ from typing import Callable, Dict, List, Optional, Sequence, Tuple
 
 import numpy as np
 
-Q4_B32, SB3_256, NL4_B32 = 1, 2, 3
+Q4_B32, SB3_256, NL4_B32, NL3_256 = 1, 2, 3, 4
 
 # 16-entry non-uniform codebook of the 4-bit NL format (ascending).
 NL4_CODEBOOK = np.array([-127, -104, -83, -65, -49, -35, -22, -10,
                          1, 13, 25, 38, 53, 69, 89, 113], dtype=np.float64)
+
+# 8-entry non-uniform codebook of the 3-bit NL format (ascending); each
+# 32-weight block may shift it up by one (its shift bit e).
+NL3_CODEBOOK = np.array([-15, -10, -6, -2, 1, 5, 9, 14], dtype=np.float64)
 
 RMS_EPS = 1e-6
 
@@ -86,6 +94,10 @@ def tensor_plane_sizes(fmt: int, rows: int, cols: int) -> List[int]:
         assert cols % 256 == 0
         n = rows * cols // 256
         return [96 * n, 4 * n, 2 * n]
+    if fmt == NL3_256:
+        assert cols % 256 == 0
+        n = rows * cols // 256
+        return [96 * n, 4 * n, 2 * n, n]
     assert fmt in (Q4_B32, NL4_B32) and cols % 32 == 0
     n = rows * cols // 32
     return [16 * n, 2 * n]
@@ -116,6 +128,36 @@ def dequant_sb3(raw: np.ndarray, rows: int, cols: int) -> np.ndarray:
     sub = np.repeat(2.0 * s.astype(np.float64) + 1.0, 32, axis=1)    # [nsb,256]
     c = 2.0 * q.astype(np.float64) - 7.0
     w = d[:, None] * sub * c / 8.0
+    return w.reshape(rows, cols)
+
+
+def dequant_nl3(raw: np.ndarray, rows: int, cols: int) -> np.ndarray:
+    """3-bit non-uniform-codebook super-block format -> float64 [rows, cols].
+
+    A super-block of 256 weights has a fp16 scale d, eight 4-bit sub-scales
+    s_j, eight shift bits e_j (one per 32 weights) and 256 3-bit codes q.
+    Weight i of the super-block (j = i // 32) is
+        w_i = d * (2*s_j + 1) * (cb3[q_i] + e_j) / 16,
+    cb3 = NL3_CODEBOOK.  Codes, sub-scales and d sit exactly as in the SB3
+    format; the shift bits are bit j of one byte per super-block.
+    """
+    n_codes, n_sc, n_d, n_ex = tensor_plane_sizes(NL3_256, rows, cols)
+    raw = np.asarray(raw, dtype=np.uint8)
+    codes = raw[:n_codes]
+    scales = raw[n_codes:n_codes + n_sc]
+    dbits = raw[n_codes + n_sc:n_codes + n_sc + n_d]
+    extra = raw[n_codes + n_sc + n_d:n_codes + n_sc + n_d + n_ex]
+    nsb = rows * cols // 256
+    bits = _bits_le(codes, 96).reshape(nsb, 256, 3)
+    q = (bits[:, :, 0] | (bits[:, :, 1] << 1) | (bits[:, :, 2] << 2))
+    sbits = _bits_le(scales, 4).reshape(nsb, 8, 4)
+    s = (sbits[:, :, 0] | (sbits[:, :, 1] << 1) | (sbits[:, :, 2] << 2) |
+         (sbits[:, :, 3] << 3))                                      # [nsb,8]
+    e = _bits_le(extra, 1).reshape(nsb, 8).astype(np.float64)        # [nsb,8]
+    d = fp16_to_f64(dbits)                                           # [nsb]
+    sub = np.repeat(2.0 * s.astype(np.float64) + 1.0, 32, axis=1)    # [nsb,256]
+    v = NL3_CODEBOOK[q] + np.repeat(e, 32, axis=1)
+    w = d[:, None] * sub * v / 16.0
     return w.reshape(rows, cols)
 
 
@@ -151,6 +193,8 @@ def dequant_b32(fmt: int, raw: np.ndarray, rows: int, cols: int) -> np.ndarray:
 def dequant(fmt: int, raw: np.ndarray, rows: int, cols: int) -> np.ndarray:
     if fmt == SB3_256:
         return dequant_sb3(raw, rows, cols)
+    if fmt == NL3_256:
+        return dequant_nl3(raw, rows, cols)
     return dequant_b32(fmt, raw, rows, cols)
 
 

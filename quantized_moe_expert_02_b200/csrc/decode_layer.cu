@@ -242,8 +242,11 @@ __global__ void __launch_bounds__(LAYER_THREADS, 1)
   constexpr int NT = NTT;            // N tiles of 4 tokens: T <= 4 * NT
   constexpr int TM = 4 * NTT;
   const int G = gridDim.x;
-  constexpr int TCU = FUG == MOE_SB3_256 ? SB3_TILE_COLS : B32_TILE_COLS;
-  constexpr int TBU = FUG == MOE_SB3_256 ? SB3_TILE_BYTES : B32_TILE_BYTES;
+  constexpr bool SBU = FUG == MOE_SB3_256 || FUG == MOE_NL3_256;
+  constexpr int TCU = SBU ? SB3_TILE_COLS : B32_TILE_COLS;
+  constexpr int TBU = FUG == MOE_SB3_256   ? SB3_TILE_BYTES
+                      : FUG == MOE_NL3_256 ? NL3_TILE_BYTES
+                                           : B32_TILE_BYTES;
   const int nk = H / TCU;                      // up tiles per row tile
   const int nkd = F / B32_TILE_COLS;           // down tiles per row tile
 
@@ -397,7 +400,7 @@ __global__ void __launch_bounds__(LAYER_THREADS, 1)
           const int sg = pow2_sigma(m);
           xsig[b * DEC_TMAX + t] = sg;
           xsc[b * DEC_TMAX + t] =
-              exp2i(-sg) * (FUG == MOE_SB3_256 ? 0.125f : 1.0f);
+              exp2i(-sg) * fmt_xfold(FUG);
         }
       }
       named_bar_sync(BAR_XF, xn);
@@ -745,10 +748,10 @@ __global__ void __launch_bounds__(LAYER_THREADS, 1)
         const uint8_t* tp = unit + pc * TBU;
         const uint32_t* xf = frag + kt * (TCU / 32) * NT * 64;
         const float* xb = xsc + (kt * TCU / XB_COLS) * DEC_TMAX;
-        if (FUG == MOE_SB3_256) {
+        if (SBU) {
           const float xs2[2] = {xb[c], xb[4 + c]};
-          if (tz == 0) piece_sb3(tp, xf, NT, xs2, au, lane, NT);
-          else piece_sb3(tp, xf, NT, xs2, ag, lane, NT);
+          if (tz == 0) piece_sbx<FUG == MOE_NL3_256>(tp, xf, NT, xs2, au, lane, NT);
+          else piece_sbx<FUG == MOE_NL3_256>(tp, xf, NT, xs2, ag, lane, NT);
         } else {
           if (tz == 0) piece_b32<FUG>(tp, xf, NT, xb + c, 0, au, lane, NT);
           else piece_b32<FUG>(tp, xf, NT, xb + c, 0, ag, lane, NT);
@@ -981,6 +984,7 @@ moe_status launch_decode_layer(const moe_layer_desc& d, const uint16_t* x,
                     : MOE_PICK2(FU, MOE_NL4_B32, 1))
   switch (d.fmt_up_gate) {
     case MOE_SB3_256: MOE_PICK(MOE_SB3_256); break;
+    case MOE_NL3_256: MOE_PICK(MOE_NL3_256); break;
     case MOE_NL4_B32: MOE_PICK(MOE_NL4_B32); break;
     default: MOE_PICK(MOE_Q4_B32);
   }

@@ -12,11 +12,17 @@ namespace moe {
 // SB3 tile (16 x 256): acc[nt][0/1] += rows g / g+8 for column token
 // (lane&3) + 4nt.  xfb = B fragments of the tile's first 32-block,
 // [blk][bnt][32][2] words; xs[nt] = 2^-sigma_t / 8 of the lane's token.
-__device__ __forceinline__ void piece_sb3(const uint8_t* tp,
+// NL3 tile (same planes plus a shift byte per row): the byte table is the
+// codebook cb3, each row's bytes raised by its block's shift bit e_j, and
+// xs[nt] = 2^-sigma_t / 16.
+template <bool NL3>
+__device__ __forceinline__ void piece_sbx(const uint8_t* tp,
                                           const uint32_t* xfb, int NT,
                                           const float (&xs)[2],
                                           float (&acc)[2][2], int lane,
-                                          int bnt = BF_NT) {
+                                          int bnt) {
+  constexpr uint32_t T0 = NL3 ? NL3_TAB0 : SB3_TAB0;
+  constexpr uint32_t T1 = NL3 ? NL3_TAB1 : SB3_TAB1;
   const int g = lane >> 2;
   const uint4 L0 = *reinterpret_cast<const uint4*>(tp + 16 * lane);
   const uint4 L1 = *reinterpret_cast<const uint4*>(tp + 512 + 16 * lane);
@@ -25,6 +31,10 @@ __device__ __forceinline__ void piece_sb3(const uint8_t* tp,
   const uint32_t DD = *reinterpret_cast<const uint32_t*>(tp + 1600 + 4 * g);
   const uint32_t lo[8] = {L0.x, L0.y, L0.z, L0.w, L1.x, L1.y, L1.z, L1.w};
   const uint32_t hi[4] = {HV.x, HV.y, HV.z, HV.w};
+  // NL3: shift bits of rows g (pi = 2g) and g+8 (pi = 2g + 1)
+  const uint32_t EX =
+      NL3 ? *reinterpret_cast<const uint16_t*>(tp + SB3_TILE_BYTES + 2 * g)
+          : 0u;
   int32_t S[2][2] = {{0, 0}, {0, 0}};
   const int32_t zero[4] = {0, 0, 0, 0};
   // (2s+1) of the eight 32-blocks as bytes: even blocks, odd blocks
@@ -40,10 +50,18 @@ __device__ __forceinline__ void piece_sb3(const uint8_t* tp,
     const uint32_t sa = (LO & 0x33333333u) | (ha & 0x44444444u);
     const uint32_t sb = ((LO >> 2) & 0x33333333u) | (hb & 0x44444444u);
     uint32_t a[4];
-    a[0] = prmt(SB3_TAB0, SB3_TAB1, sa);
-    a[1] = prmt(SB3_TAB0, SB3_TAB1, sa >> 16);
-    a[2] = prmt(SB3_TAB0, SB3_TAB1, sb);
-    a[3] = prmt(SB3_TAB0, SB3_TAB1, sb >> 16);
+    a[0] = prmt(T0, T1, sa);          // row g,   k 4c..4c+3
+    a[1] = prmt(T0, T1, sa >> 16);    // row g+8
+    a[2] = prmt(T0, T1, sb);          // row g,   k 16+4c..
+    a[3] = prmt(T0, T1, sb >> 16);    // row g+8
+    if (NL3) {
+      const uint32_t inc = ((EX >> j) & 1u) * 0x01010101u;
+      const uint32_t inc8 = ((EX >> (8 + j)) & 1u) * 0x01010101u;
+      a[0] += inc;
+      a[2] += inc;
+      a[1] += inc8;
+      a[3] += inc8;
+    }
     // byte j/2 of the even/odd word, zero-extended (prmt selector 0x444m)
     const uint32_t bsel = 0x4440u | (uint32_t)(j >> 1);
     const int mg = (int)prmt((j & 1) ? mgo : mge, 0u, bsel);
@@ -68,6 +86,26 @@ __device__ __forceinline__ void piece_sb3(const uint8_t* tp,
       acc[nt][1] = fmaf((float)S[nt][1], dv.y * xs[nt], acc[nt][1]);
     }
   }
+}
+
+__device__ __forceinline__ void piece_sb3(const uint8_t* tp,
+                                          const uint32_t* xfb, int NT,
+                                          const float (&xs)[2],
+                                          float (&acc)[2][2], int lane,
+                                          int bnt = BF_NT) {
+  piece_sbx<false>(tp, xfb, NT, xs, acc, lane, bnt);
+}
+__device__ __forceinline__ void piece_nl3(const uint8_t* tp,
+                                          const uint32_t* xfb, int NT,
+                                          const float (&xs)[2],
+                                          float (&acc)[2][2], int lane,
+                                          int bnt = BF_NT) {
+  piece_sbx<true>(tp, xfb, NT, xs, acc, lane, bnt);
+}
+// Scale that folds the fixed denominator of a super-block format's value
+// into the activation scale: 1/8 (SB3), 1/16 (NL3), 1 (the 4-bit formats).
+__host__ __device__ constexpr float fmt_xfold(int fmt) {
+  return fmt == MOE_SB3_256 ? 0.125f : fmt == MOE_NL3_256 ? 0.0625f : 1.0f;
 }
 
 // Q4 / NL4 tile (16 x 64, two 32-blocks).  cs = column scales of the

@@ -72,8 +72,11 @@ template <int FMT>
 __global__ void __launch_bounds__(DEC_THREADS, 1)
     ffn_up_decode_kernel(DecParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
-  constexpr int TB = FMT == MOE_SB3_256 ? SB3_TILE_BYTES : B32_TILE_BYTES;
-  constexpr int TC = FMT == MOE_SB3_256 ? SB3_TILE_COLS : B32_TILE_COLS;
+  constexpr bool SBF = FMT == MOE_SB3_256 || FMT == MOE_NL3_256;
+  constexpr int TB = FMT == MOE_SB3_256   ? SB3_TILE_BYTES
+                     : FMT == MOE_NL3_256 ? NL3_TILE_BYTES
+                                          : B32_TILE_BYTES;
+  constexpr int TC = SBF ? SB3_TILE_COLS : B32_TILE_COLS;
   const int nk = p.H / TC;
   const int nsplit = nk < NSPLIT_MAX ? nk : NSPLIT_MAX;
   const int kmax = (nk + nsplit - 1) / nsplit;
@@ -118,7 +121,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 1)
       const int s = pow2_sigma(m);
       xsig[b * DEC_TMAX + t] = s;
       xsc[b * DEC_TMAX + t] =
-          exp2i(-s) * (FMT == MOE_SB3_256 ? 0.125f : 1.0f);
+          exp2i(-s) * fmt_xfold(FMT);
     }
   }
   __syncthreads();
@@ -194,9 +197,11 @@ __global__ void __launch_bounds__(DEC_THREADS, 1)
     for (int kt = 0; kt < k1 - k0; ++kt) {
       const int blk0 = (k0 + kt) * (TC / 32);
       const float* xb = xsc + ((k0 + kt) * TC / XB_COLS) * DEC_TMAX;
-      if (FMT == MOE_SB3_256) {
+      if (SBF) {
         const float xs[2] = {xb[c], xb[4 + c]};
-        piece_sb3(chunk + kt * TB, xf + blk0 * BF_NT * 64, NT, xs, acc, lane);
+        piece_sbx<FMT == MOE_NL3_256>(chunk + kt * TB,
+                                      xf + blk0 * BF_NT * 64, NT, xs, acc,
+                                      lane, BF_NT);
       } else {
         piece_b32<FMT>(chunk + kt * TB, xf + blk0 * BF_NT * 64, NT, xb + c,
                        0, acc, lane);
@@ -526,6 +531,9 @@ moe_status launch_up_decode(const moe_layer_desc& d, const uint16_t* x,
                         prm);
     case MOE_NL4_B32:
       return launch_pdl(ffn_up_decode_kernel<MOE_NL4_B32>, grid, su, s, pdl,
+                        prm);
+    case MOE_NL3_256:
+      return launch_pdl(ffn_up_decode_kernel<MOE_NL3_256>, grid, su, s, pdl,
                         prm);
     default:
       return launch_pdl(ffn_up_decode_kernel<MOE_Q4_B32>, grid, su, s, pdl,

@@ -37,20 +37,35 @@ namespace moe {
 //              nibble n of W[2b+h] = code of row g + 8*(n>>2), column
 //              32b + 16h + 4c + (n&3)
 //   [512,576)  fp16 d: row r, block b at 2*(4*(r%8) + 2*(r/8) + b)
+//
+// NL3 tile (MOE_NL3_256) = the SB3 tile (codes, sub-scales, d at the same
+// offsets) followed by
+//   [1632,1648)  codebook-shift bytes, row r at 1632 + pi(r) (bit j = e_j
+//                of 32-block j)
+// 1648 bytes.
 constexpr int SB3_TILE_BYTES = 1632;
 constexpr int SB3_TILE_COLS = 256;
+constexpr int NL3_TILE_BYTES = 1648;
 constexpr int B32_TILE_BYTES = 576;
 constexpr int B32_TILE_COLS = 64;
 constexpr int TILE_ROWS = 16;
 
+// The super-block formats (256 columns per tile, 3-bit codes in LO/HI
+// planes): SB3 and NL3.
+__host__ __device__ inline bool fmt_sb(int fmt) {
+  return fmt == MOE_SB3_256 || fmt == MOE_NL3_256;
+}
 __host__ __device__ inline int tile_bytes(int fmt) {
-  return fmt == MOE_SB3_256 ? SB3_TILE_BYTES : B32_TILE_BYTES;
+  return fmt == MOE_SB3_256   ? SB3_TILE_BYTES
+         : fmt == MOE_NL3_256 ? NL3_TILE_BYTES
+                              : B32_TILE_BYTES;
 }
 __host__ __device__ inline int tile_cols(int fmt) {
-  return fmt == MOE_SB3_256 ? SB3_TILE_COLS : B32_TILE_COLS;
+  return fmt_sb(fmt) ? SB3_TILE_COLS : B32_TILE_COLS;
 }
 inline bool fmt_valid(int fmt) {
-  return fmt == MOE_Q4_B32 || fmt == MOE_SB3_256 || fmt == MOE_NL4_B32;
+  return fmt == MOE_Q4_B32 || fmt == MOE_SB3_256 || fmt == MOE_NL4_B32 ||
+         fmt == MOE_NL3_256;
 }
 // Shape accepted by the packed layout.
 inline bool packed_shape_ok(int fmt, int rows, int cols) {
@@ -74,6 +89,11 @@ constexpr uint32_t NL4_TA0 = 0xBFAD9881u;   // -127,-104,-83,-65
 constexpr uint32_t NL4_TA1 = 0xF6EADDCFu;   //  -49, -35,-22,-10
 constexpr uint32_t NL4_TB0 = 0x271A0E02u;   //    2,  14, 26, 39
 constexpr uint32_t NL4_TB1 = 0x725A4636u;   //   54,  70, 90,114
+// NL3: the 3-bit codebook {-15,-10,-6,-2,1,5,9,14} as int8 bytes, q = 0..3
+// and 4..7; a set shift bit e adds 1 to every byte (no byte is -1, so the
+// 32-bit add never carries across bytes).
+constexpr uint32_t NL3_TAB0 = 0xFEFAF6F1u;  // -15,-10, -6, -2
+constexpr uint32_t NL3_TAB1 = 0x0E090501u;  //   1,  5,  9, 14
 // Q4: q - 8 in the same split.
 constexpr uint32_t Q4_TA0 = 0xFBFAF9F8u;    // -8..-5
 constexpr uint32_t Q4_TA1 = 0xFFFEFDFCu;    // -4..-1
@@ -343,7 +363,7 @@ __device__ inline float dq_packed(int fmt, const uint8_t* t, int cols,
       t + ((int64_t)(row / TILE_ROWS) * ntc + col / tc) * tile_bytes(fmt);
   const int r = row % TILE_ROWS, g = r % 8, half = r / 8;
   const int pi = 2 * g + half;
-  if (fmt == MOE_SB3_256) {
+  if (fmt_sb(fmt)) {
     const int kk = col % 256, j = kk / 32, k32 = kk % 32;
     const int hsel = k32 / 16, c = (k32 % 16) / 4, w = k32 % 4;
     const int lane = 4 * g + c;
@@ -359,6 +379,11 @@ __device__ inline float dq_packed(int fmt, const uint8_t* t, int cols,
     const int s = (sw >> (4 * j)) & 15;
     const float d =
         __half2float(*(const __half*)(tile + 1600 + 2 * pi));
+    if (fmt == MOE_NL3_256) {
+      const int8_t cb[8] = {-15, -10, -6, -2, 1, 5, 9, 14};
+      const int e = (tile[1632 + pi] >> j) & 1;
+      return d * (float)((2 * s + 1) * (cb[q] + e)) * 0.0625f;
+    }
     return d * (float)(2 * s + 1) * (float)(2 * q - 7) * 0.125f;
   } else {
     const int kk = col % 64, b = kk / 32, k32 = kk % 32;

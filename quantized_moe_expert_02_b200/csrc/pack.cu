@@ -1,7 +1,8 @@
 // Natural -> packed tile layout, and the dequantisation export.
 // Formats: the expert quant types of the Avalon GGUF model card ("Files"):
 // the 3.25-bpw super-block variant (one scale per 256 weights, 4-bit
-// sub-scales per 32) and the 4-bit non-uniform-codebook type.
+// sub-scales per 32), the 4-bit non-uniform-codebook type, and this
+// library's 3-bit non-uniform-codebook super-block (NL3).
 #include "moe_internal.cuh"
 
 namespace moe {
@@ -24,20 +25,24 @@ __device__ inline int nat_b32_code(const uint8_t* codes, int cols, int row,
   return (i & 1) ? (b >> 4) : (b & 15);
 }
 
-// One thread per 32-bit word of the packed tensor.
+// One thread per 32-bit word of the packed tensor.  SB3 and NL3 (the NL3
+// tile appends the codebook-shift bytes of its 16 rows).
+template <bool NL3>
 __global__ void pack_sb3_kernel(const uint8_t* __restrict__ nat, int rows,
                                 int cols, uint32_t* __restrict__ out) {
+  constexpr int TBW = (NL3 ? NL3_TILE_BYTES : SB3_TILE_BYTES) / 4;
   const int ntc = cols / 256;
   const int64_t ntiles = (int64_t)(rows / 16) * ntc;
-  const int64_t nwords = ntiles * (SB3_TILE_BYTES / 4);
+  const int64_t nwords = ntiles * TBW;
   const int64_t nsb = (int64_t)rows * ntc;
   const uint8_t* codes = nat;
   const uint32_t* scales = (const uint32_t*)(nat + nsb * 96);
   const uint16_t* dplane = (const uint16_t*)(nat + nsb * 100);
+  const uint8_t* extra = nat + nsb * 102;   // NL3 only
   for (int64_t wi = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
        wi < nwords; wi += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t tile = wi / (SB3_TILE_BYTES / 4);
-    const int w = (int)(wi % (SB3_TILE_BYTES / 4));
+    const int64_t tile = wi / TBW;
+    const int w = (int)(wi % TBW);
     const int rt = (int)(tile / ntc), kb = (int)(tile % ntc);
     uint32_t word = 0;
     if (w < 384) {
@@ -70,7 +75,7 @@ __global__ void pack_sb3_kernel(const uint8_t* __restrict__ nat, int rows,
       const int pi = w - 384;
       const int r = pi / 2 + 8 * (pi % 2);
       word = scales[(int64_t)(16 * rt + r) * ntc + kb];
-    } else {  // d: two fp16 per word
+    } else if (w < 408) {  // d: two fp16 per word
       const int p0 = 2 * (w - 400);
       uint32_t lohi[2];
       for (int h = 0; h < 2; ++h) {
@@ -79,6 +84,12 @@ __global__ void pack_sb3_kernel(const uint8_t* __restrict__ nat, int rows,
         lohi[h] = dplane[(int64_t)(16 * rt + r) * ntc + kb];
       }
       word = lohi[0] | (lohi[1] << 16);
+    } else {  // NL3 codebook-shift bytes: four per word
+      for (int h = 0; h < 4; ++h) {
+        const int pi = 4 * (w - 408) + h;
+        const int r = pi / 2 + 8 * (pi % 2);
+        word |= (uint32_t)extra[(int64_t)(16 * rt + r) * ntc + kb] << (8 * h);
+      }
     }
     out[wi] = word;
   }
@@ -165,8 +176,11 @@ extern "C" moe_status moe_pack_tensor(int fmt, const uint8_t* natural,
   cudaStream_t s = (cudaStream_t)stream;
   const int64_t words = tensor_bytes_of(fmt, rows, cols) / 4;
   if (fmt == MOE_SB3_256)
-    pack_sb3_kernel<<<grid_for(words, 256), 256, 0, s>>>(natural, rows, cols,
-                                                         (uint32_t*)packed);
+    pack_sb3_kernel<false><<<grid_for(words, 256), 256, 0, s>>>(
+        natural, rows, cols, (uint32_t*)packed);
+  else if (fmt == MOE_NL3_256)
+    pack_sb3_kernel<true><<<grid_for(words, 256), 256, 0, s>>>(
+        natural, rows, cols, (uint32_t*)packed);
   else
     pack_b32_kernel<<<grid_for(words, 256), 256, 0, s>>>(natural, rows, cols,
                                                          (uint32_t*)packed);

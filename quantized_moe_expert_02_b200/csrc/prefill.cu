@@ -40,6 +40,17 @@ constexpr int PF_NDQ = 8;    // dequant warps
 constexpr int PF_A_BYTES = PF_BM * PF_BK * 2;         // 16 KB
 constexpr int PF_B_BYTES = PF_BN * PF_BK * 2;         // 32 KB
 constexpr int PF_TMEM_COLS = 512;
+// A operand formats of the GEMM kernels: the 4-bit 32-weight blocks (Q4,
+// NL4), and the 3-bit super-blocks SB3 and NL3.
+constexpr int AF_B32 = 0, AF_SB3 = 1, AF_NL3 = 2;
+__host__ __device__ constexpr int af_of(int fmt) {
+  return fmt == MOE_SB3_256 ? AF_SB3 : fmt == MOE_NL3_256 ? AF_NL3 : AF_B32;
+}
+__host__ __device__ constexpr int af_tile_bytes(int af) {
+  return af == AF_SB3 ? SB3_TILE_BYTES
+         : af == AF_NL3 ? NL3_TILE_BYTES
+                        : B32_TILE_BYTES;
+}
 
 template <bool UP>
 struct PfCfg {
@@ -137,6 +148,7 @@ struct Sb3Half {
   uint2 hi[2];      // [lane]: HI[gamma], HI[gamma+2]
   uint2 sc;         // sub-scale words of rows g, g+8
   uint32_t d;       // fp16 d of rows g (low), g+8 (high)
+  uint32_t ex;      // NL3: shift bytes of rows g (bits 0-7), g+8 (8-15)
 };
 
 __device__ __forceinline__ void sb3_load(const uint8_t* tp, int g, int p,
@@ -152,6 +164,11 @@ __device__ __forceinline__ void sb3_load(const uint8_t* tp, int g, int p,
   }
   q.sc = ldg_u64(tp + 1536 + 8 * g);
   q.d = ldg_u32(tp + 1600 + 4 * g);
+}
+__device__ __forceinline__ void nl3_load(const uint8_t* tp, int g, int p,
+                                         int gamma, Sb3Half& q) {
+  sb3_load(tp, g, p, gamma, q);
+  q.ex = __ldg(reinterpret_cast<const uint16_t*>(tp + SB3_TILE_BYTES + 2 * g));
 }
 
 // 8 codes of one lane word (nibble n = 4*rowhalf + w) -> fp16 c values as
@@ -214,6 +231,89 @@ __device__ __forceinline__ void sb3_store(const Sb3Half& sb, int g, int p,
                    w[0][h][3], w[1][h][2], w[1][h][3]);
     }
   }
+}
+
+// ------------------------------------------------------------- NL3 ----
+// cb3[q] + 16 as unsigned bytes (1..30), q = 0..3 and 4..7
+constexpr uint32_t NL3_U0 = 0x0E0A0601u;
+constexpr uint32_t NL3_U1 = 0x1E191511u;
+constexpr uint32_t H16_1040 = 0x64106410u;   // fp16 1040 = 1024 + 16, twice
+
+// 8 codes of one lane word (as sb3_codes_to_h16) -> fp16 cb3[q] + e, with
+// inc / inc8 the byte-replicated shift bits of rows g and g+8: the bytes
+// u = cb3[q] + 16 + e go under a 0x64 high byte (fp16 1024 + u, exact),
+// minus fp16 1040.
+__device__ __forceinline__ void nl3_codes_to_h16(uint32_t Q, uint32_t inc,
+                                                 uint32_t inc8,
+                                                 uint32_t (&o)[4]) {
+  const uint32_t P0 = prmt(NL3_U0, NL3_U1, Q) + inc;          // row g
+  const uint32_t P1 = prmt(NL3_U0, NL3_U1, Q >> 16) + inc8;   // row g+8
+  o[0] = hsub2u(prmt(P0, 0x64646464u, 0x5140u), H16_1040);
+  o[1] = hsub2u(prmt(P0, 0x64646464u, 0x7362u), H16_1040);
+  o[2] = hsub2u(prmt(P1, 0x64646464u, 0x5140u), H16_1040);
+  o[3] = hsub2u(prmt(P1, 0x64646464u, 0x7362u), H16_1040);
+}
+
+// The NL3 counterpart of sb3_store: value (cb3[q] + e_j) * (2s+1)/16 (exact
+// in fp16) times d, one rounding.
+__device__ __forceinline__ void nl3_store(const Sb3Half& sb, int g, int p,
+                                          int gamma, int qh, int row0,
+                                          uint32_t a_smem) {
+  const int q = gamma + 2 * qh;
+  const int j0 = 2 * q;
+  const uint32_t dg = half_bcast((uint16_t)(sb.d & 0xFFFFu));
+  const uint32_t dg8 = half_bcast((uint16_t)(sb.d >> 16));
+#pragma unroll
+  for (int jj = 0; jj < 2; ++jj) {
+    const int j = j0 + jj;
+    const int sg = (sb.sc.x >> (4 * j)) & 15, sg8 = (sb.sc.y >> (4 * j)) & 15;
+    const __half tg = __float2half_rn((float)(2 * sg + 1) * 0.0625f);
+    const __half tg8 = __float2half_rn((float)(2 * sg8 + 1) * 0.0625f);
+    const uint32_t t2g = half_bcast(__half_as_ushort(tg));
+    const uint32_t t2g8 = half_bcast(__half_as_ushort(tg8));
+    const uint32_t inc = ((sb.ex >> j) & 1u) * 0x01010101u;
+    const uint32_t inc8 = ((sb.ex >> (8 + j)) & 1u) * 0x01010101u;
+    uint32_t w[2][2][4];   // [lane][h][words]
+#pragma unroll
+    for (int l = 0; l < 2; ++l) {
+      const uint32_t lo = jj ? sb.lo[qh][l].y : sb.lo[qh][l].x;
+      const uint32_t hi = (qh ? sb.hi[l].y : sb.hi[l].x) >> (2 * jj);
+      const uint32_t Q0 = (lo & 0x33333333u) | ((hi << 2) & 0x44444444u);
+      const uint32_t Q1 = ((lo >> 2) & 0x33333333u) | ((hi << 1) & 0x44444444u);
+      nl3_codes_to_h16(Q0, inc, inc8, w[l][0]);
+      nl3_codes_to_h16(Q1, inc, inc8, w[l][1]);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        w[l][h][0] = hmul2u(hmul2u(w[l][h][0], t2g), dg);
+        w[l][h][1] = hmul2u(hmul2u(w[l][h][1], t2g), dg);
+        w[l][h][2] = hmul2u(hmul2u(w[l][h][2], t2g8), dg8);
+        w[l][h][3] = hmul2u(hmul2u(w[l][h][3], t2g8), dg8);
+      }
+    }
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int chunk = 4 * jj + 2 * h + p;
+      st_shared_v4(a_smem + sw128(row0 + g, chunk), w[0][h][0], w[0][h][1],
+                   w[1][h][0], w[1][h][1]);
+      st_shared_v4(a_smem + sw128(row0 + g + 8, chunk), w[0][h][2],
+                   w[0][h][3], w[1][h][2], w[1][h][3]);
+    }
+  }
+}
+
+// Super-block format of a GEMM's A operand: SB3 or NL3 load / store.
+template <int AF>
+__device__ __forceinline__ void sbx_load(const uint8_t* tp, int g, int p,
+                                         int gamma, Sb3Half& q) {
+  if constexpr (AF == AF_NL3) nl3_load(tp, g, p, gamma, q);
+  else sb3_load(tp, g, p, gamma, q);
+}
+template <int AF>
+__device__ __forceinline__ void sbx_store(const Sb3Half& sb, int g, int p,
+                                          int gamma, int qh, int row0,
+                                          uint32_t a_smem) {
+  if constexpr (AF == AF_NL3) nl3_store(sb, g, p, gamma, qh, row0, a_smem);
+  else sb3_store(sb, g, p, gamma, qh, row0, a_smem);
 }
 
 // ------------------------------------------------------------- B32 ----
@@ -282,10 +382,11 @@ __device__ __forceinline__ void b32_store(const B32Q& q, int g, int p,
 // super-block (group gamma writes k-steps gamma and gamma + 2); Q4/NL4: two
 // k-steps, one per group -- then un-swizzled to fp16 [rows][cols].  Used
 // only by moe_dequant_path, to check these decoders bit for bit.
-template <bool SB3>
+template <int AF>
 __global__ void __launch_bounds__(256)
     pf_dequant_export_kernel(const uint8_t* __restrict__ t, int cols,
                              uint4 tab4, uint16_t* __restrict__ out) {
+  constexpr bool SB3 = AF != AF_B32;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
@@ -295,17 +396,17 @@ __global__ void __launch_bounds__(256)
   const int tg = tt & 7, tp_ = (tt >> 3) & 1, tti = tt >> 4;
   const int m = blockIdx.x, kg = blockIdx.y;
   const int tcols = SB3 ? SB3_TILE_COLS : B32_TILE_COLS;
-  const int tbytes = SB3 ? SB3_TILE_BYTES : B32_TILE_BYTES;
+  const int tbytes = af_tile_bytes(AF);
   const int64_t trow_stride = (int64_t)(cols / tcols) * tbytes;
   const uint8_t* ptp = t + (int64_t)(m * (PF_BM / 16) + tti) * trow_stride;
   const int nks_total = cols / PF_BK;
   if constexpr (SB3) {
     Sb3Half q;
-    sb3_load(ptp + (int64_t)kg * SB3_TILE_BYTES, tg, tp_, gamma, q);
+    sbx_load<AF>(ptp + (int64_t)kg * tbytes, tg, tp_, gamma, q);
 #pragma unroll
     for (int qh = 0; qh < 2; ++qh)
-      sb3_store(q, tg, tp_, gamma, qh, 16 * tti,
-                sbase + (uint32_t)((gamma + 2 * qh) * PF_A_BYTES));
+      sbx_store<AF>(q, tg, tp_, gamma, qh, 16 * tti,
+                    sbase + (uint32_t)((gamma + 2 * qh) * PF_A_BYTES));
   } else {
     const B32Tab tab = {tab4.x, tab4.y, tab4.z, tab4.w};
     const int ks = NKS * kg + gamma;
@@ -333,9 +434,10 @@ __global__ void __launch_bounds__(256)
 // --------------------------------------------------------------- kernel --
 // maps: up: x_g [P][H], down: h16 [P][F], both fp16 in grouped row
 // order, boxes of 64 columns, 128-byte swizzle.
-template <bool UP, bool SB3>
+template <bool UP, int AF>
 __global__ void __launch_bounds__(PfCfg<UP>::THREADS, 1)
     pf_gemm_kernel(const PfParams p, const __grid_constant__ PfMaps maps) {
+  constexpr bool SB3 = AF != AF_B32;   // a super-block format (SB3, NL3)
   using C = PfCfg<UP>;
   constexpr int NA = C::NA, S = C::STAGES;
   extern __shared__ uint8_t smem_raw[];
@@ -471,7 +573,7 @@ __global__ void __launch_bounds__(PfCfg<UP>::THREADS, 1)
     const int t = threadIdx.x - (C::WDQ0 + 4 * gamma) * 32;   // 0..127
     const int tg = t & 7, tp_ = (t >> 3) & 1, tti = t >> 4;
     const int tcols = SB3 ? SB3_TILE_COLS : B32_TILE_COLS;
-    const int tbytes = SB3 ? SB3_TILE_BYTES : B32_TILE_BYTES;
+    const int tbytes = af_tile_bytes(AF);
     const int64_t trow_stride = (int64_t)(p.K / tcols) * tbytes;  // 16 rows
     const B32Tab tab = {p.tab[0], p.tab[1], p.tab[2], p.tab[3]};
     // tile pointers of the prefetch position's unit
@@ -522,7 +624,7 @@ __global__ void __launch_bounds__(PfCfg<UP>::THREADS, 1)
         if (it != pf_it) set_unit(it);
 #pragma unroll
         for (int a = 0; a < NA; ++a)
-          sb3_load(ptp[a] + (int64_t)sb * SB3_TILE_BYTES, tg, tp_, gamma, q[a]);
+          sbx_load<AF>(ptp[a] + (int64_t)sb * tbytes, tg, tp_, gamma, q[a]);
         ++pf_sb;
       };
       Sb3Half cur[NA], nxt[NA];
@@ -539,8 +641,8 @@ __global__ void __launch_bounds__(PfCfg<UP>::THREADS, 1)
           }
 #pragma unroll
           for (int a = 0; a < NA; ++a)
-            sb3_store(cur[a], tg, tp_, gamma, qh, 16 * tti,
-                      st + a * PF_A_BYTES);
+            sbx_store<AF>(cur[a], tg, tp_, gamma, qh, 16 * tti,
+                          st + a * PF_A_BYTES);
           stage_end(ksg);
         }
 #pragma unroll
@@ -816,28 +918,34 @@ static void pf_tables(int fmt, uint32_t (&t)[4]) {
 
 bool pf_export_supported(int fmt, int rows, int cols) {
   return rows > 0 && cols > 0 && rows % PF_BM == 0 &&
-         cols % (fmt == MOE_SB3_256 ? SB3_TILE_COLS : B32_TILE_COLS) == 0;
+         cols % tile_cols(fmt) == 0;
 }
 
 moe_status launch_pf_dequant_export(int fmt, const uint8_t* t, int rows,
                                     int cols, uint16_t* out, cudaStream_t s) {
   uint32_t tb[4] = {0u, 0u, 0u, 0u};
-  if (fmt != MOE_SB3_256) pf_tables(fmt, tb);
+  if (!fmt_sb(fmt)) pf_tables(fmt, tb);
   const uint4 tab4 = make_uint4(tb[0], tb[1], tb[2], tb[3]);
-  const bool sb3 = fmt == MOE_SB3_256;
+  const bool sb3 = fmt_sb(fmt);
   const int nks = sb3 ? 4 : 2;
   const size_t smem = (size_t)nks * PF_A_BYTES + 1024;
-  const void* fn = sb3 ? (const void*)&pf_dequant_export_kernel<true>
-                       : (const void*)&pf_dequant_export_kernel<false>;
+  const int af = af_of(fmt);
+  const void* fn = af == AF_SB3   ? (const void*)&pf_dequant_export_kernel<AF_SB3>
+                   : af == AF_NL3 ? (const void*)&pf_dequant_export_kernel<AF_NL3>
+                                  : (const void*)&pf_dequant_export_kernel<AF_B32>;
   moe_status st = ensure_smem(fn, smem);
   if (st != MOE_OK) return st;
   const dim3 grid(rows / PF_BM, sb3 ? cols / SB3_TILE_COLS
                                     : (cols / PF_BK + 1) / 2);
-  if (sb3)
-    pf_dequant_export_kernel<true><<<grid, 256, smem, s>>>(t, cols, tab4, out);
+  if (af == AF_SB3)
+    pf_dequant_export_kernel<AF_SB3><<<grid, 256, smem, s>>>(t, cols, tab4,
+                                                             out);
+  else if (af == AF_NL3)
+    pf_dequant_export_kernel<AF_NL3><<<grid, 256, smem, s>>>(t, cols, tab4,
+                                                             out);
   else
-    pf_dequant_export_kernel<false><<<grid, 256, smem, s>>>(t, cols, tab4,
-                                                            out);
+    pf_dequant_export_kernel<AF_B32><<<grid, 256, smem, s>>>(t, cols, tab4,
+                                                             out);
   return launch_status();
 }
 
@@ -882,15 +990,24 @@ static moe_status encode_maps(PfMaps* maps, const void* base, uint64_t inner,
   return MOE_OK;
 }
 
-template <bool UP, bool SB3>
+template <bool UP, int AF>
 static moe_status pf_launch(const PfParams& prm, const PfMaps& map,
                             cudaStream_t s) {
-  const void* fn = reinterpret_cast<const void*>(&pf_gemm_kernel<UP, SB3>);
+  const void* fn = reinterpret_cast<const void*>(&pf_gemm_kernel<UP, AF>);
   moe_status st = ensure_smem(fn, PfCfg<UP>::SMEM);
   if (st != MOE_OK) return st;
-  pf_gemm_kernel<UP, SB3>
+  pf_gemm_kernel<UP, AF>
       <<<num_sms(), PfCfg<UP>::THREADS, PfCfg<UP>::SMEM, s>>>(prm, map);
   return launch_status();
+}
+template <bool UP>
+static moe_status pf_launch_fmt(int fmt, const PfParams& prm,
+                                const PfMaps& map, cudaStream_t s) {
+  switch (af_of(fmt)) {
+    case AF_SB3: return pf_launch<UP, AF_SB3>(prm, map, s);
+    case AF_NL3: return pf_launch<UP, AF_NL3>(prm, map, s);
+    default: return pf_launch<UP, AF_B32>(prm, map, s);
+  }
 }
 
 moe_status launch_pf_up(const moe_layer_desc& d, const uint16_t* x, int T,
@@ -923,8 +1040,7 @@ moe_status launch_pf_up(const moe_layer_desc& d, const uint16_t* x, int T,
   prm.h16 = reinterpret_cast<__half*>(w.h);
   prm.err = w.err;
   pf_tables(d.fmt_up_gate, prm.tab);
-  return d.fmt_up_gate == MOE_SB3_256 ? pf_launch<true, true>(prm, map, s)
-                                      : pf_launch<true, false>(prm, map, s);
+  return pf_launch_fmt<true>(d.fmt_up_gate, prm, map, s);
 }
 
 moe_status launch_pf_down(const moe_layer_desc& d, int T, int k,
@@ -949,8 +1065,7 @@ moe_status launch_pf_down(const moe_layer_desc& d, int T, int k,
   prm.y = y;
   prm.err = w.err;
   pf_tables(d.fmt_down, prm.tab);
-  return d.fmt_down == MOE_SB3_256 ? pf_launch<false, true>(prm, map, s)
-                                   : pf_launch<false, false>(prm, map, s);
+  return pf_launch_fmt<false>(d.fmt_down, prm, map, s);
 }
 
 }  // namespace moe

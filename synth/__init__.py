@@ -31,8 +31,10 @@ import numpy as np
 Q4_B32 = 1    # 4-bit codes, 32 weights per block, fp16 scale: w = d*(q-8)
 SB3_256 = 2   # 3-bit codes, 256-weight super-block, 8 4-bit sub-scales
 NL4_B32 = 3   # 4-bit codes into a 16-entry int8 codebook, fp16 scale
+NL3_256 = 4   # 3-bit codes into an 8-entry codebook, 256-weight super-block
 
-FMT_NAMES = {Q4_B32: "q4_b32", SB3_256: "sb3_256", NL4_B32: "nl4_b32"}
+FMT_NAMES = {Q4_B32: "q4_b32", SB3_256: "sb3_256", NL4_B32: "nl4_b32",
+             NL3_256: "nl3_256"}
 
 BLOB_ALIGN = 4096  # expert blobs start on 4 KiB boundaries
 
@@ -46,14 +48,19 @@ def tensor_planes(fmt: int, rows: int, cols: int) -> List[Tuple[str, int]]:
                scales  rows*(cols/256)*4 B (sub-scale j at bit 4*j of a
                        little-endian 32-bit word),
                d       rows*(cols/256) fp16.
+      NL3_256: the three SB3 planes, then
+               extra   rows*(cols/256) B (bit j = codebook shift of 32-block j).
       Q4_B32 / NL4_B32: codes rows*cols/2 B (weight i of a row in byte i/2,
                        low nibble for even i), d rows*(cols/32) fp16.
     """
-    if fmt == SB3_256:
+    if fmt in (SB3_256, NL3_256):
         if cols % 256:
-            raise ValueError("SB3_256 needs cols % 256 == 0")
+            raise ValueError("super-block formats need cols % 256 == 0")
         nsb = rows * (cols // 256)
-        return [("codes", nsb * 96), ("scales", nsb * 4), ("d", nsb * 2)]
+        planes = [("codes", nsb * 96), ("scales", nsb * 4), ("d", nsb * 2)]
+        if fmt == NL3_256:
+            planes.append(("extra", nsb))
+        return planes
     if fmt in (Q4_B32, NL4_B32):
         if cols % 32:
             raise ValueError("32-weight block formats need cols % 32 == 0")
@@ -108,6 +115,12 @@ BIG = LayerShape(H=3072, F=1024, E=512, k=10, fmt_up_gate=SB3_256,
                  fmt_down=NL4_B32, d_up_gate=(0.002, 0.01),
                  d_down=(0.002, 0.01))
 
+# The decode layer shape with up/gate in the 3-bit non-uniform-codebook
+# format (64 experts, top-8: a smaller pool for the format's parity tests).
+NL3_SHAPE = LayerShape(H=3072, F=1024, E=64, k=8, fmt_up_gate=NL3_256,
+                       fmt_down=NL4_B32, d_up_gate=(0.002, 0.01),
+                       d_down=(0.002, 0.01))
+
 ZIPF_S = 1.1
 ROUTER_STD = 0.02
 
@@ -150,7 +163,7 @@ def stream_words(key: int, start: int, n: int) -> np.ndarray:
 
 # Stream ids of the three tensors and their planes.
 TENSOR_ID = {"up": 0, "gate": 1, "down": 2}
-PLANE_ID = {"codes": 0, "scales": 1, "d": 2}
+PLANE_ID = {"codes": 0, "scales": 1, "d": 2, "extra": 3}
 
 
 def _random_bytes(key: int, n: int) -> np.ndarray:

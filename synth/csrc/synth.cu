@@ -36,11 +36,11 @@ __device__ inline uint64_t word(uint64_t key, uint64_t i) {
 struct Plane {
   int64_t offset;   // byte offset in the tensor
   int64_t bytes;
-  int id;           // 0 codes, 1 scales, 2 d
+  int id;           // 0 codes, 1 scales, 2 d, 3 extra (NL3)
 };
 
 struct TensorSpec {
-  Plane planes[3];
+  Plane planes[4];
   int nplanes;
   int64_t bytes;
   int tensor_id;
@@ -104,13 +104,18 @@ TensorSpec make_spec(int fmt, int rows, int cols, int tensor_id, double lo,
   s.tensor_id = tensor_id;
   s.lo = lo;
   s.hi = hi;
-  if (fmt == 2) {  // SB3
+  if (fmt == 2 || fmt == 4) {  // SB3, NL3 (+ one shift byte per block)
     const int64_t nsb = (int64_t)rows * (cols / 256);
     s.planes[0] = {0, nsb * 96, 0};
     s.planes[1] = {nsb * 96, nsb * 4, 1};
     s.planes[2] = {nsb * 100, nsb * 2, 2};
     s.nplanes = 3;
     s.bytes = nsb * 102;
+    if (fmt == 4) {
+      s.planes[3] = {nsb * 102, nsb, 3};
+      s.nplanes = 4;
+      s.bytes = nsb * 103;
+    }
   } else {  // Q4 / NL4
     const int64_t nb = (int64_t)rows * (cols / 32);
     s.planes[0] = {0, nb * 16, 0};

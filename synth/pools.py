@@ -14,7 +14,10 @@ from . import device as sdev
 
 
 def dev(a) -> torch.Tensor:
-    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    a = np.ascontiguousarray(a)
+    if not a.flags.writeable:      # e.g. a view of an immutable buffer
+        a = a.copy()
+    return torch.from_numpy(a).cuda()
 
 
 def build_pool(shape: LayerShape, seed: int, layer: int,

@@ -52,6 +52,7 @@ def check(fmt, path, nat, rows, cols):
     (synth.NL4_B32, 128, 64), (synth.NL4_B32, 128, 192),
     (synth.NL4_B32, 3072, 1024),
     (synth.Q4_B32, 128, 128), (synth.Q4_B32, 256, 256),
+    (synth.NL3_256, 128, 256), (synth.NL3_256, 1024, 3072),
 ])
 def test_hot_path_decoders_random(fmt, rows, cols, path):
     nat = synth.gen_tensor(13, 1, rows + cols, "up", fmt, rows, cols,
@@ -87,6 +88,37 @@ def sb3_every_pair(rows=128, dmin=0.001, dmax=0.03):
         scales += acc.to_bytes(4, "little")
     d = np.linspace(dmin, dmax, rows).astype(np.float16).tobytes()
     return np.frombuffer(bytes(codes) + bytes(scales) + d, np.uint8)
+
+
+def nl3_every_triple(rows=256, dmin=0.001, dmax=0.03):
+    """Natural NL3 tensor [rows x 256]: row r has sub-scales
+    (r//16 + j) % 16, codes (r + i) % 8 and shift byte 0x55 or 0xAA
+    (alternate blocks shifted, both phases), so every (s, q, e) occurs."""
+    codes, scales, extra = bytearray(), bytearray(), bytearray()
+    for r in range(rows):
+        s, q = (r // 16) % 16, r % 8
+        acc = 0
+        for i in range(256):
+            acc |= ((q + i) % 8) << (3 * i)
+        codes += acc.to_bytes(96, "little")
+        acc = 0
+        for j in range(8):
+            acc |= ((s + j) % 16) << (4 * j)
+        scales += acc.to_bytes(4, "little")
+        extra.append(0x55 if (r // 8) % 2 == 0 else 0xAA)
+    d = np.linspace(dmin, dmax, rows).astype(np.float16).tobytes()
+    return np.frombuffer(bytes(codes) + bytes(scales) + d + bytes(extra),
+                         np.uint8)
+
+
+@pytest.mark.parametrize("path", [DEC, PF])
+def test_nl3_every_subscale_code_and_shift(path):
+    nat = nl3_every_triple()
+    trip = {(((r // 16) + i // 32) % 16, (r + i) % 8,
+             ((0x55 if (r // 8) % 2 == 0 else 0xAA) >> (i // 32)) & 1)
+            for r in range(256) for i in range(256)}
+    assert len(trip) == 16 * 8 * 2
+    check(synth.NL3_256, path, nat, 256, 256)
 
 
 def b32_every_code(rows=128, cols=128, dmin=0.001, dmax=0.03):

@@ -15,6 +15,7 @@ pytestmark = pytest.mark.gpu
 @pytest.mark.parametrize("shape,layer,experts", [
     (synth.TINY, 0, list(range(16))),
     (synth.BIG, 3, [0, 257, 511]),
+    (synth.NL3_SHAPE, 1, [0, 5, 63]),
 ])
 def test_device_generator_matches_host(shape, layer, experts):
     stride = shape.blob_stride
@@ -35,6 +36,8 @@ def test_device_generator_matches_host(shape, layer, experts):
     (synth.NL4_B32, 16, 64), (synth.NL4_B32, 48, 192),
     (synth.NL4_B32, 3072, 1024),
     (synth.Q4_B32, 32, 128), (synth.Q4_B32, 128, 256),
+    (synth.NL3_256, 16, 256), (synth.NL3_256, 48, 768),
+    (synth.NL3_256, 1024, 3072),
 ])
 def test_pack_dequant_bit_exact(fmt, rows, cols):
     nat = synth.gen_tensor(11, 2, rows + cols, "up", fmt, rows, cols,

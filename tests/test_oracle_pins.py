@@ -110,6 +110,69 @@ def test_sb3_bit_positions_are_a_bijection():
     assert np.all(seen.sum(1) == 3)
 
 
+def test_nl3_hand_worked_superblock():
+    meta, rows = _read_golden("nl3_superblock.txt")
+    raw = np.frombuffer(meta["codes_hex"] + meta["scales_hex"] +
+                        meta["d_hex"] + meta["extra_hex"], np.uint8)
+    assert raw.size == 103
+    w = o.dequant_nl3(raw, 1, 256)[0]
+    for i, exp in rows:
+        assert w[int(i)] == exp, (i, w[int(i)], exp)
+
+
+def test_nl3_every_subscale_code_and_shift():
+    # one super-block per (s, q, e), d = 1: every weight is
+    # (2s+1)(cb3[q]+e)/16 with the configured codebook written out here
+    cb3 = [-15, -10, -6, -2, 1, 5, 9, 14]
+    trip = list(itertools.product(range(16), range(8), range(2)))
+    codes = b"".join(_pack_bits([q] * 256, 3) for s, q, e in trip)
+    scales = b"".join(_pack_bits([s] * 8, 4) for s, q, e in trip)
+    d = np.full(len(trip), 1.0, np.float16).tobytes()
+    extra = bytes([0xFF if e else 0x00 for s, q, e in trip])
+    raw = np.frombuffer(codes + scales + d + extra, np.uint8)
+    w = o.dequant_nl3(raw, len(trip), 256)
+    for r, (s, q, e) in enumerate(trip):
+        assert np.all(w[r] == (2 * s + 1) * (cb3[q] + e) / 16.0), (s, q, e)
+
+
+def test_nl3_shift_bits_and_code_positions():
+    # Flipping shift bit j raises exactly the 32 weights of block j, by
+    # d(2s_j+1)/16; flipping code bit b of weight i changes weight i alone.
+    rng = np.random.default_rng(2)
+    s = rng.integers(0, 16, 8)
+    q = rng.integers(0, 8, 256)
+    codes, scales = _pack_bits(q, 3), _pack_bits(s, 4)
+    d = np.array([0.5], np.float16).tobytes()
+    base = o.dequant_nl3(np.frombuffer(codes + scales + d + bytes(1),
+                                       np.uint8), 1, 256)[0]
+    for j in range(8):
+        w = o.dequant_nl3(np.frombuffer(codes + scales + d + bytes([1 << j]),
+                                        np.uint8), 1, 256)[0]
+        diff = np.nonzero(w != base)[0]
+        assert diff.tolist() == list(range(32 * j, 32 * j + 32))
+        assert np.all(w[diff] - base[diff] == 0.5 * (2 * s[j] + 1) / 16.0)
+    for bit in range(0, 768, 7):
+        cb = bytearray(codes)
+        cb[bit // 8] ^= 1 << (bit % 8)
+        w = o.dequant_nl3(np.frombuffer(bytes(cb) + scales + d + bytes(1),
+                                        np.uint8), 1, 256)[0]
+        assert np.nonzero(w != base)[0].tolist() == [bit // 3]
+
+
+def test_nl3_codebook_and_generated_range():
+    assert o.NL3_CODEBOOK.tolist() == [-15, -10, -6, -2, 1, 5, 9, 14]
+    raw = synth.gen_tensor(0, 0, 0, "up", synth.NL3_256, 16, 512,
+                           (0.002, 0.01))
+    assert raw.size == 16 * 2 * 103
+    w = o.dequant_nl3(raw, 16, 512)
+    assert np.abs(w).max() <= 0.01 * 31 * 15 / 16 + 1e-12
+    # every weight exact in fp32 (|(2s+1)(cb3+e)| <= 465, d fp16)
+    assert np.array_equal(w.astype(np.float32).astype(np.float64), w)
+    # both shift values occur
+    ex = raw[-32:]
+    assert 0 < np.unpackbits(ex).sum() < 256
+
+
 @pytest.mark.parametrize("fmt,col", [(o.NL4_B32, 1), (o.Q4_B32, 2)])
 def test_b32_hand_worked_block(fmt, col):
     meta, rows = _read_golden("b32_block.txt")
