@@ -177,6 +177,24 @@ moe_status moe_group_tokens(const int32_t* topk_idx, int T, int k, int E,
                             int32_t* active, int32_t* n_active, void* ws,
                             size_t ws_bytes, void* stream);
 
+/* A grouping restricted to a list of experts, for computing a layer's
+ * experts in waves (prefill through the expert-slot pool: the experts whose
+ * blobs are on the device first, the others as their blobs arrive; Avalon
+ * README, "Expert prefetch during prefill").  From a grouping made by
+ * moe_group_tokens (expert_offsets [E+1], pair_ids [T*k]) and a device list
+ * experts[0..n-1] of distinct expert ids, builds the grouping of just those
+ * experts' pairs, in the same order: sub_offsets int32 [E+1] (empty ranges
+ * for unlisted experts), sub_pairs int32 [T*k] (the first sub_offsets[E]
+ * entries are valid), sub_active int32 [E] and sub_n_active int32 [1] as in
+ * moe_group_tokens.  An id outside [0, E) sets MOE_ERR_DEVICE in err
+ * (device word) and is ignored.  E <= 4096, 0 <= n <= E. */
+moe_status moe_group_subset(const int32_t* expert_offsets,
+                            const int32_t* pair_ids, int E,
+                            const int32_t* experts, int n,
+                            int32_t* sub_offsets, int32_t* sub_pairs,
+                            int32_t* sub_active, int32_t* sub_n_active,
+                            int32_t* err, void* stream);
+
 /* Allocation-free variant of moe_group_tokens (no counterpart in the
  * source pages: it exists for callers of this library that cannot
  * allocate device memory where they call it -- a plugin or custom operator
@@ -311,7 +329,10 @@ moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream);
  *   A bf16 activation keeps every bit when it is at least 2^-6 times the
  *   largest magnitude of its 256-column block.
  * T > 8 with H, F multiples of 128 (the prefill path): grouped GEMMs on the
- *   5th-generation tensor cores in fp16 with fp32 accumulation.  Each
+ *   5th-generation tensor cores in fp16 with fp32 accumulation.  On this
+ *   path the grouping may list a subset of the T*k pairs (moe_group_subset):
+ *   only the listed pairs' rows of y_pairs are written, and each is
+ *   bit-identical to the row the full grouping gives.  Each
  *   weight enters as the round-to-nearest fp16 of its exact value, each
  *   activation row as fp16 after a per-row power-of-two scale that keeps
  *   it below 2^15, and h = silu(g) u is kept as fp16 (silu formed with the

@@ -60,6 +60,8 @@ _SIGS = {
                                  _P, c_size_t, _P]),
     "moe_group_tokens_static": (c_int, [_P, c_int, c_int, c_int, _P, _P,
                                         _P, _P, _P, _P]),
+    "moe_group_subset": (c_int, [_P, _P, c_int, _P, c_int, _P, _P, _P, _P,
+                                 _P, _P]),
     "moe_slot_resolve": (c_int, [_P, c_int, c_int, c_int, _P, _P, _P, c_int,
                                  c_int, c_uint32, _P, _P, _P, _P, _P, _P]),
     "moe_ffn_workspace_bytes": (c_size_t, [c_int, c_int, c_int, c_int]),
@@ -189,6 +191,14 @@ def moe_group_tokens_static(topk_idx, T, k, E, expert_offsets, pair_ids,
     _check("moe_group_tokens_static", lib.moe_group_tokens_static(
         _ptr(topk_idx), T, k, E, _ptr(expert_offsets), _ptr(pair_ids),
         _ptr(active), _ptr(n_active), _ptr(err), _stream(stream)))
+
+
+def moe_group_subset(expert_offsets, pair_ids, E, experts, n, sub_offsets,
+                     sub_pairs, sub_active, sub_n_active, err, stream=None):
+    _check("moe_group_subset", lib.moe_group_subset(
+        _ptr(expert_offsets), _ptr(pair_ids), E, _ptr(experts), n,
+        _ptr(sub_offsets), _ptr(sub_pairs), _ptr(sub_active),
+        _ptr(sub_n_active), _ptr(err), _stream(stream)))
 
 
 def moe_slot_resolve(topk_idx, T, k, E, slot_table, slot_owner, last_use,

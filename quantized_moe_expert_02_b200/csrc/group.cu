@@ -158,6 +158,61 @@ moe_status launch_group(const int32_t* idx, int T, int k, int E,
   return launch_status();
 }
 
+// The grouping restricted to a list of experts: the first block builds
+// the sub-offsets (counts of the listed experts, exclusive scan) and the
+// active list; every block then copies the listed experts' pair ranges.
+// One launch of SUB_BLOCKS blocks; block 0's scan is redone by every block
+// (E <= EMAX words in shared memory), so no inter-block sync is needed.
+constexpr int SUB_BLOCKS = 64;
+
+__global__ void __launch_bounds__(1024)
+    group_subset_kernel(const int32_t* __restrict__ offsets,
+                        const int32_t* __restrict__ pair_ids, int E,
+                        const int32_t* __restrict__ experts, int n,
+                        int32_t* __restrict__ sub_offsets,
+                        int32_t* __restrict__ sub_pairs,
+                        int32_t* __restrict__ sub_active,
+                        int32_t* __restrict__ sub_n_active, int32_t* err) {
+  __shared__ int32_t cnt[EMAX + 1];
+  __shared__ int32_t mark[EMAX + 1];
+  __shared__ int32_t tmp[32];
+  for (int e = threadIdx.x; e <= E; e += blockDim.x) { cnt[e] = 0; mark[e] = 0; }
+  __syncthreads();
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const int e = experts[i];
+    if (e < 0 || e >= E) {
+      if (blockIdx.x == 0) set_err(err, MOE_ERR_DEVICE);
+      continue;
+    }
+    mark[e] = 1;
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    const int c = mark[e] ? offsets[e + 1] - offsets[e] : 0;
+    cnt[e] = c;
+    mark[e] = c > 0;
+  }
+  __syncthreads();
+  block_exclusive_scan(cnt, E + 1, tmp);
+  const int na = block_exclusive_scan(mark, E + 1, tmp);
+  if (blockIdx.x == 0) {
+    for (int e = threadIdx.x; e <= E; e += blockDim.x) {
+      sub_offsets[e] = cnt[e];
+      if (e < E && mark[e + 1] != mark[e]) sub_active[mark[e]] = e;
+    }
+    if (threadIdx.x == 0) *sub_n_active = na;
+  }
+  // copy: expert e's pairs go to sub_pairs[cnt[e] ..), block b takes the
+  // experts e with e % gridDim.x == b
+  for (int e = blockIdx.x; e < E; e += gridDim.x) {
+    const int c = cnt[e + 1] - cnt[e];
+    if (c <= 0) continue;
+    const int src = offsets[e];
+    for (int i = threadIdx.x; i < c; i += blockDim.x)
+      sub_pairs[cnt[e] + i] = pair_ids[src + i];
+  }
+}
+
 }  // namespace moe
 
 // ---------------------------------------------------------------------
@@ -231,6 +286,20 @@ moe_status group_scratch_address(int32_t** out) {
 }  // namespace moe
 
 using namespace moe;
+
+extern "C" moe_status moe_group_subset(
+    const int32_t* expert_offsets, const int32_t* pair_ids, int E,
+    const int32_t* experts, int n, int32_t* sub_offsets, int32_t* sub_pairs,
+    int32_t* sub_active, int32_t* sub_n_active, int32_t* err, void* stream) {
+  if (!expert_offsets || !pair_ids || !experts || !sub_offsets ||
+      !sub_pairs || !sub_active || !sub_n_active || !err)
+    return MOE_ERR_INVALID;
+  if (E <= 0 || E > EMAX || n < 0 || n > E) return MOE_ERR_SHAPE;
+  group_subset_kernel<<<SUB_BLOCKS, 1024, 0, (cudaStream_t)stream>>>(
+      expert_offsets, pair_ids, E, experts, n, sub_offsets, sub_pairs,
+      sub_active, sub_n_active, err);
+  return launch_status();
+}
 
 extern "C" moe_status moe_group_tokens_static(
     const int32_t* topk_idx, int T, int k, int E, int32_t* expert_offsets,

@@ -843,10 +843,22 @@ __global__ void __launch_bounds__(1024)
 
 // inv[pair_ids[r]] = r: the grouped row of every pair (pair_ids is a
 // permutation of 0 .. P-1, as the grouping produces it).
-__global__ void pf_inv_kernel(const int32_t* __restrict__ pair_ids, int P,
-                              int32_t* __restrict__ inv) {
+// Grouped row of each pair: inv[pair_ids[r]] = r for the n_rows listed
+// pairs (the grouping may list a subset of the P pairs); unlisted pairs
+// keep -1 (inv is filled with -1 first by pf_fill_kernel).
+__global__ void pf_inv_kernel(const int32_t* __restrict__ pair_ids,
+                              const int32_t* __restrict__ offsets, int E,
+                              int P, int32_t* __restrict__ inv) {
+  const int n_rows = offsets[E];
   const int r = blockIdx.x * blockDim.x + threadIdx.x;
-  if (r < P) inv[pair_ids[r]] = r;
+  if (r < n_rows && r < P) {
+    const int q = pair_ids[r];
+    if (q >= 0 && q < P) inv[q] = r;
+  }
+}
+__global__ void pf_fill_kernel(int32_t* __restrict__ v, int n, int32_t val) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) v[i] = val;
 }
 
 // One block per token t: x[t] as fp16, scaled by a power of two 2^-sigma
@@ -861,6 +873,11 @@ __global__ void __launch_bounds__(256)
   __shared__ int32_t rows[32];
   const int64_t t = blockIdx.x;
   if (threadIdx.x < k) rows[threadIdx.x] = inv[t * k + threadIdx.x];
+  __syncthreads();
+  // a token none of whose pairs the grouping lists is not needed
+  bool any = false;
+  for (int j = 0; j < k; ++j) any |= rows[j] >= 0;
+  if (!any) return;
   const uint4* xr = reinterpret_cast<const uint4*>(x + t * H);
   const int nch = H / 8;
   float m = 0.f;
@@ -881,7 +898,8 @@ __global__ void __launch_bounds__(256)
   int sigma = 0;
   if (m >= 32768.f && m <= 3.0e38f) sigma = ilogbf(m) - 14;
   const float inv_s = ldexpf(1.f, -sigma);
-  if (threadIdx.x < k) xscale[rows[threadIdx.x]] = ldexpf(1.f, sigma);
+  if (threadIdx.x < k && rows[threadIdx.x] >= 0)
+    xscale[rows[threadIdx.x]] = ldexpf(1.f, sigma);
   for (int c = threadIdx.x; c < nch; c += blockDim.x) {
     const uint4 v = __ldg(xr + c);
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -894,7 +912,8 @@ __global__ void __launch_bounds__(256)
     }
     const uint4 hv = make_uint4(h[0], h[1], h[2], h[3]);
     for (int j = 0; j < k; ++j)
-      reinterpret_cast<uint4*>(xg + (int64_t)rows[j] * H)[c] = hv;
+      if (rows[j] >= 0)
+        reinterpret_cast<uint4*>(xg + (int64_t)rows[j] * H)[c] = hv;
   }
 }
 
@@ -1018,8 +1037,10 @@ moe_status launch_pf_up(const moe_layer_desc& d, const uint16_t* x, int T,
   PfMaps map;
   moe_status st = encode_maps(&map, w.x16, (uint64_t)d.H, (uint64_t)P);
   if (st != MOE_OK) return st;
-  pf_inv_kernel<<<(unsigned)((P + 255) / 256), 256, 0, s>>>(pair_ids, (int)P,
-                                                           w.inv);
+  pf_fill_kernel<<<(unsigned)((P + 255) / 256), 256, 0, s>>>(w.inv, (int)P,
+                                                            -1);
+  pf_inv_kernel<<<(unsigned)((P + 255) / 256), 256, 0, s>>>(
+      pair_ids, offsets, d.E, (int)P, w.inv);
   pf_xg_kernel<<<T, 256, 0, s>>>(x, d.H, k, w.inv, w.x16, w.xscale);
   pf_plan_kernel<<<1, 1024, 0, s>>>(offsets, d.E, w.tiles, w.n_tiles);
   st = launch_status();
