@@ -16,6 +16,7 @@ the decode layer does not shard); max-over-ranks device time.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import os
 import statistics
@@ -280,12 +281,12 @@ class Layers:
     """Resident layers (packed expert pools, router weights) and the
     per-T step buffers."""
 
-    def __init__(self, L: int, n_x: int = 64):
+    def __init__(self, L: int, n_x: int = 64, shape=None):
         import torch
         from synth.pools import build_pool, dev, layer_desc
         import quantized_moe_expert_02_b200 as moe
         self.moe, self.torch, self.dev = moe, torch, dev
-        shp = synth.BIG
+        shp = self.shape = synth.BIG if shape is None else shape
         self.L, self.n_x = L, n_x
         self.pools = [build_pool(shp, 0, l) for l in range(L)]
         self.descs = [layer_desc(shp, p) for p in self.pools]
@@ -295,7 +296,7 @@ class Layers:
     def buffers(self, T: int):
         if T in self.bufs:
             return self.bufs[T]
-        torch, moe, shp = self.torch, self.moe, synth.BIG
+        torch, moe, shp = self.torch, self.moe, self.shape
         b = {}
         b["xs"] = [self.dev(synth.gen_x(0, T, shp.H, s)) for s in range(self.n_x)]
         b["ws_bytes"] = moe.moe_layer_workspace_bytes(T, shp.k, shp.E, shp.H,
@@ -320,7 +321,7 @@ class Layers:
 
     def step(self, T: int, i: int, x=None, out=None):
         """One decode layer through the C ABI (one launch)."""
-        b, shp = self.buffers(T), synth.BIG
+        b, shp = self.buffers(T), self.shape
         l = i % self.L
         xx = b["xs"][i % self.n_x] if x is None else x
         self.moe.moe_layer_forward(self.descs[l], xx, T, shp.k, self.wr[l],
@@ -331,7 +332,7 @@ class Layers:
 
     def unique_experts(self, T: int, i: int) -> int:
         """Distinct experts of step i (untimed: routing only)."""
-        b, shp = self.buffers(T), synth.BIG
+        b, shp = self.buffers(T), self.shape
         l = i % self.L
         self.moe.moe_route_topk(b["xs"][i % self.n_x], T, shp.H, self.wr[l],
                                 shp.E, None, shp.k, b["idx"], b["w"], b["lg"])
@@ -530,10 +531,90 @@ def decode_measure(lay, T, K, W):
     uniq = [lay.unique_experts(T, W + i) for i in range(min(K, lay.L * 4))]
     u_avg = sum(uniq) / len(uniq)
     ms = graph_time(K, W, lambda i: lay.step(T, i), per_graph=lay.L * 4)
-    bytes_step = WR_BYTES + u_avg * BLOB + T * 3072 * 6
+    bytes_step = WR_BYTES + u_avg * lay.shape.blob_bytes + T * 3072 * 6
+    hbm, _, _ = peaks()
+    gbs = bytes_step / (ms / K * 1e-3) / 1e9
     return {"tokens_per_s": T * K / (ms / 1e3), "ms_per_step": ms / K,
-            "layer_gbs": bytes_step / (ms / K * 1e-3) / 1e9,
+            "layer_gbs": gbs, "frac_of_hbm": gbs / hbm,
             "unique_experts_per_step": u_avg}, ms
+
+
+def clock_soak(lay, T: int, ms_per_step: float, seconds: float = 1.0):
+    """nvidia-smi clock samples over about `seconds` of the same decode
+    steps (graph replays): the timed region itself may be too short for
+    the 200 ms sampler."""
+    import torch
+    props = torch.cuda.get_device_properties(torch.cuda.current_device())
+    uuid = getattr(props, "uuid", None)
+    clk = ClockSampler(f"GPU-{uuid}" if uuid else None)
+    n = max(lay.L * 4, int(seconds / max(ms_per_step * 1e-3, 1e-6)))
+    clk.start()
+    graph_time(n, 0, lambda i: lay.step(T, i), per_graph=lay.L * 4)
+    out = clk.stop()
+    if out is not None:
+        out["steps"] = n
+    return out
+
+
+def nl3_decode(T: int, K: int, W: int) -> dict:
+    """The decode layer with up/gate in the 3-bit non-uniform-codebook
+    format (NL3) at the 512-expert shape: two resident layers rotated."""
+    import torch
+    shape = dataclasses.replace(synth.BIG, fmt_up_gate=synth.NL3_256)
+    lay = Layers(2, shape=shape)
+    d, _ = decode_measure(lay, T, K, W)
+    d["workload"] = (f"decode, one MoE layer: {T} tokens, 512 experts "
+                     "top-10, NL3 up/gate + NL4 down")
+    d["blob_bytes"] = shape.blob_bytes
+    del lay
+    torch.cuda.empty_cache()
+    return d
+
+
+def prefill_slots_measure(pool, cap: int = 92, borrow: int = 8,
+                          l: int = 0) -> dict:
+    """The prefill chunk through one layer's slot partition (`cap` slots
+    holding the layer's hottest experts, `borrow` of them borrowed), the
+    misses streamed from a pinned host store: device time of one call and
+    bit-exactness against the all-resident layer."""
+    import torch
+    from synth.pools import dev, layer_desc
+    from synth.prefill_slots import Partition, PrefillSlots
+    import quantized_moe_expert_02_b200 as moe
+    shp, T = synth.BIG, PF_T
+    _, rank = synth.gen_zipf_bias(0, l, shp.E)
+    part = Partition(shp, pool, synth.hottest_experts(rank, cap), cap)
+    store = torch.empty((shp.E, shp.blob_bytes), dtype=torch.uint8)
+    store = store.pin_memory()
+    for e in range(shp.E):
+        o = e * shp.blob_stride
+        store[e].copy_(pool[o:o + shp.blob_bytes])
+    ps = PrefillSlots(shp, part, store, {e: e for e in range(shp.E)}, T,
+                      borrow=borrow)
+    pf = Prefill(pool, layer_desc(shp, pool), l)
+    pf.step()
+    out = torch.empty((T, shp.H), device="cuda")
+    ps.forward(pf.x, pf.wr, pf.bias, out)          # warm
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    stats = ps.forward(pf.x, pf.wr, pf.bias, out)
+    e1.record()
+    e1.synchronize()
+    ms = e0.elapsed_time(e1)
+    exact = bool(torch.equal(out, pf.out))
+    del ps, part, store, pf
+    torch.cuda.empty_cache()
+    return {"workload": (f"prefill chunk ({T} tokens) through one layer's "
+                         f"{cap}-slot partition, {borrow} slots borrowed, "
+                         "misses streamed from pinned host memory"),
+            "ms_per_step": ms, "tokens_per_s": T / (ms / 1e3),
+            "chosen_experts": stats["chosen"], "hits": stats["hits"],
+            "misses": stats["misses"], "waves": stats["waves"],
+            "h2d_bytes": stats["h2d_bytes"],
+            "h2d_gbs": stats["h2d_bytes"] / (ms * 1e-3) / 1e9,
+            "bit_exact_vs_resident": exact}
 
 
 # -------------------------------------------------------------- prefill ---
@@ -763,12 +844,48 @@ def run_ours(args) -> None:
             "gpu_launches": LAUNCHES_PER_STEP * K,
             "clocks": clocks,
         }
+        line["clocks_soak"] = clock_soak(lay, T, ms / K)
         if not args.no_prefill:
             pf = Prefill(lay.pools[0], lay.descs[0])
             line["prefill"] = prefill_measure(pf, 10, 3)
             del pf
+            torch.cuda.empty_cache()
+            if world == 1:
+                line["prefill"]["through_slots"] = prefill_slots_measure(
+                    lay.pools[0])
+        if world == 1 and not args.no_extras:
+            line["decode_nl3"] = nl3_decode(T, 4096, W)
         if not args.no_cpu_baseline and world == 1:
             line["cpu_baseline"] = cpu_baseline(T)
+            line["speedup_vs_cpu_baseline"] = \
+                tok_s / line["cpu_baseline"]["value"]
+        if world == 1 and not args.no_extras:
+            del lay
+            torch.cuda.empty_cache()
+            res = stack_measure(args.stack_steps, 3, 2, 8.0, False)
+            line["stack"] = {
+                "workload": ("decode, 48-layer MoE stack: 3 tokens per step,"
+                             " Zipf(1.1) routing bias, residual add; all "
+                             "48 x 512 experts resident, one CUDA graph per"
+                             " step"),
+                "steps": res["S"], "tokens_per_s": res["tokens_per_s"],
+                "ms_per_step": res["ms_per_step"], "layer_gbs": res["gbs"],
+                "frac_of_hbm": res["frac"],
+                "unique_experts_per_layer_step": res["u_avg"],
+                "graph_replay_matches_eager":
+                    res["graph_replay_matches_eager"],
+                "slot_cache": {
+                    "capacities": res["slot_capacities"],
+                    "steps": res["slot_cache_in_stream"]["steps"],
+                    "in_stream_tokens_per_s":
+                        res["slot_cache_in_stream"]["tokens_per_s"],
+                    "one_graph_per_step_tokens_per_s":
+                        res["slot_cache_in_stream"]["graph"]["tokens_per_s"],
+                    "bit_exact_vs_resident":
+                        res["slot_cache_in_stream"]["bit_exact_vs_resident"]
+                        and res["slot_cache_in_stream"]["graph"][
+                            "bit_exact_vs_resident"]},
+                "clocks": res["clocks"]}
     if dist:
         dist.barrier()
         dist.destroy_process_group()
@@ -776,15 +893,18 @@ def run_ours(args) -> None:
         print(json.dumps(line), flush=True)
 
 
-def run_stack(args) -> None:
-    """`--workload stack`: the 48-layer decode stack (3 tokens per step,
-    Zipf-biased routing, residual add between layers).  All 48 x 512 experts
-    resident (105 GB) for the headline; then the same steps through the
-    expert-slot pool (240 / 92 / 60 slots per layer, 19.9 GB), misses copied
-    from pinned host memory, checked bit-exact against the resident run."""
+def stack_measure(S: int, W: int, reps: int, store_gb: float,
+                  host_roundtrip: bool = True) -> dict:
+    """The 48-layer decode stack (3 tokens per step, Zipf-biased routing,
+    residual add between layers) over S steps.  All 48 x 512 experts
+    resident (105 GB), one CUDA graph per step; then the same steps through
+    the expert-slot pool (240 / 92 / 60 slots per layer, 19.9 GB), misses
+    from a pinned host store -- after a host round trip per layer (if
+    host_roundtrip), pulled in-stream eagerly, and as one captured graph
+    per step -- each checked bit-exact against the resident run."""
     import torch
     from synth.stack import SlotPool, Stack
-    L, T, S, W = 48, 3, args.steps, args.warmup
+    L, T = 48, 3
     shp = synth.BIG
     t0 = time.perf_counter()
     st = Stack(L, shp, seed=0, T=T)
@@ -817,7 +937,7 @@ def run_stack(args) -> None:
     uuid = getattr(props, "uuid", None)
     clk = ClockSampler(f"GPU-{uuid}" if uuid else None)
     clk.start()
-    reps = max(1, args.stack_reps)
+    reps = max(1, reps)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record()
@@ -833,11 +953,10 @@ def run_stack(args) -> None:
     same_resident = bool(torch.equal(r, ref[-1]))
     del graphs
     # slot cache: a discovery run (misses copied from the resident pools)
-    # tells which blobs the pinned host store must hold; the timed run then
-    # copies every miss from that store
+    # tells which blobs the pinned host store must hold
     caps = [synth.slot_capacity(l) for l in range(L)]
     disc = SlotPool(st, caps, None)
-    max_blobs = int(args.store_gb * 1e9 // shp.blob_bytes)
+    max_blobs = int(store_gb * 1e9 // shp.blob_bytes)
     S4 = 0   # slot-cache steps: the longest prefix whose misses fit the store
     for s in range(S):
         r.copy_(xs[s])
@@ -853,30 +972,50 @@ def run_stack(args) -> None:
     t0 = time.perf_counter()
     pool = SlotPool(st, caps, keys)
     store_s = time.perf_counter() - t0
-    outs = []
-    torch.cuda.synchronize()
-    e0.record()
-    t0 = time.perf_counter()
-    for s in range(S4):
-        r.copy_(xs[s])
-        pool.run(r, s + 1)
-        outs.append(r.clone())
-    e1.record()
-    e1.synchronize()
-    slot_ms = e0.elapsed_time(e1)
-    slot_wall = time.perf_counter() - t0
-    bit_exact = all(torch.equal(a, b) for a, b in zip(outs, ref[:S4]))
-    host_misses = pool.misses
-    # the same steps with the misses pulled from the pinned host store by
-    # the library on the stream itself: no host sync per layer
+    hbm, tf, src = peaks()
+    gbs = bytes_step / (ms / S * 1e-3) / 1e9
+    res = {"S": S, "ms": ms, "ms_per_step": ms / S,
+           "tokens_per_s": T * S / (ms / 1e3), "gbs": gbs,
+           "frac": gbs / hbm, "peak": hbm, "peak_source": src,
+           "bytes_step": bytes_step, "u_avg": u_avg,
+           "graph_replay_matches_eager": same_resident, "setup_s": setup_s,
+           "clocks": clocks}
+    if host_roundtrip:
+        outs = []
+        torch.cuda.synchronize()
+        e0.record()
+        t0 = time.perf_counter()
+        for s in range(S4):
+            r.copy_(xs[s])
+            pool.run(r, s + 1)
+            outs.append(r.clone())
+        e1.record()
+        e1.synchronize()
+        slot_ms = e0.elapsed_time(e1)
+        slot_wall = time.perf_counter() - t0
+        bit_exact = all(torch.equal(a, b) for a, b in zip(outs, ref[:S4]))
+        res["slot_cache"] = {
+            "steps": S4,
+            "tokens_per_s": T * S4 / (slot_ms / 1e3),
+            "ms_per_step": slot_ms / max(1, S4), "wall_s": slot_wall,
+            "capacities": "240 (layers 0-4), 92 (5-31), 60 (32-47)",
+            "misses": pool.misses,
+            "miss_rate": pool.misses / float(np.sum(uniq[:S4])),
+            "h2d_bytes": pool.misses * shp.blob_bytes,
+            "host_store_blobs": len(keys),
+            "host_store_build_s": store_s,
+            "bit_exact_vs_resident": bit_exact}
+        del outs
+    # the misses pulled from the pinned host store by the library on the
+    # stream itself: no host sync per layer
     pool.reset()
     pool.start_staging()
-    outs = []
     for s in range(min(S4, W)):          # untimed: the launch path warm
         r.copy_(xs[s])
         pool.run_staged(r)
     pool.reset()
     torch.cuda.synchronize()
+    outs = []
     e0.record()
     for s in range(S4):
         r.copy_(xs[s])
@@ -905,11 +1044,37 @@ def run_stack(args) -> None:
     gr_exact = all(torch.equal(a, b) for a, b in zip(outs, ref[:S4])) and \
         int(pool.err.item()) == 0
     del outs, g
-    hbm, tf, src = peaks()
-    gbs = bytes_step / (ms / S * 1e-3) / 1e9
+    res["slot_cache_in_stream"] = {
+        "steps": S4,
+        "tokens_per_s": T * S4 / (db_ms / 1e3),
+        "ms_per_step": db_ms / max(1, S4),
+        "how": ("per layer on one stream: route, resolve, a kernel that "
+                "pulls each missed blob from the pinned host store over "
+                "PCIe into its slot, FFN; no host sync per layer"),
+        "bit_exact_vs_resident": db_exact,
+        "graph": {
+            "tokens_per_s": T * S4 / (gr_ms / 1e3),
+            "ms_per_step": gr_ms / max(1, S4),
+            "how": ("the whole step (48 x route, device-stamped "
+                    "resolve, pull, FFN) captured once as one CUDA "
+                    "graph, one replay per step"),
+            "bit_exact_vs_resident": gr_exact}}
+    res["slot_capacities"] = "240 (layers 0-4), 92 (5-31), 60 (32-47)"
+    res["host_store_blobs"] = len(keys)
+    del pool, st
+    torch.cuda.empty_cache()
+    return res
+
+
+def run_stack(args) -> None:
+    """`--workload stack`: the 48-layer decode stack as the headline line
+    (see stack_measure)."""
+    L, T, S, W = 48, 3, args.steps, args.warmup
+    res = stack_measure(S, W, args.stack_reps, args.store_gb, True)
     line = {
-        "metric": METRIC, "value": T * S / (ms / 1e3), "unit": "tokens/s",
-        "n_gpus": 1, "steps": S, "warmup": W, "ms_per_step": ms / S,
+        "metric": METRIC, "value": res["tokens_per_s"], "unit": "tokens/s",
+        "n_gpus": 1, "steps": S, "warmup": W,
+        "ms_per_step": res["ms_per_step"],
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "int8 mma (s32 accumulate) + f32", "data": "synthetic",
         "config": {"workload": ("decode, 48-layer MoE stack: 3 tokens per "
@@ -919,49 +1084,26 @@ def run_stack(args) -> None:
                    "T": T, "layers": L, "H": 3072, "F": 1024, "E": 512,
                    "k": 10, "l2": "inputs larger than L2: 105 GB of experts",
                    "parallelism": "replicas x1"},
-        "layer_gbs": gbs, "layer_frac_of_hbm": gbs / hbm,
+        "layer_gbs": res["gbs"], "layer_frac_of_hbm": res["frac"],
         "roofline": {"bound": "hbm", "kernel": "decode_layer_kernel x 48",
-                     "achieved": gbs, "peak": hbm, "unit": "GB/s",
-                     "frac": gbs / hbm, "peak_source": src, "traffic": None,
-                     "algorithmic_bytes_per_step": bytes_step},
-        "unique_experts_per_layer_step": u_avg,
-        "graph_replay_matches_eager": same_resident,
-        "slot_cache": {
-            "steps": S4,
-            "tokens_per_s": T * S4 / (slot_ms / 1e3),
-            "ms_per_step": slot_ms / max(1, S4), "wall_s": slot_wall,
-            "capacities": "240 (layers 0-4), 92 (5-31), 60 (32-47)",
-            "misses": host_misses,
-            "miss_rate": host_misses / float(np.sum(uniq[:S4])),
-            "h2d_bytes": host_misses * shp.blob_bytes,
-            "host_store_blobs": len(keys),
-            "host_store_build_s": store_s,
-            "bit_exact_vs_resident": bit_exact},
-        "slot_cache_in_stream": {
-            "steps": S4,
-            "tokens_per_s": T * S4 / (db_ms / 1e3),
-            "ms_per_step": db_ms / max(1, S4),
-            "how": ("per layer on one stream: route, resolve, a kernel that "
-                    "pulls each missed blob from the pinned host store over "
-                    "PCIe into its slot, FFN; no host sync per layer"),
-            "bit_exact_vs_resident": db_exact,
-            "graph": {
-                "tokens_per_s": T * S4 / (gr_ms / 1e3),
-                "ms_per_step": gr_ms / max(1, S4),
-                "how": ("the whole step (48 x route, device-stamped "
-                        "resolve, pull, FFN) captured once as one CUDA "
-                        "graph, one replay per step"),
-                "bit_exact_vs_resident": gr_exact}},
-        "setup_s": setup_s,
+                     "achieved": res["gbs"], "peak": res["peak"],
+                     "unit": "GB/s", "frac": res["frac"],
+                     "peak_source": res["peak_source"], "traffic": None,
+                     "algorithmic_bytes_per_step": res["bytes_step"]},
+        "unique_experts_per_layer_step": res["u_avg"],
+        "graph_replay_matches_eager": res["graph_replay_matches_eager"],
+        "slot_cache": res.get("slot_cache"),
+        "slot_cache_in_stream": res["slot_cache_in_stream"],
+        "setup_s": res["setup_s"],
         "gpu_launches": L * S,
-        "clocks": clocks,
+        "clocks": res["clocks"],
     }
     if not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(T)
     print(json.dumps(line), flush=True)
 
 
-PF_LAUNCHES_PER_STEP = 11   # route 2, group 3, pair rows + x16 + plan + up, down, combine
+PF_LAUNCHES_PER_STEP = 12   # route 2, group 3, row-map fill + pair rows + x16 + plan + up, down, combine
 
 
 def run_prefill(args) -> None:
@@ -1055,6 +1197,11 @@ def main():
                     help="stack: timed passes over the steps")
     ap.add_argument("--store-gb", type=float, default=24.0,
                     help="stack: pinned host store limit for slot misses")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the NL3 decode and 48-layer stack objects "
+                         "of the default line")
+    ap.add_argument("--stack-steps", type=int, default=16,
+                    help="steps of the default line's compact stack object")
     ap.add_argument("--no-prefill", action="store_true",
                     help="leave the prefill figures out of the decode line")
     args = ap.parse_args()
