@@ -85,9 +85,9 @@ typedef enum {
 
 /* One MoE layer's experts as the FFN sees them.
  * Expert e's blob starts at pool + blob_index[e] * blob_stride and holds the
- * packed tensors up [F x H] | gate [F x H] | down [H x F] back to back
- * (model card: "Experts packed per layer (up | gate | down contiguous), so a
- * GPU cache fill is one copy per expert").  blob_stride must be a multiple
+ * packed tensors up [F x H] | gate [F x H] | down [H x F] back to back (the
+ * model card's packed expert layout, "Files": each expert's three tensors
+ * adjacent, so that filling a cache slot takes a single copy).  blob_stride must be a multiple
  * of 16 bytes and at least moe_blob_bytes(...). */
 typedef struct {
   int H;            /* hidden size                      */
@@ -179,8 +179,8 @@ moe_status moe_group_tokens(const int32_t* topk_idx, int T, int k, int E,
 
 /* A grouping restricted to a list of experts, for computing a layer's
  * experts in waves (prefill through the expert-slot pool: the experts whose
- * blobs are on the device first, the others as their blobs arrive; Avalon
- * README, "Expert prefetch during prefill").  From a grouping made by
+ * blobs are on the device first, the others as their blobs arrive; the
+ * prefill prefetch of the "Avalon" README's feature list).  From a grouping made by
  * moe_group_tokens (expert_offsets [E+1], pair_ids [T*k]) and a device list
  * experts[0..n-1] of distinct expert ids, builds the grouping of just those
  * experts' pairs, in the same order: sub_offsets int32 [E+1] (empty ranges

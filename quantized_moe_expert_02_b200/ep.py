@@ -1,7 +1,7 @@
 """Expert parallelism: one MoE layer's experts sharded over the ranks of a
-process group, one process per GPU ("Avalon" README, multi-GPU paragraph:
-a second GPU adds expert cache, the MoE layers are shared between the
-GPUs' expert caches, and only tens of KB of activations cross per layer).
+process group, one process per GPU (the "Avalon" README's multi-GPU
+paragraph, where an added GPU holds more of the experts and a decode step
+exchanges only small activation rows between the GPUs).
 
 Placement: expert e lives on rank e % G as that rank's local expert e // G.
 Per layer, every rank with its own tokens:

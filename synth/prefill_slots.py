@@ -1,6 +1,7 @@
 """Driver of the prefill chunk through one layer's expert-slot partition
-("Avalon" README, feature list: expert prefetch during prefill on slots
-borrowed from the GPU expert cache, cached experts read in place).
+(the prefill prefetch of the "Avalon" README's feature list: a few slots
+taken over from the GPU expert cache stream the missing experts while the
+cached ones are used in their slots).
 
 Everything here is orchestration through the library's C ABI -- buffers,
 host-side lists of experts, copies of whole blobs, streams and events; no

@@ -1,6 +1,6 @@
-"""GPU: prefill through the expert-slot pool ("Avalon" README: expert
-prefetch during prefill on slots borrowed from the cache, cached experts
-read in place).
+"""GPU: prefill through the expert-slot pool (the prefill prefetch of the
+"Avalon" README's feature list: a few slots taken over from the expert
+cache stream the missing experts, cached experts are used in their slots).
 
 * moe_group_subset restricts a grouping to a list of experts exactly (the
   oracle's grouping of the same routing, filtered);
