@@ -461,6 +461,28 @@ moe_status moe_layer_ffn_residual(const moe_layer_desc* desc, const float* r,
                                   uint16_t* out_bf16, void* ws,
                                   size_t ws_bytes, void* stream);
 
+/* moe_stage_misses then moe_layer_ffn_residual in one launch, with the
+ * copies overlapping the compute ("Betelgeuse": the decode pass waits on
+ * the pager only for the experts that missed).  The chosen experts that
+ * missed (the slot resolve's n_miss / miss_expert / miss_slot, device) are
+ * computed after the others; while the hit experts are computed, every
+ * block pulls its share of each missed blob from its pinned host copy
+ * table[layer * E + e] (moe_stage_table) into pool slot slot_base +
+ * miss_slot[i] (the layer's partition: slot_base .. slot_base + n_slots - 1
+ * of pool_slots slots of desc->blob_stride bytes at desc->pool), and a
+ * missed expert's tiles are read only once all blocks have written theirs
+ * (a bounded wait: MOE_ERR_TIMEOUT after 0.5 s).  The result is bit for bit
+ * that of the two calls.  Copy errors are reported as in moe_stage_misses,
+ * in the workspace's error word.  Needs the one-kernel shapes of
+ * moe_layer_forward (T <= 8 ...); other shapes run the two calls in turn. */
+moe_status moe_layer_ffn_residual_staged(
+    const moe_layer_desc* desc, const float* r, int T, int k,
+    const int32_t* topk_idx, const float* topk_w, const int32_t* blob_index,
+    float* r_out, uint16_t* out_bf16, const int32_t* n_miss,
+    const int32_t* miss_expert, const int32_t* miss_slot, int layer, int L,
+    const uint64_t* table, int slot_base, int n_slots, int64_t pool_slots,
+    void* ws, size_t ws_bytes, void* stream);
+
 /* Synchronise `stream`, read the FFN/grouping workspace's device error word
  * into *host_err (host pointer, may be NULL) and clear it.  Returns
  * MOE_ERR_DEVICE if it was set, MOE_OK otherwise. */

@@ -89,6 +89,10 @@ _SIGS = {
     "moe_layer_ffn_residual": (c_int, [_P, _P, c_int, c_int, _P, _P, _P, _P,
                                        _P, _P, c_size_t, _P]),
     "moe_stage_table": (c_int, [_P, c_int, _P, _P]),
+    "moe_layer_ffn_residual_staged": (c_int, [_P, _P, c_int, c_int, _P, _P,
+                                              _P, _P, _P, _P, _P, _P, c_int,
+                                              c_int, _P, c_int, c_int,
+                                              c_int64, _P, c_size_t, _P]),
     "moe_stage_misses": (c_int, [_P, _P, _P, c_int, c_int, c_int, c_int, _P,
                                  _P, c_int, c_int, c_int64, c_int64, c_int64,
                                  _P, _P]),
@@ -316,6 +320,20 @@ def moe_layer_ffn_residual(desc, r, T, k, topk_idx, topk_w, blob_index,
         _ptr(desc), _ptr(r), T, k, _ptr(topk_idx), _ptr(topk_w),
         _ptr(blob_index), _ptr(r_out), _ptr(out_bf16), _ptr(ws), ws_bytes,
         _stream(stream)))
+
+
+def moe_layer_ffn_residual_staged(desc, r, T, k, topk_idx, topk_w,
+                                  blob_index, r_out, out_bf16, n_miss,
+                                  miss_expert, miss_slot, layer, L, table,
+                                  slot_base, n_slots, pool_slots, ws,
+                                  ws_bytes, stream=None):
+    _check("moe_layer_ffn_residual_staged",
+           lib.moe_layer_ffn_residual_staged(
+               _ptr(desc), _ptr(r), T, k, _ptr(topk_idx), _ptr(topk_w),
+               _ptr(blob_index), _ptr(r_out), _ptr(out_bf16), _ptr(n_miss),
+               _ptr(miss_expert), _ptr(miss_slot), layer, L, _ptr(table),
+               slot_base, n_slots, pool_slots, _ptr(ws), ws_bytes,
+               _stream(stream)))
 
 
 def moe_stage_table(host_blob, table, stream=None):

@@ -62,7 +62,8 @@ moe_status launch_decode_layer(const moe_layer_desc& d, const uint16_t* x,
                                const float* residual, float* out,
                                uint16_t* out_bf16, int32_t* topk_idx,
                                float* topk_w, float* logits, void* ws,
-                               int32_t* err, cudaStream_t s, int mode);
+                               int32_t* err, cudaStream_t s, int mode,
+                               const StageArgs* stg = nullptr);
 moe_status launch_rmsnorm_bf16(const float* r, int T, int H, uint16_t* x,
                                cudaStream_t s);
 
@@ -555,6 +556,57 @@ extern "C" moe_status moe_layer_ffn_residual(
   return run_down(*desc, T, k, w.offsets, w.pair_ids, w.active, w.n_active,
                   blob_index, w.ffn, nullptr, topk_w, r, r_out, out_bf16, s,
                   true);
+}
+
+extern "C" moe_status moe_stage_misses(const int32_t* n_miss,
+                                       const int32_t* miss_expert,
+                                       const int32_t* miss_slot, int P,
+                                       int layer, int L, int E,
+                                       const uint64_t* table, uint8_t* pool,
+                                       int slot_base, int n_slots,
+                                       int64_t pool_slots,
+                                       int64_t blob_stride,
+                                       int64_t blob_bytes, int32_t* err,
+                                       void* stream);
+
+extern "C" moe_status moe_layer_ffn_residual_staged(
+    const moe_layer_desc* desc, const float* r, int T, int k,
+    const int32_t* topk_idx, const float* topk_w, const int32_t* blob_index,
+    float* r_out, uint16_t* out_bf16, const int32_t* n_miss,
+    const int32_t* miss_expert, const int32_t* miss_slot, int layer, int L,
+    const uint64_t* table, int slot_base, int n_slots, int64_t pool_slots,
+    void* ws, size_t ws_bytes, void* stream) {
+  LayerWs w;
+  moe_status st = check_residual_args(desc, r, T, k, ws, ws_bytes, &w);
+  if (st != MOE_OK) return st;
+  if (!r_out || !topk_idx || !topk_w || !blob_index || !n_miss ||
+      !miss_expert || !miss_slot || !table)
+    return MOE_ERR_INVALID;
+  if (layer < 0 || layer >= L || slot_base < 0 || n_slots < 1 ||
+      pool_slots < 1 || slot_base + (int64_t)n_slots > pool_slots)
+    return MOE_ERR_SHAPE;
+  const int64_t blob = 2 * tensor_bytes_of(desc->fmt_up_gate, desc->F,
+                                           desc->H) +
+                       tensor_bytes_of(desc->fmt_down, desc->H, desc->F);
+  if (blob % 16) return MOE_ERR_SHAPE;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (decode_layer_supported(*desc, T, k)) {
+    const StageArgs sa{n_miss, miss_expert, miss_slot, table, layer,
+                       slot_base, n_slots, pool_slots, blob};
+    return launch_decode_layer(*desc, nullptr, r, T, k, nullptr, nullptr,
+                               blob_index, r, r_out, out_bf16,
+                               const_cast<int32_t*>(topk_idx),
+                               const_cast<float*>(topk_w), w.logits, w.fused,
+                               w.ffn.err, s, DL_FFN, &sa);
+  }
+  // other shapes: the pull kernel, then the FFN half
+  st = moe_stage_misses(n_miss, miss_expert, miss_slot, T * k, layer, L,
+                        desc->E, table, const_cast<uint8_t*>(desc->pool),
+                        slot_base, n_slots, pool_slots, desc->blob_stride,
+                        blob, w.ffn.err, stream);
+  if (st != MOE_OK) return st;
+  return moe_layer_ffn_residual(desc, r, T, k, topk_idx, topk_w, blob_index,
+                                r_out, out_bf16, ws, ws_bytes, stream);
 }
 
 extern "C" moe_status moe_get_device_status(void* ws, int32_t* host_err,

@@ -34,6 +34,13 @@
 //       group of four warps: y of each pair -> global
 //   ||
 //   P5  combine: out[t] = sum_j w[t,j] y[t,j] (+ residual), j ascending
+//
+// Staged FFN variant (STG, expert-slot cache): one more warp per block
+// pulls this block's share of every missed expert's blob from pinned host
+// memory into its slot while the others compute; the grouping puts the
+// missed experts after the hits, and the producer waits (bounded) for a
+// missed expert's blob to be complete in every block before it copies that
+// expert's tiles.
 #include <float.h>
 
 #include "decode_pieces.cuh"
@@ -57,6 +64,12 @@ constexpr int BAR_XF = 8;                   // warps that build x fragments
 constexpr int UPG = 2, UPW = CW / UPG;      // up: 2 groups of 8 warps
 constexpr int DNG = 4, DNW = CW / DNG;      // down: 4 groups of 4 warps
 constexpr int EMAX_FUSED = 1024;            // widest router of this kernel
+constexpr int PULLER = CW + 4;              // STG: pulls missed blobs
+constexpr int LAYER_THREADS_STG = LAYER_THREADS + 32;
+#ifndef MOE_PULL_DEPTH
+#define MOE_PULL_DEPTH 8
+#endif
+constexpr int PULL_DEPTH = MOE_PULL_DEPTH;  // STG: 16-byte loads in flight per lane
 
 struct LayerParams {
   const uint8_t* pool;
@@ -80,6 +93,15 @@ struct LayerParams {
   int32_t* bar;            // ws [2]: grid barrier, exit counter
   int32_t* up_done;        // ws [MAXP]: finished up units per expert
   int32_t* err;
+  // STG: the slot resolve's misses, pulled from pinned host memory
+  const int32_t* n_miss;
+  const int32_t* miss_expert;    // [P], ascending expert id
+  const int32_t* miss_slot;      // [P], slot inside the partition
+  const uint64_t* stage_table;   // device addresses of the host blobs
+  int stage_layer;               // row stage_layer * E of the table
+  int slot_base, n_slots;        // the layer's partition of the pool
+  int64_t pool_slots, blob_bytes;
+  int32_t* ready;                // ws [MAXP]: blocks done with miss m
   int mode;                // DL_FULL, DL_ROUTE (P0-P1 top-k only) or
                            // DL_FFN (top-k read from topk_idx/topk_w)
 };
@@ -133,7 +155,10 @@ struct Misc {
   int32_t off[MAXP + 1];     // pairs of active[u]: sorted[off[u]..off[u+1])
   float hsc[2][8];           // 2^-sigma of each pair slot, down experts
   int32_t up_fin[MAXP];      // up units of each expert finished here
+  uint32_t missmap[EMAX_FUSED / 32];   // STG: experts pulled this call
   int U;
+  int Uhit;                  // STG: active experts before the misses
+  int nmiss;
   int flag;
 };
 
@@ -222,9 +247,10 @@ __device__ __forceinline__ uint32_t frag_word(const float (&v)[4], float sc,
 
 }  // namespace
 
-template <int FUG, int FDN, int NTT, int EPL>
-__global__ void __launch_bounds__(LAYER_THREADS, 1)
+template <int FUG, int FDN, int NTT, int EPL, bool STG>
+__global__ void __launch_bounds__(STG ? LAYER_THREADS_STG : LAYER_THREADS, 1)
     decode_layer_kernel(LayerParams p) {
+  constexpr int NTHR = STG ? LAYER_THREADS_STG : LAYER_THREADS;
   extern __shared__ __align__(128) uint8_t smem[];
   const Smem L = smem_layout(FUG, p.H, p.F, p.T);
   Misc& M = *reinterpret_cast<Misc*>(smem + L.misc);
@@ -258,7 +284,8 @@ __global__ void __launch_bounds__(LAYER_THREADS, 1)
     }
     fence_mbar_init();
   }
-  for (int i = tid; i < MAXP; i += LAYER_THREADS) M.up_fin[i] = 0;
+  for (int i = tid; i < MAXP; i += NTHR) M.up_fin[i] = 0;
+  if (STG && tid < EMAX_FUSED / 32) M.missmap[tid] = 0u;
   // router rows of this block (not in DL_FFN): four warps per row, each a
   // quarter of H.  The kernel is launched as a programmatic dependent of
   // the previous kernel on the stream, and the router weights are the one
@@ -289,10 +316,10 @@ __global__ void __launch_bounds__(LAYER_THREADS, 1)
   grid_dep_wait();
   uint16_t* xs = reinterpret_cast<uint16_t*>(ring);   // [T][H] bf16
   if (p.x) {
-    for (int i = tid; i < T * H / 8; i += LAYER_THREADS)
+    for (int i = tid; i < T * H / 8; i += NTHR)
       reinterpret_cast<uint4*>(xs)[i] = reinterpret_cast<const uint4*>(p.x)[i];
   } else {
-    for (int t = warp; t < T; t += LAYER_THREADS / 32) {
+    for (int t = warp; t < T; t += NTHR / 32) {
       const float* r = p.r_in + (int64_t)t * H;
       float s = 0.f;
       for (int h = lane; h < H; h += 32) s = fmaf(r[h], r[h], s);
@@ -304,8 +331,21 @@ __global__ void __launch_bounds__(LAYER_THREADS, 1)
     }
   }
   if (blockIdx.x == 0)
-    for (int i = tid; i < T * k; i += LAYER_THREADS) p.hmax[i] = 0u;
+    for (int i = tid; i < T * k; i += NTHR) p.hmax[i] = 0u;
   __syncthreads();
+  if (STG) {
+    // the experts this call pulls (the slot resolve's misses)
+    int nm = *p.n_miss;
+    if (nm < 0 || nm > T * k) {
+      if (tid == 0) set_err(p.err, MOE_ERR_DEVICE);
+      nm = 0;
+    }
+    for (int i = tid; i < nm; i += NTHR) {
+      const int e = p.miss_expert[i];
+      if (e >= 0 && e < E) atomicOr(&M.missmap[e >> 5], 1u << (e & 31));
+    }
+    if (tid == 0) M.nmiss = nm;
+  }
   // a lane issues all its loads of the row first (up to RCH 16-byte
   // chunks), then accumulates in fp32; lane sums by a fixed butterfly and
   // the quarters in fixed order (deterministic)
@@ -362,7 +402,7 @@ __global__ void __launch_bounds__(LAYER_THREADS, 1)
       }
     }
     __syncthreads();
-    for (int i = tid; i < nrow * T; i += LAYER_THREADS) {
+    for (int i = tid; i < nrow * T; i += NTHR) {
       const int r = i / T, t = i % T;
       float a = 0.f;
       for (int q = 0; q < RQ; ++q) a += part[(r * RQ + q) * DEC_TMAX + t];
@@ -494,12 +534,19 @@ __global__ void __launch_bounds__(LAYER_THREADS, 1)
     named_bar_sync(BAR_ALL, CW * 32);
     // grouping: rank of pair q = #{r : (e_r, r) < (e_q, q)}
     const int P = p.mode == DL_ROUTE ? 0 : T * k;   // DL_ROUTE: no units
+    // STG: the pulled experts sort after the others (their units come
+    // last, so the hits are computed while the pulls fly)
+    auto gkey = [&](int e) -> int {
+      return (STG && e >= 0 && e < E &&
+              ((M.missmap[e >> 5] >> (e & 31)) & 1u)) ? e + EMAX_FUSED : e;
+    };
     if (tid < P) {
       const int eq = M.tk_idx[tid];
+      const int kq = gkey(eq);
       int rank = 0;
       for (int r = 0; r < P; ++r) {
-        const int er = M.tk_idx[r];
-        rank += (er < eq) || (er == eq && r < tid);
+        const int kr = gkey(M.tk_idx[r]);
+        rank += (kr < kq) || (kr == kq && r < tid);
       }
       M.sorted[rank] = tid;
       if (eq < 0 || eq >= E) set_err(p.err, MOE_ERR_DEVICE);
@@ -522,7 +569,17 @@ __global__ void __launch_bounds__(LAYER_THREADS, 1)
         }
         U += __popc(b);
       }
-      if (lane == 0) { M.U = U; M.off[U] = P; }
+      if (lane == 0) {
+        M.U = U;
+        M.off[U] = P;
+        if (STG) {
+          int uh = 0;
+          while (uh < U && gkey(M.active[uh]) < EMAX_FUSED) ++uh;
+          M.Uhit = uh;
+          // every miss must be a chosen expert of this call
+          if (U - uh != M.nmiss) set_err(p.err, MOE_ERR_DEVICE);
+        }
+      }
     }
   }
   __syncthreads();   // the producer may start now
@@ -573,6 +630,21 @@ __global__ void __launch_bounds__(LAYER_THREADS, 1)
     if (lane == 0) {
       int i = 0;
       bool ok = true;   // false once a wait for a free slot gave up
+      // STG: a pulled expert's tiles are copied only once every block has
+      // written its share of the blob (bounded wait; the bulk copies read
+      // through the async proxy what other SMs stored)
+      uint32_t seen[MAXP / 32] = {0u, 0u, 0u};
+      auto pulled = [&](int u) -> bool {
+        if (!STG) return true;
+        const int m = u - M.Uhit;
+        if (m < 0 || m >= M.nmiss) return true;
+        if ((seen[m >> 5] >> (m & 31)) & 1u) return true;
+        spin_until(p.ready + m, G, p.err);
+        if (ld_acquire(p.ready + m) < G) return false;
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+        seen[m >> 5] |= 1u << (m & 31);
+        return true;
+      };
       auto acquire = [&](int slot_i) {
         const int s = slot_i % NSLOT;
         if (slot_i >= NSLOT &&
@@ -585,6 +657,10 @@ __global__ void __launch_bounds__(LAYER_THREADS, 1)
         const int s = acquire(i);
         if (!ok) break;
         const int u = v / nrt_f, rt = v % nrt_f;
+        if (!pulled(u)) {
+          ok = false;
+          break;
+        }
         const uint8_t* b = expert_base(p, M.active[u]);
         if (!b) { mbar_arrive_expect_tx(&M.full[s], 0); continue; }
         const uint32_t nb = (uint32_t)(nk * TBU);
@@ -597,6 +673,8 @@ __global__ void __launch_bounds__(LAYER_THREADS, 1)
         const int s = acquire(i);
         if (!ok) break;
         const int n = (d1 - v) < dps ? (d1 - v) : dps;
+        for (int j = 0; j < n && ok; ++j) ok = pulled((v + j) / nrt_h);
+        if (!ok) break;
         uint32_t tot = 0;
         const uint8_t* src[DNG];
         for (int j = 0; j < n; ++j) {
@@ -658,6 +736,50 @@ __global__ void __launch_bounds__(LAYER_THREADS, 1)
             break;
           }
         }
+      }
+    }
+    return;
+  }
+
+  // ------------------------------------------------------- puller (STG) --
+  // Copies this block's share (a contiguous 16-byte range) of every missed
+  // blob from its pinned host copy into its slot, PULL_DEPTH loads in flight
+  // per lane, and counts each finished share in ready[m] (release).  A missing
+  // host copy or a slot outside the partition sets MOE_ERR_CAPACITY and the
+  // share is skipped -- and still counted, so that no wait runs out.
+  if (STG && warp == PULLER) {
+    const int nm = M.nmiss;
+    const int64_t words = p.blob_bytes / 16;
+    const int64_t per = (words + G - 1) / G;
+    const int64_t w0 = per * blockIdx.x;
+    const int64_t w1 = w0 + per < words ? w0 + per : words;
+    for (int m = 0; m < nm; ++m) {
+      const int e = p.miss_expert[m];
+      const int ls = p.miss_slot[m];
+      const uint64_t src =
+          (e >= 0 && e < E) ? p.stage_table[(int64_t)p.stage_layer * E + e]
+                            : 0ull;
+      const int64_t slot = (int64_t)p.slot_base + ls;
+      if (src != 0ull && ls >= 0 && ls < p.n_slots && slot < p.pool_slots) {
+        const uint4* s4 = reinterpret_cast<const uint4*>(src);
+        uint4* d4 = reinterpret_cast<uint4*>(const_cast<uint8_t*>(p.pool) +
+                                             slot * p.stride);
+        for (int64_t i0 = w0 + lane; i0 < w1; i0 += 32 * PULL_DEPTH) {
+          uint4 v[PULL_DEPTH];
+#pragma unroll
+          for (int u = 0; u < PULL_DEPTH; ++u)
+            if (i0 + 32 * u < w1) v[u] = s4[i0 + 32 * u];
+#pragma unroll
+          for (int u = 0; u < PULL_DEPTH; ++u)
+            if (i0 + 32 * u < w1) d4[i0 + 32 * u] = v[u];
+        }
+      } else if (lane == 0 && blockIdx.x == 0) {
+        set_err(p.err, MOE_ERR_CAPACITY);
+      }
+      __syncwarp();
+      if (lane == 0) {
+        __threadfence();
+        atomicAdd(p.ready + m, 1);
       }
     }
     return;
@@ -902,6 +1024,8 @@ __global__ void __launch_bounds__(LAYER_THREADS, 1)
   named_bar_sync(BAR_ALL, CW * 32);
   if (M.flag) {   // last block out: re-arm the counters for the next call
     for (int i = tid; i < U; i += CW * 32) p.up_done[i] = 0;
+    if (STG)
+      for (int i = tid; i < M.nmiss; i += CW * 32) p.ready[i] = 0;
     if (tid == 0) {
       p.bar[0] = 0;
       p.bar[1] = 0;
@@ -935,7 +1059,8 @@ moe_status launch_decode_layer(const moe_layer_desc& d, const uint16_t* x,
                                const float* residual, float* out,
                                uint16_t* out_bf16, int32_t* topk_idx,
                                float* topk_w, float* logits, void* ws,
-                               int32_t* err, cudaStream_t s, int mode) {
+                               int32_t* err, cudaStream_t s, int mode,
+                               const StageArgs* stg) {
   LayerParams p;
   p.mode = mode;
   p.pool = d.pool;
@@ -969,14 +1094,26 @@ moe_status launch_decode_layer(const moe_layer_desc& d, const uint16_t* x,
   b += (P * 4 + 255) & ~(size_t)255;
   p.y = reinterpret_cast<float*>(b);
   p.err = err;
+  p.n_miss = stg ? stg->n_miss : nullptr;
+  p.miss_expert = stg ? stg->miss_expert : nullptr;
+  p.miss_slot = stg ? stg->miss_slot : nullptr;
+  p.stage_table = stg ? stg->table : nullptr;
+  p.stage_layer = stg ? stg->layer : 0;
+  p.slot_base = stg ? stg->slot_base : 0;
+  p.n_slots = stg ? stg->n_slots : 0;
+  p.pool_slots = stg ? stg->pool_slots : 0;
+  p.blob_bytes = stg ? stg->blob_bytes : 0;
+  p.ready = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + 512);
   const Smem L = smem_layout(d.fmt_up_gate, d.H, d.F, T);
   void (*kern)(LayerParams) = nullptr;
   const bool q4d = d.fmt_down == MOE_Q4_B32;
   const bool two = T > 4;
   const bool wide = d.E > 512;
+#define MOE_K(FU, FD, NTT, EPLV)                                            \
+  (stg ? decode_layer_kernel<FU, FD, NTT, EPLV, true>                        \
+       : decode_layer_kernel<FU, FD, NTT, EPLV, false>)
 #define MOE_PICK2(FU, FD, NTT)                                               \
-  (wide ? decode_layer_kernel<FU, FD, NTT, 32>                               \
-        : decode_layer_kernel<FU, FD, NTT, 16>)
+  (wide ? MOE_K(FU, FD, NTT, 32) : MOE_K(FU, FD, NTT, 16))
 #define MOE_PICK(FU)                                                        \
   kern = q4d ? (two ? MOE_PICK2(FU, MOE_Q4_B32, 2)                          \
                     : MOE_PICK2(FU, MOE_Q4_B32, 1))                         \
@@ -990,11 +1127,12 @@ moe_status launch_decode_layer(const moe_layer_desc& d, const uint16_t* x,
   }
 #undef MOE_PICK
 #undef MOE_PICK2
+#undef MOE_K
   moe_status st = ensure_smem((const void*)kern, (size_t)L.total);
   if (st != MOE_OK) return st;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(num_sms());
-  cfg.blockDim = dim3(LAYER_THREADS);
+  cfg.blockDim = dim3(stg ? LAYER_THREADS_STG : LAYER_THREADS);
   cfg.dynamicSmemBytes = (size_t)L.total;
   cfg.stream = s;
   cudaLaunchAttribute attr[2];

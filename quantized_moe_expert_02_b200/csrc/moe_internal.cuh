@@ -134,6 +134,18 @@ constexpr int BF_NT = 2;        // N tiles (4 tokens each) of the B layouts
 // a bit of the result.
 constexpr int DL_FULL = 0, DL_ROUTE = 1, DL_FFN = 2;
 
+// In-kernel staging of a slot-cache layer's misses (DL_FFN): the slot
+// resolve's miss list, the host blob table and the layer's partition.
+struct StageArgs {
+  const int32_t* n_miss;
+  const int32_t* miss_expert;
+  const int32_t* miss_slot;
+  const uint64_t* table;
+  int layer;
+  int slot_base, n_slots;
+  int64_t pool_slots, blob_bytes;
+};
+
 struct FfnWs {
   int32_t* err;       // [4]  error word, route counter, spare
   int32_t* up_cnt;    // [P * F/32]   arrival counters, 32-row up tiles

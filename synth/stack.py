@@ -232,8 +232,11 @@ class SlotPool:
         if hasattr(self, "stamps"):
             self.stamps.zero_()
 
-    def layer_staged(self, l: int, r) -> None:
-        """One layer through the slot pool, in place, with no host sync."""
+    def layer_staged(self, l: int, r, fused: bool = False) -> None:
+        """One layer through the slot pool, in place, with no host sync.
+        fused: the pull inside the FFN launch, overlapping the hits'
+        compute (moe_layer_ffn_residual_staged); else the pull kernel
+        (moe_stage_misses), then the FFN."""
         st, moe, shp = self.stack, self.moe, self.stack.shape
         T, k, E = st.T, shp.k, shp.E
         moe.moe_layer_route_residual(self.descs[l], r, T, k, st.wr[l],
@@ -245,6 +248,13 @@ class SlotPool:
                                  self.stamps.data_ptr() + 4 * l,
                                  self.blob_index, self.mexp, self.mslot,
                                  self.nmiss, self.err)
+        if fused:
+            moe.moe_layer_ffn_residual_staged(
+                self.descs[l], r, T, k, st.idx, st.w, self.blob_index, r,
+                None, self.nmiss, self.mexp, self.mslot, l, len(self.caps),
+                self.table_dev, int(self.base[l]), self.caps[l],
+                self.n_slots, st.ws, st.ws_bytes)
+            return
         moe.moe_stage_misses(self.nmiss, self.mexp, self.mslot, T * k, l,
                              len(self.caps), E, self.table_dev, self.pool,
                              int(self.base[l]), self.caps[l], self.n_slots,
@@ -253,13 +263,13 @@ class SlotPool:
                                    self.blob_index, r, None, st.ws,
                                    st.ws_bytes)
 
-    def run_staged(self, r):
+    def run_staged(self, r, fused: bool = False):
         """One step: every layer in order, in place on r."""
         for l in range(len(self.caps)):
-            self.layer_staged(l, r)
+            self.layer_staged(l, r, fused)
         return r
 
-    def capture_step(self, x_in, r):
+    def capture_step(self, x_in, r, fused: bool = False):
         """The whole step -- r <- x_in, then route, resolve, pull and FFN of
         every layer -- captured once as one CUDA graph; each replay runs
         the next step (the slot state and the stamp counters live on the
@@ -267,5 +277,5 @@ class SlotPool:
         g = self.torch.cuda.CUDAGraph()
         with self.torch.cuda.graph(g):
             r.copy_(x_in)
-            self.run_staged(r)
+            self.run_staged(r, fused)
         return g

@@ -86,3 +86,29 @@ def test_stage_argument_errors_without_gpu():
     # an unaligned host address is refused before it is looked up
     table[0] = f + 4
     assert lib.moe_stage_table(table, 1, f, None) == moe.MOE_ERR_INVALID
+
+
+def test_staged_ffn_argument_errors_without_gpu():
+    """moe_layer_ffn_residual_staged rejects bad arguments on the host."""
+    f = 4096
+    lib = moe.lib
+    desc = moe.moe_layer_desc(H=3072, F=1024, E=512,
+                              fmt_up_gate=moe.MOE_SB3_256,
+                              fmt_down=moe.MOE_NL4_B32, pool=f,
+                              blob_stride=4276224)
+    ws_b = moe.moe_layer_workspace_bytes(3, 10, 512, 3072, 1024)
+
+    def call(**kw):
+        a = dict(n_miss=f, table=f, layer=0, L=48, slot_base=0, n_slots=60,
+                 pool_slots=4644, ws=f, ws_bytes=ws_b)
+        a.update(kw)
+        return lib.moe_layer_ffn_residual_staged(
+            ctypes.addressof(desc), f, 3, 10, f, f, f, f, None, a["n_miss"],
+            f, f, a["layer"], a["L"], a["table"], a["slot_base"],
+            a["n_slots"], a["pool_slots"], a["ws"], a["ws_bytes"], None)
+
+    assert call(n_miss=None) == moe.MOE_ERR_INVALID
+    assert call(table=None) == moe.MOE_ERR_INVALID
+    assert call(layer=48) == moe.MOE_ERR_SHAPE
+    assert call(slot_base=4600, n_slots=60) == moe.MOE_ERR_SHAPE
+    assert call(ws_bytes=16) == moe.MOE_ERR_WORKSPACE

@@ -66,3 +66,51 @@ def test_layer_grid_barrier_timeout_is_reported_and_recovers():
     assert torch.equal(out, ref)
     del pool
     torch.cuda.empty_cache()
+
+
+def test_staged_pull_wait_timeout_is_reported_and_recovers():
+    """The wait of the staged FFN (moe_layer_ffn_residual_staged) for a
+    missed expert's blob: its ready counter is planted with a value that the
+    blocks' arrivals cannot bring up to the grid size, so the producers'
+    bounded waits run out -- MOE_ERR_TIMEOUT, counters re-armed, and the
+    pulls themselves complete: the plain FFN half on the same routing then
+    gives the resident result bit for bit."""
+    from synth.stack import SlotPool, Stack
+    shape = synth.BIG
+    T, k, E, H, F = 3, shape.k, shape.E, shape.H, shape.F
+    st = Stack(1, shape, seed=0, T=T)
+    ref = st.run_resident(st.x0(0)).clone()
+    # the first step's misses with a 32-slot partition
+    disc = SlotPool(st, [32], None)
+    disc.run(st.x0(0), 1)
+    keys = sorted(disc.seen_keys)
+    del disc
+    assert keys
+    pool = SlotPool(st, [32], keys)
+    pool.start_staging()
+    r = st.x0(0)
+    r_in = r.clone()
+    moe.moe_layer_route_residual(pool.descs[0], r, T, k, st.wr[0], st.bias[0],
+                                 st.idx, st.w, None, st.ws, st.ws_bytes)
+    moe.moe_slot_resolve_dev(st.idx, T, k, E, pool.table[0], pool.owner[0],
+                             pool.last[0], 32, 0, pool.stamps.data_ptr(),
+                             pool.blob_index, pool.mexp, pool.mslot,
+                             pool.nmiss, pool.err)
+    assert int(pool.nmiss.item()) > 0
+    off = fused_offset(T, k, E, H, F)
+    ready = st.ws[off + 512:off + 516].view(torch.int32)
+    assert int(ready.item()) == 0
+    ready[0] = -(1 << 30)
+    moe.moe_layer_ffn_residual_staged(
+        pool.descs[0], r, T, k, st.idx, st.w, pool.blob_index, r, None,
+        pool.nmiss, pool.mexp, pool.mslot, 0, 1, pool.table_dev, 0, 32,
+        pool.n_slots, st.ws, st.ws_bytes)
+    assert moe.moe_get_device_status(st.ws) == moe.MOE_ERR_TIMEOUT
+    assert int(ready.item()) == 0          # re-armed by the last block
+    r2 = r_in.clone()
+    moe.moe_layer_ffn_residual(pool.descs[0], r2, T, k, st.idx, st.w,
+                               pool.blob_index, r2, None, st.ws, st.ws_bytes)
+    assert moe.moe_get_device_status(st.ws) == 0
+    assert torch.equal(r2, ref)
+    del pool, st
+    torch.cuda.empty_cache()

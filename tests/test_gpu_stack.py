@@ -196,6 +196,48 @@ def test_slot_cache_step_as_one_graph_bit_exact():
     del g
 
 
+def test_slot_cache_fused_staging_bit_exact():
+    """The pull inside the FFN launch (moe_layer_ffn_residual_staged: the
+    misses computed last, their blobs copied by every block while the hits
+    compute): bit-identical to the resident run, eagerly and as one graph
+    per step, with the slot state of the separate-pull run."""
+    L, steps, cap = 3, 8, 32
+    st = stack_for(L)
+    resident, routing = [], []
+    for s in range(steps):
+        rec = []
+        resident.append(st.run_resident(st.x0(s), record=rec).clone())
+        routing.append([i.cpu().numpy() for i in rec])
+    expect, keys = _replay_misses(st, routing, L, steps, cap)
+    assert keys
+    fused = SlotPool(st, [cap] * L, sorted(keys))
+    fused.start_staging()
+    for s in range(steps):
+        r = fused.run_staged(st.x0(s), fused=True)
+        assert torch.equal(r, resident[s]), s
+    assert int(fused.err.item()) == 0
+    assert moe.moe_get_device_status(st.ws) == 0
+    ref = SlotPool(st, [cap] * L, sorted(keys))
+    ref.start_staging()
+    for s in range(steps):
+        ref.run_staged(st.x0(s))
+    for l in range(L):
+        assert torch.equal(fused.table[l], ref.table[l])
+        assert torch.equal(fused.last[l], ref.last[l])
+    # one graph per step
+    fused.reset()
+    x_in = st.x0(0)
+    r = torch.empty_like(x_in)
+    g = fused.capture_step(x_in, r, fused=True)
+    for s in range(steps):
+        x_in.copy_(st.x0(s))
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(r, resident[s]), s
+    assert moe.moe_get_device_status(st.ws) == 0
+    del g
+
+
 def test_slot_cache_full_capacities_48_layers():
     """The slot-cache workload at its real shape: 48 layers, 240 / 92 / 60
     slots per layer, Zipf-hot initial fill, 3 tokens per step.  Misses
@@ -235,6 +277,17 @@ def test_slot_cache_full_capacities_48_layers():
     x_in = st.x0(0)
     r = torch.empty_like(x_in)
     g = pool.capture_step(x_in, r)
+    for s in range(steps):
+        x_in.copy_(st.x0(s))
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(r, resident[s]), s
+    assert int(pool.err.item()) == 0
+    assert moe.moe_get_device_status(st.ws) == 0
+    del g
+    # the same with the pulls inside the FFN launches
+    pool.reset()
+    g = pool.capture_step(x_in, r, fused=True)
     for s in range(steps):
         x_in.copy_(st.x0(s))
         g.replay()
