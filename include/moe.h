@@ -368,6 +368,20 @@ moe_status moe_expert_down_q(const moe_layer_desc* desc, int T, int k,
                              float* out, uint16_t* out_bf16, void* ws,
                              size_t ws_bytes, void* stream);
 
+/* The prefill path's up/gate GEMM launch alone (T > 8, H and F multiples
+ * of 128; else MOE_ERR_UNSUPPORTED): it recomputes h from the grouped fp16
+ * activations, row scales and unit plan that a moe_expert_up_q call with
+ * the same arguments and workspace staged, reading nothing else of x.  A
+ * measurement hook: it times the tensor-core kernel without the activation
+ * pass in front of it.  Same result as that moe_expert_up_q call. */
+moe_status moe_expert_up_gemm_q(const moe_layer_desc* desc, int T, int k,
+                                const int32_t* expert_offsets,
+                                const int32_t* pair_ids,
+                                const int32_t* active,
+                                const int32_t* n_active,
+                                const int32_t* blob_index, void* ws,
+                                size_t ws_bytes, void* stream);
+
 /* Weighted combine: out[t] = sum_j topk_w[t,j] * y_pairs[t*k+j]
  * (+ residual[t]), summed in j order.  out fp32 [T x H]; out_bf16 bf16
  * [T x H] or NULL; residual fp32 [T x H] or NULL (may alias out). */

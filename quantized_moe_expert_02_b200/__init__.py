@@ -70,6 +70,8 @@ _SIGS = {
                                  _P, _P, c_size_t, _P]),
     "moe_expert_up_q": (c_int, [_P, _P, c_int, c_int, _P, _P, _P, _P, _P,
                                 _P, c_size_t, _P]),
+    "moe_expert_up_gemm_q": (c_int, [_P, c_int, c_int, _P, _P, _P, _P, _P,
+                                     _P, c_size_t, _P]),
     "moe_expert_down_q": (c_int, [_P, c_int, c_int, _P, _P, _P, _P, _P, _P,
                                   _P, _P, _P, _P, _P, c_size_t, _P]),
     "moe_combine": (c_int, [_P, _P, c_int, c_int, c_int, _P, _P, _P, _P]),
@@ -252,6 +254,14 @@ def moe_expert_up_q(desc, x, T, k, expert_offsets, pair_ids, active,
     _check("moe_expert_up_q", lib.moe_expert_up_q(
         _ptr(desc), _ptr(x), T, k, _ptr(expert_offsets), _ptr(pair_ids),
         _ptr(active), _ptr(n_active), _ptr(blob_index), _ptr(ws), ws_bytes,
+        _stream(stream)))
+
+
+def moe_expert_up_gemm_q(desc, T, k, expert_offsets, pair_ids, active,
+                         n_active, blob_index, ws, ws_bytes, stream=None):
+    _check("moe_expert_up_gemm_q", lib.moe_expert_up_gemm_q(
+        _ptr(desc), T, k, _ptr(expert_offsets), _ptr(pair_ids), _ptr(active),
+        _ptr(n_active), _ptr(blob_index), _ptr(ws), ws_bytes,
         _stream(stream)))
 
 

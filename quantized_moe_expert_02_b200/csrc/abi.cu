@@ -49,6 +49,10 @@ moe_status launch_pf_up(const moe_layer_desc& d, const uint16_t* x, int T,
                         int k, const int32_t* offsets,
                         const int32_t* pair_ids, const int32_t* blob_index,
                         const FfnWs& w, cudaStream_t s);
+moe_status launch_pf_up_gemm(const moe_layer_desc& d, int T, int k,
+                             const int32_t* pair_ids,
+                             const int32_t* blob_index, const FfnWs& w,
+                             cudaStream_t s);
 moe_status launch_pf_down(const moe_layer_desc& d, int T, int k,
                           const int32_t* pair_ids, const int32_t* blob_index,
                           const FfnWs& w, float* y, cudaStream_t s);
@@ -360,6 +364,20 @@ extern "C" moe_status moe_expert_up_q(
   const FfnWs w = carve_ffn_ws(ws, T, k, desc->H, desc->F);
   return run_up(*desc, x, T, k, expert_offsets, pair_ids, active, n_active,
                 blob_index, w, (cudaStream_t)stream, false);
+}
+
+extern "C" moe_status moe_expert_up_gemm_q(
+    const moe_layer_desc* desc, int T, int k, const int32_t* expert_offsets,
+    const int32_t* pair_ids, const int32_t* active, const int32_t* n_active,
+    const int32_t* blob_index, void* ws, size_t ws_bytes, void* stream) {
+  moe_status st = check_ffn_args(desc, T, k, expert_offsets, pair_ids, active,
+                                 n_active, ws, ws_bytes);
+  if (st != MOE_OK) return st;
+  if (ffn_decode_supported(*desc, T, k) || !pf_supported(*desc, T))
+    return MOE_ERR_UNSUPPORTED;
+  const FfnWs w = carve_ffn_ws(ws, T, k, desc->H, desc->F);
+  return launch_pf_up_gemm(*desc, T, k, pair_ids, blob_index, w,
+                           (cudaStream_t)stream);
 }
 
 extern "C" moe_status moe_expert_down_q(

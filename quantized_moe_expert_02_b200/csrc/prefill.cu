@@ -1029,21 +1029,15 @@ static moe_status pf_launch_fmt(int fmt, const PfParams& prm,
   }
 }
 
-moe_status launch_pf_up(const moe_layer_desc& d, const uint16_t* x, int T,
-                        int k, const int32_t* offsets,
-                        const int32_t* pair_ids, const int32_t* blob_index,
-                        const FfnWs& w, cudaStream_t s) {
+// The up/gate GEMM launch alone, on the grouped activations, row scales
+// and unit plan that launch_pf_up staged in the workspace.
+moe_status launch_pf_up_gemm(const moe_layer_desc& d, int T, int k,
+                             const int32_t* pair_ids,
+                             const int32_t* blob_index, const FfnWs& w,
+                             cudaStream_t s) {
   const int64_t P = (int64_t)T * k;
   PfMaps map;
   moe_status st = encode_maps(&map, w.x16, (uint64_t)d.H, (uint64_t)P);
-  if (st != MOE_OK) return st;
-  pf_fill_kernel<<<(unsigned)((P + 255) / 256), 256, 0, s>>>(w.inv, (int)P,
-                                                            -1);
-  pf_inv_kernel<<<(unsigned)((P + 255) / 256), 256, 0, s>>>(
-      pair_ids, offsets, d.E, (int)P, w.inv);
-  pf_xg_kernel<<<T, 256, 0, s>>>(x, d.H, k, w.inv, w.x16, w.xscale);
-  pf_plan_kernel<<<1, 1024, 0, s>>>(offsets, d.E, w.tiles, w.n_tiles);
-  st = launch_status();
   if (st != MOE_OK) return st;
   PfParams prm{};
   prm.pool = d.pool;
@@ -1062,6 +1056,22 @@ moe_status launch_pf_up(const moe_layer_desc& d, const uint16_t* x, int T,
   prm.err = w.err;
   pf_tables(d.fmt_up_gate, prm.tab);
   return pf_launch_fmt<true>(d.fmt_up_gate, prm, map, s);
+}
+
+moe_status launch_pf_up(const moe_layer_desc& d, const uint16_t* x, int T,
+                        int k, const int32_t* offsets,
+                        const int32_t* pair_ids, const int32_t* blob_index,
+                        const FfnWs& w, cudaStream_t s) {
+  const int64_t P = (int64_t)T * k;
+  pf_fill_kernel<<<(unsigned)((P + 255) / 256), 256, 0, s>>>(w.inv, (int)P,
+                                                            -1);
+  pf_inv_kernel<<<(unsigned)((P + 255) / 256), 256, 0, s>>>(
+      pair_ids, offsets, d.E, (int)P, w.inv);
+  pf_xg_kernel<<<T, 256, 0, s>>>(x, d.H, k, w.inv, w.x16, w.xscale);
+  pf_plan_kernel<<<1, 1024, 0, s>>>(offsets, d.E, w.tiles, w.n_tiles);
+  const moe_status st = launch_status();
+  if (st != MOE_OK) return st;
+  return launch_pf_up_gemm(d, T, k, pair_ids, blob_index, w, s);
 }
 
 moe_status launch_pf_down(const moe_layer_desc& d, int T, int k,

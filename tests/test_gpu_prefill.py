@@ -156,6 +156,19 @@ def test_up_then_down_matches_ffn():
                           None, None, None, None, ws.t, ws.nbytes)
     torch.cuda.synchronize()
     assert torch.equal(y1, y2)
+    # the up/gate GEMM launch alone, on the activations staged above
+    y3 = torch.full_like(y1, float("nan"))
+    moe.moe_expert_up_gemm_q(desc, T, shape.k, off, pairs, act, na, None,
+                             ws.t, ws.nbytes)
+    moe.moe_expert_down_q(desc, T, shape.k, off, pairs, act, na, None, y3,
+                          None, None, None, None, ws.t, ws.nbytes)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y3)
+    # decode shapes have no separate GEMM launch
+    with pytest.raises(moe.MoeError) as ei:
+        moe.moe_expert_up_gemm_q(desc, 4, shape.k, off, pairs, act, na, None,
+                                 ws.t, ws.nbytes)
+    assert ei.value.code == moe.MOE_ERR_UNSUPPORTED
 
 
 def test_prefill_bad_blob_index_sets_error_word():
