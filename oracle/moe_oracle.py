@@ -33,6 +33,9 @@ design notes; the ones that shape arithmetic here are:
     below and one shift bit e per 32 weights (this repository's own 3-bit
     non-uniform format; the model card lists such a type, IQ3_K, by name
     and bit rate only).
+  * SB2 value: w = d * (2s+1) * c / 4 with c = 2q - 3 (q the 2-bit code;
+    this repository's 2-bit super-block format, a stand-in for the 2-bit
+    up/gate type, IQ2_S, that the model card names without its layout).
   * Q4 value:  w = d * (q - 8).
   * Stacked decode layers use the pre-norm residual r <- r + MoE(x),
     x = bf16(rmsnorm(r)), rmsnorm without a learned weight, eps = 1e-6.
@@ -46,7 +49,7 @@ from typing import Callable, Dict, List, Optional, Sequence, Tuple
 
 import numpy as np
 
-Q4_B32, SB3_256, NL4_B32, NL3_256 = 1, 2, 3, 4
+Q4_B32, SB3_256, NL4_B32, NL3_256, SB2_256 = 1, 2, 3, 4, 5
 
 # 16-entry non-uniform codebook of the 4-bit NL format (ascending).
 NL4_CODEBOOK = np.array([-127, -104, -83, -65, -49, -35, -22, -10,
@@ -98,6 +101,10 @@ def tensor_plane_sizes(fmt: int, rows: int, cols: int) -> List[int]:
         assert cols % 256 == 0
         n = rows * cols // 256
         return [96 * n, 4 * n, 2 * n, n]
+    if fmt == SB2_256:
+        assert cols % 256 == 0
+        n = rows * cols // 256
+        return [64 * n, 4 * n, 2 * n]
     assert fmt in (Q4_B32, NL4_B32) and cols % 32 == 0
     n = rows * cols // 32
     return [16 * n, 2 * n]
@@ -161,6 +168,33 @@ def dequant_nl3(raw: np.ndarray, rows: int, cols: int) -> np.ndarray:
     return w.reshape(rows, cols)
 
 
+def dequant_sb2(raw: np.ndarray, rows: int, cols: int) -> np.ndarray:
+    """2-bit super-block format -> float64 [rows, cols].
+
+    A super-block of 256 weights has a fp16 scale d, eight 4-bit sub-scales
+    s_j (one per 32 weights, in a little-endian 32-bit word as in SB3) and
+    256 2-bit codes q, code i at bits 2i, 2i+1 of its 64-byte stream.
+    Weight i of the super-block is
+        w_i = d * (2*s_{i//32} + 1) * (2*q_i - 3) / 4.
+    """
+    n_codes, n_sc, n_d = tensor_plane_sizes(SB2_256, rows, cols)
+    raw = np.asarray(raw, dtype=np.uint8)
+    codes = raw[:n_codes]
+    scales = raw[n_codes:n_codes + n_sc]
+    dbits = raw[n_codes + n_sc:n_codes + n_sc + n_d]
+    nsb = rows * cols // 256
+    bits = _bits_le(codes, 64).reshape(nsb, 256, 2)
+    q = bits[:, :, 0] | (bits[:, :, 1] << 1)
+    sbits = _bits_le(scales, 4).reshape(nsb, 8, 4)
+    s = (sbits[:, :, 0] | (sbits[:, :, 1] << 1) | (sbits[:, :, 2] << 2) |
+         (sbits[:, :, 3] << 3))                                      # [nsb,8]
+    d = fp16_to_f64(dbits)                                           # [nsb]
+    sub = np.repeat(2.0 * s.astype(np.float64) + 1.0, 32, axis=1)    # [nsb,256]
+    c = 2.0 * q.astype(np.float64) - 3.0
+    w = d[:, None] * sub * c / 4.0
+    return w.reshape(rows, cols)
+
+
 def _nibbles(codes: np.ndarray) -> np.ndarray:
     """Codes plane -> one 4-bit code per weight (low nibble first)."""
     b = np.asarray(codes, dtype=np.uint8)
@@ -195,6 +229,8 @@ def dequant(fmt: int, raw: np.ndarray, rows: int, cols: int) -> np.ndarray:
         return dequant_sb3(raw, rows, cols)
     if fmt == NL3_256:
         return dequant_nl3(raw, rows, cols)
+    if fmt == SB2_256:
+        return dequant_sb2(raw, rows, cols)
     return dequant_b32(fmt, raw, rows, cols)
 
 

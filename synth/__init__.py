@@ -32,9 +32,10 @@ Q4_B32 = 1    # 4-bit codes, 32 weights per block, fp16 scale: w = d*(q-8)
 SB3_256 = 2   # 3-bit codes, 256-weight super-block, 8 4-bit sub-scales
 NL4_B32 = 3   # 4-bit codes into a 16-entry int8 codebook, fp16 scale
 NL3_256 = 4   # 3-bit codes into an 8-entry codebook, 256-weight super-block
+SB2_256 = 5   # 2-bit codes, 256-weight super-block, 8 4-bit sub-scales
 
 FMT_NAMES = {Q4_B32: "q4_b32", SB3_256: "sb3_256", NL4_B32: "nl4_b32",
-             NL3_256: "nl3_256"}
+             NL3_256: "nl3_256", SB2_256: "sb2_256"}
 
 BLOB_ALIGN = 4096  # expert blobs start on 4 KiB boundaries
 
@@ -50,14 +51,17 @@ def tensor_planes(fmt: int, rows: int, cols: int) -> List[Tuple[str, int]]:
                d       rows*(cols/256) fp16.
       NL3_256: the three SB3 planes, then
                extra   rows*(cols/256) B (bit j = codebook shift of 32-block j).
+      SB2_256: codes   rows*cols/4 B (64 B per super-block, code i at bits
+                       2*(i%4) of byte i/4), then scales and d as SB3.
       Q4_B32 / NL4_B32: codes rows*cols/2 B (weight i of a row in byte i/2,
                        low nibble for even i), d rows*(cols/32) fp16.
     """
-    if fmt in (SB3_256, NL3_256):
+    if fmt in (SB3_256, NL3_256, SB2_256):
         if cols % 256:
             raise ValueError("super-block formats need cols % 256 == 0")
         nsb = rows * (cols // 256)
-        planes = [("codes", nsb * 96), ("scales", nsb * 4), ("d", nsb * 2)]
+        cb = 64 if fmt == SB2_256 else 96
+        planes = [("codes", nsb * cb), ("scales", nsb * 4), ("d", nsb * 2)]
         if fmt == NL3_256:
             planes.append(("extra", nsb))
         return planes
@@ -118,6 +122,11 @@ BIG = LayerShape(H=3072, F=1024, E=512, k=10, fmt_up_gate=SB3_256,
 # The decode layer shape with up/gate in the 3-bit non-uniform-codebook
 # format (64 experts, top-8: a smaller pool for the format's parity tests).
 NL3_SHAPE = LayerShape(H=3072, F=1024, E=64, k=8, fmt_up_gate=NL3_256,
+                       fmt_down=NL4_B32, d_up_gate=(0.002, 0.01),
+                       d_down=(0.002, 0.01))
+
+# The same decode shape with up/gate in the 2-bit super-block format.
+SB2_SHAPE = LayerShape(H=3072, F=1024, E=64, k=8, fmt_up_gate=SB2_256,
                        fmt_down=NL4_B32, d_up_gate=(0.002, 0.01),
                        d_down=(0.002, 0.01))
 

@@ -104,13 +104,15 @@ TensorSpec make_spec(int fmt, int rows, int cols, int tensor_id, double lo,
   s.tensor_id = tensor_id;
   s.lo = lo;
   s.hi = hi;
-  if (fmt == 2 || fmt == 4) {  // SB3, NL3 (+ one shift byte per block)
+  if (fmt == 2 || fmt == 4 || fmt == 5) {
+    // SB3, NL3 (+ one shift byte per block), SB2 (64 code bytes per block)
     const int64_t nsb = (int64_t)rows * (cols / 256);
-    s.planes[0] = {0, nsb * 96, 0};
-    s.planes[1] = {nsb * 96, nsb * 4, 1};
-    s.planes[2] = {nsb * 100, nsb * 2, 2};
+    const int64_t cb = fmt == 5 ? 64 : 96;
+    s.planes[0] = {0, nsb * cb, 0};
+    s.planes[1] = {nsb * cb, nsb * 4, 1};
+    s.planes[2] = {nsb * (cb + 4), nsb * 2, 2};
     s.nplanes = 3;
-    s.bytes = nsb * 102;
+    s.bytes = nsb * (cb + 6);
     if (fmt == 4) {
       s.planes[3] = {nsb * 102, nsb, 3};
       s.nplanes = 4;

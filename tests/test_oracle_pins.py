@@ -110,6 +110,76 @@ def test_sb3_bit_positions_are_a_bijection():
     assert np.all(seen.sum(1) == 3)
 
 
+def test_sb2_hand_worked_superblock():
+    meta, rows = _read_golden("sb2_superblock.txt")
+    raw = np.frombuffer(meta["codes_hex"] + meta["scales_hex"] + meta["d_hex"],
+                        np.uint8)
+    assert raw.size == 70
+    w = o.dequant_sb2(raw, 1, 256)[0]
+    for i, exp in rows:
+        assert w[int(i)] == exp, (i, w[int(i)], exp)
+
+
+def test_sb2_every_subscale_and_code():
+    # one super-block per (s, q), d = 1: every weight is (2s+1)(2q-3)/4
+    pairs = list(itertools.product(range(16), range(4)))
+    codes = b"".join(_pack_bits([q] * 256, 2) for s, q in pairs)
+    scales = b"".join(_pack_bits([s] * 8, 4) for s, q in pairs)
+    d = np.full(len(pairs), 1.0, np.float16).tobytes()
+    w = o.dequant_sb2(np.frombuffer(codes + scales + d, np.uint8),
+                      len(pairs), 256)
+    for r, (s, q) in enumerate(pairs):
+        assert np.all(w[r] == (2 * s + 1) * (2 * q - 3) / 4.0), (s, q)
+
+
+def test_sb2_bit_positions_and_rows():
+    # Code bit b of weight i is stream bit 2i+b: flipping it from the
+    # all-zero codes raises weight i alone by 2^(b+1) units of d(2s+1)/4;
+    # super-blocks follow one another along a row, then rows.
+    rng = np.random.default_rng(4)
+    s = rng.integers(0, 16, 8)
+    scales = _pack_bits(s, 4)
+    d = np.array([0.25], np.float16).tobytes()
+    base = o.dequant_sb2(np.frombuffer(bytes(64) + scales + d, np.uint8),
+                         1, 256)[0]
+    assert np.all(base == -3 * 0.25 * (2 * np.repeat(s, 32) + 1) / 4.0)
+    for bit in range(512):
+        codes = bytearray(64)
+        codes[bit // 8] |= 1 << (bit % 8)
+        w = o.dequant_sb2(np.frombuffer(bytes(codes) + scales + d, np.uint8),
+                          1, 256)[0]
+        i, b = bit // 2, bit % 2
+        assert np.nonzero(w != base)[0].tolist() == [i]
+        assert w[i] - base[i] == 0.25 * (2 * s[i // 32] + 1) / 4.0 * 2 ** (b + 1)
+    # 2 rows x 512 columns: super-block m = row * 2 + column // 256, its
+    # codes, scale word and d in plane order
+    q = rng.integers(0, 4, (4, 256))
+    sc = rng.integers(0, 16, (4, 8))
+    dd = np.array([0.5, 0.25, 1.0, 2.0], np.float16)
+    raw = np.frombuffer(b"".join(_pack_bits(r, 2) for r in q) +
+                        b"".join(_pack_bits(r, 4) for r in sc) +
+                        dd.tobytes(), np.uint8)
+    w = o.dequant_sb2(raw, 2, 512)
+    for m in range(4):
+        want = (dd[m].astype(np.float64) * (2 * np.repeat(sc[m], 32) + 1) *
+                (2 * q[m] - 3) / 4.0)
+        assert np.array_equal(w[m // 2, 256 * (m % 2):256 * (m % 2) + 256],
+                              want)
+
+
+def test_sb2_generated_planes_and_range():
+    raw = synth.gen_tensor(0, 0, 0, "up", synth.SB2_256, 16, 512,
+                           (0.002, 0.01))
+    assert raw.size == 16 * 2 * 70
+    w = o.dequant_sb2(raw, 16, 512)
+    assert np.abs(w).max() <= 0.01 * 31 * 3 / 4 + 1e-12
+    assert np.array_equal(w.astype(np.float32).astype(np.float64), w)
+    # all four codes occur in the codes plane
+    cb = raw[:16 * 2 * 64]
+    assert {int(v) for k in range(4) for v in np.unique((cb >> 2 * k) & 3)} \
+        == {0, 1, 2, 3}
+
+
 def test_nl3_hand_worked_superblock():
     meta, rows = _read_golden("nl3_superblock.txt")
     raw = np.frombuffer(meta["codes_hex"] + meta["scales_hex"] +
