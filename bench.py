@@ -556,15 +556,20 @@ def clock_soak(lay, T: int, ms_per_step: float, seconds: float = 1.0):
     return out
 
 
-def nl3_decode(T: int, K: int, W: int) -> dict:
-    """The decode layer with up/gate in the 3-bit non-uniform-codebook
-    format (NL3) at the 512-expert shape: two resident layers rotated."""
+ALT_UP_GATE = {"nl3": (synth.NL3_256, "NL3"), "sb2": (synth.SB2_256, "SB2")}
+
+
+def alt_decode(T: int, K: int, W: int, which: str) -> dict:
+    """The decode layer with up/gate in another format -- the 3-bit
+    non-uniform-codebook super-block (NL3) or the 2-bit super-block (SB2) --
+    at the 512-expert shape: two resident layers rotated."""
     import torch
-    shape = dataclasses.replace(synth.BIG, fmt_up_gate=synth.NL3_256)
+    fmt, name = ALT_UP_GATE[which]
+    shape = dataclasses.replace(synth.BIG, fmt_up_gate=fmt)
     lay = Layers(2, shape=shape)
     d, _ = decode_measure(lay, T, K, W)
     d["workload"] = (f"decode, one MoE layer: {T} tokens, 512 experts "
-                     "top-10, NL3 up/gate + NL4 down")
+                     f"top-10, {name} up/gate + NL4 down")
     d["blob_bytes"] = shape.blob_bytes
     del lay
     torch.cuda.empty_cache()
@@ -865,7 +870,8 @@ def run_ours(args) -> None:
                 line["prefill"]["through_slots"] = prefill_slots_measure(
                     lay.pools[0])
         if world == 1 and not args.no_extras:
-            line["decode_nl3"] = nl3_decode(T, 4096, W)
+            line["decode_nl3"] = alt_decode(T, 4096, W, "nl3")
+            line["decode_sb2"] = alt_decode(T, 4096, W, "sb2")
         if not args.no_cpu_baseline and world == 1:
             line["cpu_baseline"] = cpu_baseline(T)
             line["speedup_vs_cpu_baseline"] = \
@@ -1249,7 +1255,7 @@ def main():
     ap.add_argument("--store-gb", type=float, default=24.0,
                     help="stack: pinned host store limit for slot misses")
     ap.add_argument("--no-extras", action="store_true",
-                    help="skip the NL3 decode and 48-layer stack objects "
+                    help="skip the NL3 / SB2 decode and 48-layer stack objects "
                          "of the default line")
     ap.add_argument("--stack-steps", type=int, default=16,
                     help="steps of the default line's compact stack object")

@@ -68,19 +68,29 @@ typedef enum {
  *               "K" type the model card lists for up/gate (IQ3_K,
  *               3.44 bpw): the card gives only its name and bit rate, so
  *               neither this layout nor this codebook follows that type.
+ *  MOE_SB2_256: 256-weight super-block, fp16 scale d, eight 4-bit
+ *               sub-scales s_j (one per 32 weights), 2-bit codes q,
+ *               w = d * (2*s_j + 1) * (2*q - 3) / 4.          (2.19 bpw)
+ *               This library's own stand-in for the 2-bit type the model
+ *               card lists for up/gate (IQ2_S): the card gives only its
+ *               name, so the layout and values are this library's.
  * Natural byte layout of a [rows x cols] tensor (rows of blocks along the
- * columns, planar): codes plane, then (SB3, NL3) sub-scale plane, then the
- * fp16 d plane.  SB3 codes: 96 bytes per super-block, a little-endian bit
- * stream with code i at bit 3i; sub-scale j at bit 4j of a little-endian
- * 32-bit word.  NL3: the SB3 planes (codes, sub-scale words, d), then a
- * plane of one byte per super-block whose bit j is e_j.  Q4/NL4 codes:
- * weight i of a row in byte i/2, low nibble for even i.  The *packed* layout (same byte count) is the GPU tile layout
- * that moe_pack_tensor produces and every compute entry point reads. */
+ * columns, planar): codes plane, then (SB3, NL3, SB2) sub-scale plane,
+ * then the fp16 d plane.  SB3 codes: 96 bytes per super-block, a
+ * little-endian bit stream with code i at bit 3i; sub-scale j at bit 4j of
+ * a little-endian 32-bit word.  NL3: the SB3 planes (codes, sub-scale
+ * words, d), then a plane of one byte per super-block whose bit j is e_j.
+ * SB2: codes 64 bytes per super-block, code i at bit 2i, then sub-scale
+ * words and d as in SB3.  Q4/NL4 codes: weight i of a row in byte i/2, low
+ * nibble for even i.  The *packed* layout (same byte count) is the GPU
+ * tile layout that moe_pack_tensor produces and every compute entry point
+ * reads. */
 typedef enum {
   MOE_Q4_B32 = 1,
   MOE_SB3_256 = 2,
   MOE_NL4_B32 = 3,
-  MOE_NL3_256 = 4
+  MOE_NL3_256 = 4,
+  MOE_SB2_256 = 5
 } moe_qfmt;
 
 /* One MoE layer's experts as the FFN sees them.
@@ -111,7 +121,7 @@ size_t moe_blob_bytes(int fmt_up_gate, int fmt_down, int H, int F);
 /* Natural layout -> packed GPU tile layout (model card, "Files": the expert
  * quant types; the packed layout is this library's own).  `natural` and
  * `packed` are distinct device buffers of moe_tensor_bytes() bytes.
- * Needs rows % 16 == 0, cols % 256 == 0 (SB3, NL3) or cols % 64 == 0
+ * Needs rows % 16 == 0, cols % 256 == 0 (SB3, NL3, SB2) or cols % 64 == 0
  * (Q4/NL4). */
 moe_status moe_pack_tensor(int fmt, const uint8_t* natural, int rows,
                            int cols, uint8_t* packed, void* stream);
@@ -320,7 +330,7 @@ moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream);
  *   expert_offsets/pair_ids/active/n_active: moe_group_tokens' outputs
  *   blob_index int32 [E] or NULL (NULL: expert e's blob is blob e); a
  *              negative entry of a chosen expert sets MOE_ERR_DEVICE
- * Needs H, F multiples of 256 (SB3, NL3) or 64 (Q4/NL4) and of 16.
+ * Needs H, F multiples of 256 (SB3, NL3, SB2) or 64 (Q4/NL4) and of 16.
  * T <= 8: int8 tensor-core decode kernels.  The weights enter exactly
  *   (int8 codes, integer sub-scale folds, fp32 scales); the activations
  *   are rounded to 15-bit fixed point with one power-of-two scale per

@@ -29,6 +29,8 @@ MOE_ERR_WORKSPACE = 8
 MOE_Q4_B32 = 1
 MOE_SB3_256 = 2
 MOE_NL4_B32 = 3
+MOE_NL3_256 = 4
+MOE_SB2_256 = 5
 
 MOE_DQ_DECODE = 1
 MOE_DQ_PREFILL = 2

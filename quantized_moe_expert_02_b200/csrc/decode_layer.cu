@@ -122,11 +122,9 @@ __host__ __device__ inline int red_up_floats(int NT) {
 __host__ __device__ inline int red_dn_floats(int NT) {
   return DNW * 32 * NT * 2;
 }
-__host__ __device__ inline Smem smem_layout(int fmt_ug, int H, int F, int T) {
+__host__ __device__ inline Smem smem_layout_slot(int slot, int H, int F,
+                                                 int T) {
   Smem L;
-  const int up = 2 * (H / tile_cols(fmt_ug)) * tile_bytes(fmt_ug);
-  const int dn = dn_unit_bytes(F);
-  int slot = up > dn ? up : dn;
   slot = (slot + 127) / 128 * 128;
   const int NT = (T + 3) / 4;
   const int xfrag = (H / 32) * NT * 64 * 4;
@@ -142,6 +140,17 @@ __host__ __device__ inline Smem smem_layout(int fmt_ug, int H, int F, int T) {
   L.xsc = L.misc + 3072;
   L.total = L.xsc + ((H + XB_COLS - 1) / XB_COLS) * DEC_TMAX * 8;
   return L;
+}
+// A ring slot holds one up unit (up and gate row tiles) or up to DNG down
+// units: it is sized for DNG down units where that fits, so that a format
+// with small up tiles (SB2) keeps the down phase's copies as deep as SB3.
+__host__ __device__ inline Smem smem_layout(int fmt_ug, int H, int F, int T) {
+  const int up = 2 * (H / tile_cols(fmt_ug)) * tile_bytes(fmt_ug);
+  const int dn = dn_unit_bytes(F);
+  const int base = up > dn ? up : dn;
+  const int deep = base > DNG * dn ? base : DNG * dn;
+  const Smem L = smem_layout_slot(deep, H, F, T);
+  return L.total <= 227 * 1024 ? L : smem_layout_slot(base, H, F, T);
 }
 
 // Small shared state (at the misc offset).
@@ -268,10 +277,12 @@ __global__ void __launch_bounds__(STG ? LAYER_THREADS_STG : LAYER_THREADS, 1)
   constexpr int NT = NTT;            // N tiles of 4 tokens: T <= 4 * NT
   constexpr int TM = 4 * NTT;
   const int G = gridDim.x;
-  constexpr bool SBU = FUG == MOE_SB3_256 || FUG == MOE_NL3_256;
+  constexpr bool SBU = FUG == MOE_SB3_256 || FUG == MOE_NL3_256 ||
+                      FUG == MOE_SB2_256;
   constexpr int TCU = SBU ? SB3_TILE_COLS : B32_TILE_COLS;
   constexpr int TBU = FUG == MOE_SB3_256   ? SB3_TILE_BYTES
                       : FUG == MOE_NL3_256 ? NL3_TILE_BYTES
+                      : FUG == MOE_SB2_256 ? SB2_TILE_BYTES
                                            : B32_TILE_BYTES;
   const int nk = H / TCU;                      // up tiles per row tile
   const int nkd = F / B32_TILE_COLS;           // down tiles per row tile
@@ -872,8 +883,8 @@ __global__ void __launch_bounds__(STG ? LAYER_THREADS_STG : LAYER_THREADS, 1)
         const float* xb = xsc + (kt * TCU / XB_COLS) * DEC_TMAX;
         if (SBU) {
           const float xs2[2] = {xb[c], xb[4 + c]};
-          if (tz == 0) piece_sbx<FUG == MOE_NL3_256>(tp, xf, NT, xs2, au, lane, NT);
-          else piece_sbx<FUG == MOE_NL3_256>(tp, xf, NT, xs2, ag, lane, NT);
+          if (tz == 0) piece_sbx<FUG>(tp, xf, NT, xs2, au, lane, NT);
+          else piece_sbx<FUG>(tp, xf, NT, xs2, ag, lane, NT);
         } else {
           if (tz == 0) piece_b32<FUG>(tp, xf, NT, xb + c, 0, au, lane, NT);
           else piece_b32<FUG>(tp, xf, NT, xb + c, 0, ag, lane, NT);
@@ -1122,6 +1133,7 @@ moe_status launch_decode_layer(const moe_layer_desc& d, const uint16_t* x,
   switch (d.fmt_up_gate) {
     case MOE_SB3_256: MOE_PICK(MOE_SB3_256); break;
     case MOE_NL3_256: MOE_PICK(MOE_NL3_256); break;
+    case MOE_SB2_256: MOE_PICK(MOE_SB2_256); break;
     case MOE_NL4_B32: MOE_PICK(MOE_NL4_B32); break;
     default: MOE_PICK(MOE_Q4_B32);
   }

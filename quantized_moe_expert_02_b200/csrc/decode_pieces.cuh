@@ -14,21 +14,27 @@ namespace moe {
 // [blk][bnt][32][2] words; xs[nt] = 2^-sigma_t / 8 of the lane's token.
 // NL3 tile (same planes plus a shift byte per row): the byte table is the
 // codebook cb3, each row's bytes raised by its block's shift bit e_j, and
-// xs[nt] = 2^-sigma_t / 16.
-template <bool NL3>
+// xs[nt] = 2^-sigma_t / 16.  SB2 tile (no HI plane): the 2-bit code is the
+// selector, the table c = 2q - 3, xs[nt] = 2^-sigma_t / 4.
+template <int FMT>
 __device__ __forceinline__ void piece_sbx(const uint8_t* tp,
                                           const uint32_t* xfb, int NT,
                                           const float (&xs)[2],
                                           float (&acc)[2][2], int lane,
                                           int bnt) {
-  constexpr uint32_t T0 = NL3 ? NL3_TAB0 : SB3_TAB0;
-  constexpr uint32_t T1 = NL3 ? NL3_TAB1 : SB3_TAB1;
+  constexpr bool NL3 = FMT == MOE_NL3_256;
+  constexpr bool SB2 = FMT == MOE_SB2_256;
+  constexpr uint32_t T0 = NL3 ? NL3_TAB0 : SB2 ? SB2_TAB0 : SB3_TAB0;
+  constexpr uint32_t T1 = NL3 ? NL3_TAB1 : SB2 ? 0u : SB3_TAB1;
+  constexpr int SC_OFF = SB2 ? 1024 : 1536, D_OFF = SB2 ? 1088 : 1600;
   const int g = lane >> 2;
   const uint4 L0 = *reinterpret_cast<const uint4*>(tp + 16 * lane);
   const uint4 L1 = *reinterpret_cast<const uint4*>(tp + 512 + 16 * lane);
-  const uint4 HV = *reinterpret_cast<const uint4*>(tp + 1024 + 16 * lane);
-  const uint2 SC = *reinterpret_cast<const uint2*>(tp + 1536 + 8 * g);
-  const uint32_t DD = *reinterpret_cast<const uint32_t*>(tp + 1600 + 4 * g);
+  const uint4 HV =
+      SB2 ? make_uint4(0u, 0u, 0u, 0u)
+          : *reinterpret_cast<const uint4*>(tp + 1024 + 16 * lane);
+  const uint2 SC = *reinterpret_cast<const uint2*>(tp + SC_OFF + 8 * g);
+  const uint32_t DD = *reinterpret_cast<const uint32_t*>(tp + D_OFF + 4 * g);
   const uint32_t lo[8] = {L0.x, L0.y, L0.z, L0.w, L1.x, L1.y, L1.z, L1.w};
   const uint32_t hi[4] = {HV.x, HV.y, HV.z, HV.w};
   // NL3: shift bits of rows g (pi = 2g) and g+8 (pi = 2g + 1)
@@ -47,8 +53,11 @@ __device__ __forceinline__ void piece_sbx(const uint8_t* tp,
     const uint32_t LO = lo[j], HH = hi[j >> 1];
     const uint32_t ha = (j & 1) ? HH : (HH << 2);
     const uint32_t hb = (j & 1) ? (HH >> 1) : (HH << 1);
-    const uint32_t sa = (LO & 0x33333333u) | (ha & 0x44444444u);
-    const uint32_t sb = ((LO >> 2) & 0x33333333u) | (hb & 0x44444444u);
+    // selector nibbles: the 3-bit code (SB3, NL3) or the 2-bit code (SB2)
+    const uint32_t sa = SB2 ? (LO & 0x33333333u)
+                            : (LO & 0x33333333u) | (ha & 0x44444444u);
+    const uint32_t sb = SB2 ? ((LO >> 2) & 0x33333333u)
+                            : ((LO >> 2) & 0x33333333u) | (hb & 0x44444444u);
     uint32_t a[4];
     a[0] = prmt(T0, T1, sa);          // row g,   k 4c..4c+3
     a[1] = prmt(T0, T1, sa >> 16);    // row g+8
@@ -93,19 +102,23 @@ __device__ __forceinline__ void piece_sb3(const uint8_t* tp,
                                           const float (&xs)[2],
                                           float (&acc)[2][2], int lane,
                                           int bnt = BF_NT) {
-  piece_sbx<false>(tp, xfb, NT, xs, acc, lane, bnt);
+  piece_sbx<MOE_SB3_256>(tp, xfb, NT, xs, acc, lane, bnt);
 }
 __device__ __forceinline__ void piece_nl3(const uint8_t* tp,
                                           const uint32_t* xfb, int NT,
                                           const float (&xs)[2],
                                           float (&acc)[2][2], int lane,
                                           int bnt = BF_NT) {
-  piece_sbx<true>(tp, xfb, NT, xs, acc, lane, bnt);
+  piece_sbx<MOE_NL3_256>(tp, xfb, NT, xs, acc, lane, bnt);
 }
 // Scale that folds the fixed denominator of a super-block format's value
-// into the activation scale: 1/8 (SB3), 1/16 (NL3), 1 (the 4-bit formats).
+// into the activation scale: 1/8 (SB3), 1/16 (NL3), 1/4 (SB2), 1 (the
+// 4-bit formats).
 __host__ __device__ constexpr float fmt_xfold(int fmt) {
-  return fmt == MOE_SB3_256 ? 0.125f : fmt == MOE_NL3_256 ? 0.0625f : 1.0f;
+  return fmt == MOE_SB3_256   ? 0.125f
+         : fmt == MOE_NL3_256 ? 0.0625f
+         : fmt == MOE_SB2_256 ? 0.25f
+                              : 1.0f;
 }
 
 // Q4 / NL4 tile (16 x 64, two 32-blocks).  cs = column scales of the

@@ -32,10 +32,12 @@ template <int FMT>
 __global__ void __launch_bounds__(XW * 32)
     dq_decode_export_kernel(const uint8_t* __restrict__ t, int rows,
                             int cols, float* __restrict__ out) {
-  constexpr bool SB3 = FMT == MOE_SB3_256 || FMT == MOE_NL3_256;
+  constexpr bool SB3 =
+      FMT == MOE_SB3_256 || FMT == MOE_NL3_256 || FMT == MOE_SB2_256;
   constexpr int TC = SB3 ? SB3_TILE_COLS : B32_TILE_COLS;
   constexpr int TB = FMT == MOE_SB3_256   ? SB3_TILE_BYTES
                      : FMT == MOE_NL3_256 ? NL3_TILE_BYTES
+                     : FMT == MOE_SB2_256 ? SB2_TILE_BYTES
                                           : B32_TILE_BYTES;
   constexpr int NBLK = TC / 32;                 // 32-blocks per tile
   constexpr int FW = NBLK * BF_NT * 64;         // B fragment words
@@ -70,9 +72,9 @@ __global__ void __launch_bounds__(XW * 32)
     __syncwarp();
     float acc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
     if constexpr (SB3) {
-      // 2^-sigma / 8 (SB3) or / 16 (NL3), sigma = 0
+      // 2^-sigma / 8 (SB3), / 16 (NL3) or / 4 (SB2), sigma = 0
       const float xs[2] = {fmt_xfold(FMT), fmt_xfold(FMT)};
-      piece_sbx<FMT == MOE_NL3_256>(tp, frag, BF_NT, xs, acc, lane, BF_NT);
+      piece_sbx<FMT>(tp, frag, BF_NT, xs, acc, lane, BF_NT);
     } else {
       const float cs[8] = {1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f};
       piece_b32<FMT>(tp, frag, BF_NT, cs, 0, acc, lane, BF_NT);
@@ -122,6 +124,10 @@ extern "C" moe_status moe_dequant_path(int fmt, int path,
       break;
     case MOE_NL3_256:
       dq_decode_export_kernel<MOE_NL3_256><<<grid, XW * 32, 0, s>>>(
+          packed, rows, cols, o);
+      break;
+    case MOE_SB2_256:
+      dq_decode_export_kernel<MOE_SB2_256><<<grid, XW * 32, 0, s>>>(
           packed, rows, cols, o);
       break;
     default:

@@ -72,9 +72,11 @@ template <int FMT>
 __global__ void __launch_bounds__(DEC_THREADS, 1)
     ffn_up_decode_kernel(DecParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
-  constexpr bool SBF = FMT == MOE_SB3_256 || FMT == MOE_NL3_256;
+  constexpr bool SBF = FMT == MOE_SB3_256 || FMT == MOE_NL3_256 ||
+                      FMT == MOE_SB2_256;
   constexpr int TB = FMT == MOE_SB3_256   ? SB3_TILE_BYTES
                      : FMT == MOE_NL3_256 ? NL3_TILE_BYTES
+                     : FMT == MOE_SB2_256 ? SB2_TILE_BYTES
                                           : B32_TILE_BYTES;
   constexpr int TC = SBF ? SB3_TILE_COLS : B32_TILE_COLS;
   const int nk = p.H / TC;
@@ -199,7 +201,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 1)
       const float* xb = xsc + ((k0 + kt) * TC / XB_COLS) * DEC_TMAX;
       if (SBF) {
         const float xs[2] = {xb[c], xb[4 + c]};
-        piece_sbx<FMT == MOE_NL3_256>(chunk + kt * TB,
+        piece_sbx<FMT>(chunk + kt * TB,
                                       xf + blk0 * BF_NT * 64, NT, xs, acc,
                                       lane, BF_NT);
       } else {
@@ -534,6 +536,9 @@ moe_status launch_up_decode(const moe_layer_desc& d, const uint16_t* x,
                         prm);
     case MOE_NL3_256:
       return launch_pdl(ffn_up_decode_kernel<MOE_NL3_256>, grid, su, s, pdl,
+                        prm);
+    case MOE_SB2_256:
+      return launch_pdl(ffn_up_decode_kernel<MOE_SB2_256>, grid, su, s, pdl,
                         prm);
     default:
       return launch_pdl(ffn_up_decode_kernel<MOE_Q4_B32>, grid, su, s, pdl,

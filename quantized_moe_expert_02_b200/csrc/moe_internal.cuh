@@ -43,21 +43,29 @@ namespace moe {
 //   [1632,1648)  codebook-shift bytes, row r at 1632 + pi(r) (bit j = e_j
 //                of 32-block j)
 // 1648 bytes.
+//
+// SB2 tile (MOE_SB2_256) = 16 rows x 256 columns of 2-bit codes, 1120
+// bytes: the SB3 tile without its HI plane --
+//   [   0,1024)  LO[0..7] as in SB3 (the 2-bit code of each weight)
+//   [1024,1088)  sub-scale words, row r at 4*pi(r)
+//   [1088,1120)  fp16 d, row r at 2*pi(r)
 constexpr int SB3_TILE_BYTES = 1632;
+constexpr int SB2_TILE_BYTES = 1120;
 constexpr int SB3_TILE_COLS = 256;
 constexpr int NL3_TILE_BYTES = 1648;
 constexpr int B32_TILE_BYTES = 576;
 constexpr int B32_TILE_COLS = 64;
 constexpr int TILE_ROWS = 16;
 
-// The super-block formats (256 columns per tile, 3-bit codes in LO/HI
-// planes): SB3 and NL3.
+// The super-block formats (256 columns per tile, codes in the LO plane and,
+// for the 3-bit ones, the HI plane): SB3, NL3 and SB2.
 __host__ __device__ inline bool fmt_sb(int fmt) {
-  return fmt == MOE_SB3_256 || fmt == MOE_NL3_256;
+  return fmt == MOE_SB3_256 || fmt == MOE_NL3_256 || fmt == MOE_SB2_256;
 }
 __host__ __device__ inline int tile_bytes(int fmt) {
   return fmt == MOE_SB3_256   ? SB3_TILE_BYTES
          : fmt == MOE_NL3_256 ? NL3_TILE_BYTES
+         : fmt == MOE_SB2_256 ? SB2_TILE_BYTES
                               : B32_TILE_BYTES;
 }
 __host__ __device__ inline int tile_cols(int fmt) {
@@ -65,7 +73,7 @@ __host__ __device__ inline int tile_cols(int fmt) {
 }
 inline bool fmt_valid(int fmt) {
   return fmt == MOE_Q4_B32 || fmt == MOE_SB3_256 || fmt == MOE_NL4_B32 ||
-         fmt == MOE_NL3_256;
+         fmt == MOE_NL3_256 || fmt == MOE_SB2_256;
 }
 // Shape accepted by the packed layout.
 inline bool packed_shape_ok(int fmt, int rows, int cols) {
@@ -94,6 +102,8 @@ constexpr uint32_t NL4_TB1 = 0x725A4636u;   //   54,  70, 90,114
 // 32-bit add never carries across bytes).
 constexpr uint32_t NL3_TAB0 = 0xFEFAF6F1u;  // -15,-10, -6, -2
 constexpr uint32_t NL3_TAB1 = 0x0E090501u;  //   1,  5,  9, 14
+// SB2: code q (0..3) -> c = 2q - 3.
+constexpr uint32_t SB2_TAB0 = 0x0301FFFDu;  // -3,-1, 1, 3
 // Q4: q - 8 in the same split.
 constexpr uint32_t Q4_TA0 = 0xFBFAF9F8u;    // -8..-5
 constexpr uint32_t Q4_TA1 = 0xFFFEFDFCu;    // -4..-1
@@ -383,6 +393,12 @@ __device__ inline float dq_packed(int fmt, const uint8_t* t, int cols,
     const int n = 4 * reg_odd + w;
     const uint32_t lo =
         *(const uint32_t*)(tile + 512 * (j / 4) + 16 * lane + 4 * (j % 4));
+    if (fmt == MOE_SB2_256) {
+      const int q2 = (lo >> (4 * n + 2 * reg_hi)) & 3;
+      const int s2 = (*(const uint32_t*)(tile + 1024 + 4 * pi) >> (4 * j)) & 15;
+      const float d2 = __half2float(*(const __half*)(tile + 1088 + 2 * pi));
+      return d2 * (float)((2 * s2 + 1) * (2 * q2 - 3)) * 0.25f;
+    }
     const uint32_t hi = *(const uint32_t*)(tile + 1024 + 16 * lane +
                                            4 * (j / 2));
     const int q = ((lo >> (4 * n + 2 * reg_hi)) & 3) |

@@ -18,6 +18,13 @@ __device__ inline int nat_sb3_code(const uint8_t* codes, int cols, int row,
   const uint32_t v = p[0] | ((bit / 8 + 1 < 96) ? ((uint32_t)p[1] << 8) : 0u);
   return (v >> (bit % 8)) & 7;
 }
+// SB2 natural: codes plane (64 B per super-block, code i at bit 2i).
+__device__ inline int nat_sb2_code(const uint8_t* codes, int cols, int row,
+                                   int col) {
+  const int64_t sb = (int64_t)row * (cols / 256) + col / 256;
+  const int i = col % 256;
+  return (codes[sb * 64 + i / 4] >> (2 * (i % 4))) & 3;
+}
 __device__ inline int nat_b32_code(const uint8_t* codes, int cols, int row,
                                    int col) {
   const int64_t i = (int64_t)row * cols + col;
@@ -90,6 +97,54 @@ __global__ void pack_sb3_kernel(const uint8_t* __restrict__ nat, int rows,
         const int r = pi / 2 + 8 * (pi % 2);
         word |= (uint32_t)extra[(int64_t)(16 * rt + r) * ntc + kb] << (8 * h);
       }
+    }
+    out[wi] = word;
+  }
+}
+
+// SB2: the LO words of the SB3 tile (the 2-bit codes), then the sub-scale
+// words and the fp16 d, one thread per 32-bit word.
+__global__ void pack_sb2_kernel(const uint8_t* __restrict__ nat, int rows,
+                                int cols, uint32_t* __restrict__ out) {
+  constexpr int TBW = SB2_TILE_BYTES / 4;
+  const int ntc = cols / 256;
+  const int64_t ntiles = (int64_t)(rows / 16) * ntc;
+  const int64_t nwords = ntiles * TBW;
+  const int64_t nsb = (int64_t)rows * ntc;
+  const uint8_t* codes = nat;
+  const uint32_t* scales = (const uint32_t*)(nat + nsb * 64);
+  const uint16_t* dplane = (const uint16_t*)(nat + nsb * 68);
+  for (int64_t wi = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+       wi < nwords; wi += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t tile = wi / TBW;
+    const int w = (int)(wi % TBW);
+    const int rt = (int)(tile / ntc), kb = (int)(tile % ntc);
+    uint32_t word = 0;
+    if (w < 256) {  // LO[j]
+      const int seg = w / 128, lane = (w % 128) / 4, iw = w % 4;
+      const int g = lane / 4, c = lane % 4;
+      const int j = 4 * seg + iw;
+      for (int r = 0; r < 4; ++r)
+        for (int e = 0; e < 4; ++e) {
+          const int row = 16 * rt + g + 8 * (r & 1);
+          const int col = 256 * kb + 32 * j + 16 * (r >> 1) + 4 * c + e;
+          const int q = nat_sb2_code(codes, cols, row, col);
+          const int n = 4 * (r & 1) + e;
+          word |= (uint32_t)q << (4 * n + 2 * (r >> 1));
+        }
+    } else if (w < 272) {  // sub-scale words, packed index pi
+      const int pi = w - 256;
+      const int r = pi / 2 + 8 * (pi % 2);
+      word = scales[(int64_t)(16 * rt + r) * ntc + kb];
+    } else {  // d: two fp16 per word
+      const int p0 = 2 * (w - 272);
+      uint32_t lohi[2];
+      for (int h = 0; h < 2; ++h) {
+        const int pi = p0 + h;
+        const int r = pi / 2 + 8 * (pi % 2);
+        lohi[h] = dplane[(int64_t)(16 * rt + r) * ntc + kb];
+      }
+      word = lohi[0] | (lohi[1] << 16);
     }
     out[wi] = word;
   }
@@ -180,6 +235,9 @@ extern "C" moe_status moe_pack_tensor(int fmt, const uint8_t* natural,
         natural, rows, cols, (uint32_t*)packed);
   else if (fmt == MOE_NL3_256)
     pack_sb3_kernel<true><<<grid_for(words, 256), 256, 0, s>>>(
+        natural, rows, cols, (uint32_t*)packed);
+  else if (fmt == MOE_SB2_256)
+    pack_sb2_kernel<<<grid_for(words, 256), 256, 0, s>>>(
         natural, rows, cols, (uint32_t*)packed);
   else
     pack_b32_kernel<<<grid_for(words, 256), 256, 0, s>>>(natural, rows, cols,

@@ -42,13 +42,17 @@ constexpr int PF_B_BYTES = PF_BN * PF_BK * 2;         // 32 KB
 constexpr int PF_TMEM_COLS = 512;
 // A operand formats of the GEMM kernels: the 4-bit 32-weight blocks (Q4,
 // NL4), and the 3-bit super-blocks SB3 and NL3.
-constexpr int AF_B32 = 0, AF_SB3 = 1, AF_NL3 = 2;
+constexpr int AF_B32 = 0, AF_SB3 = 1, AF_NL3 = 2, AF_SB2 = 3;
 __host__ __device__ constexpr int af_of(int fmt) {
-  return fmt == MOE_SB3_256 ? AF_SB3 : fmt == MOE_NL3_256 ? AF_NL3 : AF_B32;
+  return fmt == MOE_SB3_256   ? AF_SB3
+         : fmt == MOE_NL3_256 ? AF_NL3
+         : fmt == MOE_SB2_256 ? AF_SB2
+                              : AF_B32;
 }
 __host__ __device__ constexpr int af_tile_bytes(int af) {
-  return af == AF_SB3 ? SB3_TILE_BYTES
+  return af == AF_SB3   ? SB3_TILE_BYTES
          : af == AF_NL3 ? NL3_TILE_BYTES
+         : af == AF_SB2 ? SB2_TILE_BYTES
                         : B32_TILE_BYTES;
 }
 
@@ -136,6 +140,8 @@ __device__ __forceinline__ uint32_t sw128(int r, int chunk) {
 // fp16 high bytes of c = 2q - 7 for q = 0..3 and 4..7 (the low bytes are 0).
 constexpr uint32_t SB3_H16_LO = 0xBCC2C5C7u;   // -1,-3,-5,-7 (bytes 3..0)
 constexpr uint32_t SB3_H16_HI = 0x4745423Cu;   //  7, 5, 3, 1
+// SB2: fp16 high bytes of c = 2q - 3 for q = 0..3 (the low bytes are 0)
+constexpr uint32_t SB2_H16 = 0x423CBCC2u;      //  3, 1,-1,-3 (bytes 3..0)
 
 // One thread's share of a 16-row SB3 tile (one super-block per row) for
 // one of the two dequant groups: group gamma takes k-steps q = gamma and
@@ -151,7 +157,8 @@ struct Sb3Half {
   uint32_t ex;      // NL3: shift bytes of rows g (bits 0-7), g+8 (8-15)
 };
 
-__device__ __forceinline__ void sb3_load(const uint8_t* tp, int g, int p,
+template <bool SB2>
+__device__ __forceinline__ void sbq_load(const uint8_t* tp, int g, int p,
                                          int gamma, Sb3Half& q) {
   const int L0 = 4 * g + 2 * p;
 #pragma unroll
@@ -159,11 +166,16 @@ __device__ __forceinline__ void sb3_load(const uint8_t* tp, int g, int p,
     const uint8_t* lw = tp + 16 * (L0 + l);
     q.lo[0][l] = ldg_u64(lw + 8 * gamma);
     q.lo[1][l] = ldg_u64(lw + 512 + 8 * gamma);
-    q.hi[l] = make_uint2(ldg_u32(lw + 1024 + 4 * gamma),
-                         ldg_u32(lw + 1024 + 8 + 4 * gamma));
+    q.hi[l] = SB2 ? make_uint2(0u, 0u)
+                  : make_uint2(ldg_u32(lw + 1024 + 4 * gamma),
+                               ldg_u32(lw + 1024 + 8 + 4 * gamma));
   }
-  q.sc = ldg_u64(tp + 1536 + 8 * g);
-  q.d = ldg_u32(tp + 1600 + 4 * g);
+  q.sc = ldg_u64(tp + (SB2 ? 1024 : 1536) + 8 * g);
+  q.d = ldg_u32(tp + (SB2 ? 1088 : 1600) + 4 * g);
+}
+__device__ __forceinline__ void sb3_load(const uint8_t* tp, int g, int p,
+                                         int gamma, Sb3Half& q) {
+  sbq_load<false>(tp, g, p, gamma, q);
 }
 __device__ __forceinline__ void nl3_load(const uint8_t* tp, int g, int p,
                                          int gamma, Sb3Half& q) {
@@ -174,24 +186,31 @@ __device__ __forceinline__ void nl3_load(const uint8_t* tp, int g, int p,
 // 8 codes of one lane word (nibble n = 4*rowhalf + w) -> fp16 c values as
 // two half2 words per row: out[0..1] row g (w = 0,1 | 2,3), out[2..3] row
 // g+8.  Q holds one 3-bit code per nibble (bit 3 clear).
-__device__ __forceinline__ void sb3_codes_to_h16(uint32_t Q,
+template <bool SB2>
+__device__ __forceinline__ void sbq_codes_to_h16(uint32_t Q,
                                                  uint32_t (&o)[4]) {
+  // SB3: table bytes 0..7; SB2: bytes 0..3, and byte 4 (a zero) for C
+  constexpr uint32_t TL = SB2 ? SB2_H16 : SB3_H16_LO;
+  constexpr uint32_t TH = SB2 ? 0u : SB3_H16_HI;
   const uint32_t S = Q << 4;
-  // selector nibbles [C, q(n), C, q(n+1)]: C = 0xC picks a zero byte
+  // selector nibbles [C, q(n), C, q(n+1)]: C = 0xC picks a zero byte (the
+  // sign, replicated, of a byte whose top bit is clear)
   const uint32_t X0 = (prmt(Q, S, 0x1504u) & 0xF0F0F0F0u) | 0x0C0C0C0Cu;
   const uint32_t X1 = (prmt(Q, S, 0x3726u) & 0xF0F0F0F0u) | 0x0C0C0C0Cu;
-  o[0] = prmt(SB3_H16_LO, SB3_H16_HI, X0);
-  o[1] = prmt(SB3_H16_LO, SB3_H16_HI, X0 >> 16);
-  o[2] = prmt(SB3_H16_LO, SB3_H16_HI, X1);
-  o[3] = prmt(SB3_H16_LO, SB3_H16_HI, X1 >> 16);
+  o[0] = prmt(TL, TH, X0);
+  o[1] = prmt(TL, TH, X0 >> 16);
+  o[2] = prmt(TL, TH, X1);
+  o[3] = prmt(TL, TH, X1 >> 16);
 }
 
 // The group's k-step qh (0/1) of the super-block, i.e. k-step
 // q = gamma + 2*qh: sub-blocks j0 = 2q and 2q+1 -> fp16 rows g and g+8 of
 // the swizzled A tile.
-__device__ __forceinline__ void sb3_store(const Sb3Half& sb, int g, int p,
+template <bool SB2>
+__device__ __forceinline__ void sbq_store(const Sb3Half& sb, int g, int p,
                                           int gamma, int qh, int row0,
                                           uint32_t a_smem) {
+  constexpr float FOLD = SB2 ? 0.25f : 0.125f;   // (2s+1)/4 or /8
   const int q = gamma + 2 * qh;
   const int j0 = 2 * q;
   const uint32_t dg = half_bcast((uint16_t)(sb.d & 0xFFFFu));
@@ -200,9 +219,9 @@ __device__ __forceinline__ void sb3_store(const Sb3Half& sb, int g, int p,
   for (int jj = 0; jj < 2; ++jj) {
     const int j = j0 + jj;
     const int sg = (sb.sc.x >> (4 * j)) & 15, sg8 = (sb.sc.y >> (4 * j)) & 15;
-    // (2s+1)/8, exact in fp16
-    const __half tg = __float2half_rn((float)(2 * sg + 1) * 0.125f);
-    const __half tg8 = __float2half_rn((float)(2 * sg8 + 1) * 0.125f);
+    // (2s+1)/8 (SB3) or /4 (SB2), exact in fp16
+    const __half tg = __float2half_rn((float)(2 * sg + 1) * FOLD);
+    const __half tg8 = __float2half_rn((float)(2 * sg8 + 1) * FOLD);
     const uint32_t t2g = half_bcast(__half_as_ushort(tg));
     const uint32_t t2g8 = half_bcast(__half_as_ushort(tg8));
     uint32_t w[2][2][4];   // [lane][h][words]
@@ -210,10 +229,13 @@ __device__ __forceinline__ void sb3_store(const Sb3Half& sb, int g, int p,
     for (int l = 0; l < 2; ++l) {
       const uint32_t lo = jj ? sb.lo[qh][l].y : sb.lo[qh][l].x;
       const uint32_t hi = (qh ? sb.hi[l].y : sb.hi[l].x) >> (2 * jj);
-      const uint32_t Q0 = (lo & 0x33333333u) | ((hi << 2) & 0x44444444u);
-      const uint32_t Q1 = ((lo >> 2) & 0x33333333u) | ((hi << 1) & 0x44444444u);
-      sb3_codes_to_h16(Q0, w[l][0]);
-      sb3_codes_to_h16(Q1, w[l][1]);
+      const uint32_t Q0 = SB2 ? (lo & 0x33333333u)
+                              : (lo & 0x33333333u) | ((hi << 2) & 0x44444444u);
+      const uint32_t Q1 = SB2 ? ((lo >> 2) & 0x33333333u)
+                              : ((lo >> 2) & 0x33333333u) |
+                                    ((hi << 1) & 0x44444444u);
+      sbq_codes_to_h16<SB2>(Q0, w[l][0]);
+      sbq_codes_to_h16<SB2>(Q1, w[l][1]);
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         w[l][h][0] = hmul2u(hmul2u(w[l][h][0], t2g), dg);
@@ -231,6 +253,12 @@ __device__ __forceinline__ void sb3_store(const Sb3Half& sb, int g, int p,
                    w[0][h][3], w[1][h][2], w[1][h][3]);
     }
   }
+}
+
+__device__ __forceinline__ void sb3_store(const Sb3Half& sb, int g, int p,
+                                          int gamma, int qh, int row0,
+                                          uint32_t a_smem) {
+  sbq_store<false>(sb, g, p, gamma, qh, row0, a_smem);
 }
 
 // ------------------------------------------------------------- NL3 ----
@@ -306,6 +334,7 @@ template <int AF>
 __device__ __forceinline__ void sbx_load(const uint8_t* tp, int g, int p,
                                          int gamma, Sb3Half& q) {
   if constexpr (AF == AF_NL3) nl3_load(tp, g, p, gamma, q);
+  else if constexpr (AF == AF_SB2) sbq_load<true>(tp, g, p, gamma, q);
   else sb3_load(tp, g, p, gamma, q);
 }
 template <int AF>
@@ -313,6 +342,8 @@ __device__ __forceinline__ void sbx_store(const Sb3Half& sb, int g, int p,
                                           int gamma, int qh, int row0,
                                           uint32_t a_smem) {
   if constexpr (AF == AF_NL3) nl3_store(sb, g, p, gamma, qh, row0, a_smem);
+  else if constexpr (AF == AF_SB2)
+    sbq_store<true>(sb, g, p, gamma, qh, row0, a_smem);
   else sb3_store(sb, g, p, gamma, qh, row0, a_smem);
 }
 
@@ -951,6 +982,7 @@ moe_status launch_pf_dequant_export(int fmt, const uint8_t* t, int rows,
   const int af = af_of(fmt);
   const void* fn = af == AF_SB3   ? (const void*)&pf_dequant_export_kernel<AF_SB3>
                    : af == AF_NL3 ? (const void*)&pf_dequant_export_kernel<AF_NL3>
+                   : af == AF_SB2 ? (const void*)&pf_dequant_export_kernel<AF_SB2>
                                   : (const void*)&pf_dequant_export_kernel<AF_B32>;
   moe_status st = ensure_smem(fn, smem);
   if (st != MOE_OK) return st;
@@ -961,6 +993,9 @@ moe_status launch_pf_dequant_export(int fmt, const uint8_t* t, int rows,
                                                              out);
   else if (af == AF_NL3)
     pf_dequant_export_kernel<AF_NL3><<<grid, 256, smem, s>>>(t, cols, tab4,
+                                                             out);
+  else if (af == AF_SB2)
+    pf_dequant_export_kernel<AF_SB2><<<grid, 256, smem, s>>>(t, cols, tab4,
                                                              out);
   else
     pf_dequant_export_kernel<AF_B32><<<grid, 256, smem, s>>>(t, cols, tab4,
@@ -1025,6 +1060,7 @@ static moe_status pf_launch_fmt(int fmt, const PfParams& prm,
   switch (af_of(fmt)) {
     case AF_SB3: return pf_launch<UP, AF_SB3>(prm, map, s);
     case AF_NL3: return pf_launch<UP, AF_NL3>(prm, map, s);
+    case AF_SB2: return pf_launch<UP, AF_SB2>(prm, map, s);
     default: return pf_launch<UP, AF_B32>(prm, map, s);
   }
 }

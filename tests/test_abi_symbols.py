@@ -43,6 +43,11 @@ def test_host_side_queries_without_gpu():
     assert moe.moe_blob_bytes(moe.MOE_SB3_256, moe.MOE_NL4_B32, 3072,
                               1024) == 4276224
     assert moe.moe_tensor_bytes(moe.MOE_SB3_256, 16, 100) == 0
+    # 16 x 256 tiles: SB3 1632 B, NL3 1648 B, SB2 1120 B
+    assert moe.moe_tensor_bytes(moe.MOE_NL3_256, 1024, 3072) == 64 * 12 * 1648
+    assert moe.moe_tensor_bytes(moe.MOE_SB2_256, 1024, 3072) == 64 * 12 * 1120
+    assert moe.moe_tensor_bytes(moe.MOE_SB2_256, 8, 256) == 0
+    assert moe.moe_tensor_bytes(6, 1024, 3072) == 0
     assert moe.moe_ffn_workspace_bytes(3, 10, 3072, 1024) > 0
     assert moe.status_string(moe.MOE_ERR_CAPACITY).startswith("slot")
 

@@ -1,8 +1,10 @@
-"""GPU: the 3-bit non-uniform-codebook format (MOE_NL3_256, this library's
-stand-in for the 3-bit non-linear type the model card lists for up/gate) end
-to end: up/gate in NL3, down in NL4, through the one-kernel decode layer,
-the split decode kernels and the tensor-core prefill path, against the
-fp64 oracle (whose NL3 dequantisation is pinned on the CPU)."""
+"""GPU: this library's two further up/gate formats end to end -- the 3-bit
+non-uniform-codebook super-block (MOE_NL3_256, stand-in for the 3-bit
+non-linear type the model card lists) and the 2-bit super-block
+(MOE_SB2_256, stand-in for the card's 2-bit up/gate type) -- with down in
+NL4, through the one-kernel decode layer, the split decode kernels and the
+tensor-core prefill path, against the fp64 oracle (whose dequantisation of
+both formats is pinned on the CPU)."""
 import numpy as np
 import pytest
 import torch
@@ -15,17 +17,22 @@ from helpers import (TOL, Ws, build_pool, dev, layer_desc, oracle_experts,
 
 pytestmark = pytest.mark.gpu
 
-SHAPE = synth.NL3_SHAPE
+SHAPES = {"nl3": synth.NL3_SHAPE, "sb2": synth.SB2_SHAPE}
 _POOL = {}
 
 
-def pool():
-    if "p" not in _POOL:
-        _POOL["p"] = build_pool(SHAPE, 0, 0)
-    return _POOL["p"]
+@pytest.fixture(params=sorted(SHAPES))
+def fmt_shape(request):
+    """(name, shape); one resident pool per format, the previous one freed."""
+    name = request.param
+    if name not in _POOL:
+        _POOL.clear()
+        torch.cuda.empty_cache()
+        _POOL[name] = build_pool(SHAPES[name], 0, 0)
+    return SHAPES[name], _POOL[name]
 
 
-def oracle_y(x_bits, idx):
+def oracle_y(SHAPE, x_bits, idx):
     src = oracle_experts(SHAPE, 0, 0)
     x = o.bf16_to_f64(x_bits)
     T, k = idx.shape
@@ -38,9 +45,10 @@ def oracle_y(x_bits, idx):
 
 
 @pytest.mark.parametrize("T", [1, 3, 8, 40, 300])
-def test_nl3_expert_ffn_vs_oracle(T):
+def test_expert_ffn_vs_oracle(fmt_shape, T):
     """T <= 8: split decode kernels; T > 8: the prefill GEMMs."""
-    desc = layer_desc(SHAPE, pool())
+    SHAPE, pool = fmt_shape
+    desc = layer_desc(SHAPE, pool)
     x, wr, _ = route_inputs(SHAPE, 0, 0, T, step=1)
     idx, _, _ = run_route(x, wr, None, SHAPE.k, T, SHAPE.H, SHAPE.E)
     _, _, _, err, (d_idx, off, pairs, act, na) = run_group(idx, SHAPE.E)
@@ -52,13 +60,14 @@ def test_nl3_expert_ffn_vs_oracle(T):
     assert moe.moe_get_device_status(ws.t) == 0
     got = y.cpu().numpy()
     assert np.isfinite(got).all()
-    assert row_max_rel(got, oracle_y(x, idx)) <= TOL
+    assert row_max_rel(got, oracle_y(SHAPE, x, idx)) <= TOL
 
 
 @pytest.mark.parametrize("T", [1, 3, 5])
-def test_nl3_layer_forward_vs_oracle(T):
-    """The one-kernel decode layer with NL3 up/gate."""
-    desc = layer_desc(SHAPE, pool())
+def test_layer_forward_vs_oracle(fmt_shape, T):
+    """The one-kernel decode layer with NL3 or SB2 up/gate."""
+    SHAPE, pool = fmt_shape
+    desc = layer_desc(SHAPE, pool)
     k, E, H = SHAPE.k, SHAPE.E, SHAPE.H
     x, wr, _ = route_inputs(SHAPE, 0, 0, T, step=2)
     ws = Ws(moe.moe_layer_workspace_bytes(T, k, E, H, SHAPE.F))

@@ -53,6 +53,8 @@ def check(fmt, path, nat, rows, cols):
     (synth.NL4_B32, 3072, 1024),
     (synth.Q4_B32, 128, 128), (synth.Q4_B32, 256, 256),
     (synth.NL3_256, 128, 256), (synth.NL3_256, 1024, 3072),
+    (synth.SB2_256, 128, 256), (synth.SB2_256, 256, 768),
+    (synth.SB2_256, 1024, 3072),
 ])
 def test_hot_path_decoders_random(fmt, rows, cols, path):
     nat = synth.gen_tensor(13, 1, rows + cols, "up", fmt, rows, cols,
@@ -63,6 +65,7 @@ def test_hot_path_decoders_random(fmt, rows, cols, path):
 @pytest.mark.parametrize("fmt,rows,cols", [
     (synth.SB3_256, 16, 256), (synth.SB3_256, 48, 512),
     (synth.NL4_B32, 16, 64), (synth.Q4_B32, 48, 192),
+    (synth.SB2_256, 16, 256), (synth.NL3_256, 48, 512),
 ])
 def test_decode_decoders_small_tiles(fmt, rows, cols):
     """The decode path's 16-row tiles (no 128-row blocks needed)."""
@@ -119,6 +122,34 @@ def test_nl3_every_subscale_code_and_shift(path):
             for r in range(256) for i in range(256)}
     assert len(trip) == 16 * 8 * 2
     check(synth.NL3_256, path, nat, 256, 256)
+
+
+def sb2_every_pair(rows=128, dmin=0.001, dmax=0.03):
+    """Natural SB2 tensor [rows x 256]: row r has sub-scales (r//8 + j) % 16
+    and codes (r + i) % 4, so every (sub-scale, code) pair occurs at every
+    position class."""
+    codes, scales = bytearray(), bytearray()
+    for r in range(rows):
+        s, q = (r // 8) % 16, r % 4
+        acc = 0
+        for i in range(256):
+            acc |= ((q + i) % 4) << (2 * i)
+        codes += acc.to_bytes(64, "little")
+        acc = 0
+        for j in range(8):
+            acc |= ((s + j) % 16) << (4 * j)
+        scales += acc.to_bytes(4, "little")
+    d = np.linspace(dmin, dmax, rows).astype(np.float16).tobytes()
+    return np.frombuffer(bytes(codes) + bytes(scales) + d, np.uint8)
+
+
+@pytest.mark.parametrize("path", [DEC, PF])
+def test_sb2_every_subscale_and_code(path):
+    nat = sb2_every_pair()
+    pairs = {(((r // 8) + i // 32) % 16, (r + i) % 4)
+             for r in range(128) for i in range(256)}
+    assert len(pairs) == 16 * 4
+    check(synth.SB2_256, path, nat, 128, 256)
 
 
 def b32_every_code(rows=128, cols=128, dmin=0.001, dmax=0.03):

@@ -16,6 +16,7 @@ pytestmark = pytest.mark.gpu
     (synth.TINY, 0, list(range(16))),
     (synth.BIG, 3, [0, 257, 511]),
     (synth.NL3_SHAPE, 1, [0, 5, 63]),
+    (synth.SB2_SHAPE, 2, [0, 9, 63]),
 ])
 def test_device_generator_matches_host(shape, layer, experts):
     stride = shape.blob_stride
@@ -38,6 +39,8 @@ def test_device_generator_matches_host(shape, layer, experts):
     (synth.Q4_B32, 32, 128), (synth.Q4_B32, 128, 256),
     (synth.NL3_256, 16, 256), (synth.NL3_256, 48, 768),
     (synth.NL3_256, 1024, 3072),
+    (synth.SB2_256, 16, 256), (synth.SB2_256, 48, 768),
+    (synth.SB2_256, 1024, 3072),
 ])
 def test_pack_dequant_bit_exact(fmt, rows, cols):
     nat = synth.gen_tensor(11, 2, rows + cols, "up", fmt, rows, cols,
