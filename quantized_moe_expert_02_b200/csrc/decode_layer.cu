@@ -611,12 +611,14 @@ __global__ void __launch_bounds__(STG ? LAYER_THREADS_STG : LAYER_THREADS, 1)
   // eight: those blocks also take the last experts' down units, whose up
   // units are the last to finish, so they wait for them before their down
   // phase.  Plain even split when that weighting does not fit (ranges must
-  // stay within two experts).
+  // stay within two experts), and for one token: with its ten experts a
+  // block has only four or five up units, and the even split is the faster
+  // deal there (30.3 vs 30.8 us per layer on one B200).
   int d0, d1;
   {
     const int q_up = nu_all / G, extra = nu_all % G;
     const int64_t ctot = 4LL * q_up * G + 8LL * extra + nd_all;
-    const bool weighted = (4LL * q_up + 8) * G <= ctot &&
+    const bool weighted = T > 1 && (4LL * q_up + 8) * G <= ctot &&
                           (ctot + G - 1) / G - 4LL * q_up <= nrt_h;
     if (weighted) {
       auto before = [&](int pos) -> int {   // down units of positions < pos
