@@ -1,4 +1,4 @@
-// Tile decoders of the decode path: packed SB3 / Q4 / NL4 tiles -> int8 A
+// Tile decoders of the decode path: packed SB3 / NL3 / SB2 / Q4 / NL4 tiles -> int8 A
 // fragments of mma.m16n8k32 (byte-table lookups with prmt), multiplied by
 // int8 B fragments of the activations (v = 256*hi + lo), exact int32 sums
 // per 32-block, scales applied in fp32.

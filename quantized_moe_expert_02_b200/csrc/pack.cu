@@ -33,7 +33,7 @@ __device__ inline int nat_b32_code(const uint8_t* codes, int cols, int row,
 }
 
 // One thread per 32-bit word of the packed tensor.  SB3 and NL3 (the NL3
-// tile appends the codebook-shift bytes of its 16 rows).
+// tile appends the codebook-shift bytes of its 16 rows); SB2 below.
 template <bool NL3>
 __global__ void pack_sb3_kernel(const uint8_t* __restrict__ nat, int rows,
                                 int cols, uint32_t* __restrict__ out) {

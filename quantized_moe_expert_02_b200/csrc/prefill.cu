@@ -41,7 +41,7 @@ constexpr int PF_A_BYTES = PF_BM * PF_BK * 2;         // 16 KB
 constexpr int PF_B_BYTES = PF_BN * PF_BK * 2;         // 32 KB
 constexpr int PF_TMEM_COLS = 512;
 // A operand formats of the GEMM kernels: the 4-bit 32-weight blocks (Q4,
-// NL4), and the 3-bit super-blocks SB3 and NL3.
+// NL4), the 3-bit super-blocks SB3 and NL3, and the 2-bit super-block SB2.
 constexpr int AF_B32 = 0, AF_SB3 = 1, AF_NL3 = 2, AF_SB2 = 3;
 __host__ __device__ constexpr int af_of(int fmt) {
   return fmt == MOE_SB3_256   ? AF_SB3
@@ -329,7 +329,7 @@ __device__ __forceinline__ void nl3_store(const Sb3Half& sb, int g, int p,
   }
 }
 
-// Super-block format of a GEMM's A operand: SB3 or NL3 load / store.
+// Super-block format of a GEMM's A operand: SB3, NL3 or SB2 load / store.
 template <int AF>
 __device__ __forceinline__ void sbx_load(const uint8_t* tp, int g, int p,
                                          int gamma, Sb3Half& q) {
@@ -468,7 +468,7 @@ __global__ void __launch_bounds__(256)
 template <bool UP, int AF>
 __global__ void __launch_bounds__(PfCfg<UP>::THREADS, 1)
     pf_gemm_kernel(const PfParams p, const __grid_constant__ PfMaps maps) {
-  constexpr bool SB3 = AF != AF_B32;   // a super-block format (SB3, NL3)
+  constexpr bool SB3 = AF != AF_B32;   // a super-block format (SB3, NL3, SB2)
   using C = PfCfg<UP>;
   constexpr int NA = C::NA, S = C::STAGES;
   extern __shared__ uint8_t smem_raw[];
