@@ -539,6 +539,20 @@ def decode_measure(lay, T, K, W):
             "unique_experts_per_step": u_avg}, ms
 
 
+def decode_sweep(lay, W: int, steps: int = 2048) -> dict:
+    """The one-kernel decode layer at every token count it serves (1..8):
+    per-layer time, tokens/s and the fraction of measured HBM bandwidth of
+    its algorithmic bytes (same resident layers, graph replay)."""
+    out = {}
+    for T in range(1, 9):
+        d, _ = decode_measure(lay, T, steps, W)
+        out[str(T)] = {"us_per_layer": d["ms_per_step"] * 1e3,
+                       "tokens_per_s": d["tokens_per_s"],
+                       "frac_of_hbm": d["frac_of_hbm"],
+                       "unique_experts": d["unique_experts_per_step"]}
+    return out
+
+
 def clock_soak(lay, T: int, ms_per_step: float, seconds: float = 1.0):
     """nvidia-smi clock samples over about `seconds` of the same decode
     steps (graph replays): the timed region itself may be too short for
@@ -861,6 +875,8 @@ def run_ours(args) -> None:
             "clocks": clocks,
         }
         line["clocks_soak"] = clock_soak(lay, T, ms / K)
+        if world == 1 and not args.no_extras:
+            line["decode_sweep"] = decode_sweep(lay, W)
         if not args.no_prefill:
             pf = Prefill(lay.pools[0], lay.descs[0])
             line["prefill"] = prefill_measure(pf, 10, 3)
@@ -1255,8 +1271,8 @@ def main():
     ap.add_argument("--store-gb", type=float, default=24.0,
                     help="stack: pinned host store limit for slot misses")
     ap.add_argument("--no-extras", action="store_true",
-                    help="skip the NL3 / SB2 decode and 48-layer stack objects "
-                         "of the default line")
+                    help="skip the decode T sweep, NL3 / SB2 decode and 48-layer stack "
+                         "objects of the default line")
     ap.add_argument("--stack-steps", type=int, default=16,
                     help="steps of the default line's compact stack object")
     ap.add_argument("--no-prefill", action="store_true",
