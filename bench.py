@@ -211,16 +211,25 @@ def blas_threads() -> int:
         return os.cpu_count() or 1
 
 
-def cpu_baseline(T: int) -> dict:
+def cpu_baseline(T: int, seconds: float = 10.0) -> dict:
+    """The oracle on whole T-token decode steps (the layers rotated as in
+    the GPU measurement) until about `seconds` of host time have passed."""
     t0 = time.perf_counter()
-    done = oracle_step(layer=0, step=0, T=T, tokens=range(T))
+    done, n = 0.0, 0
+    while True:
+        done += oracle_step(layer=n % 8, step=n, T=T, tokens=range(T))
+        n += 1
+        if time.perf_counter() - t0 >= seconds:
+            break
     dt = time.perf_counter() - t0
+    steps = (f"one whole {T}-token decode step of layer 0" if n == 1 else
+             f"{n} whole {T}-token decode steps (layers 0..{min(n, 8) - 1} "
+             f"in turn)")
     return {"value": done / dt, "unit": "tokens/s", "cores": blas_threads(),
             "kind": "oracle",
-            "sample": (f"one {T}-token decode step of layer 0: fp64 routing of "
-                       f"all {T} tokens, then dequantisation and fp64 SwiGLU "
-                       f"FFN of every chosen expert and the combine "
-                       f"({dt:.1f} s)")}
+            "sample": (f"{steps}: fp64 routing of all {T} tokens, then "
+                       f"dequantisation and fp64 SwiGLU FFN of every chosen "
+                       f"expert and the combine ({dt:.1f} s)")}
 
 
 def run_reference(args) -> None:
