@@ -121,6 +121,22 @@ class ExpertParallelLayer:
             blob_stride=shape.blob_stride)
         self.torch = torch
         self.last_rows: Optional[int] = None
+        # name -> (device buffer, rows it was last laid out for): reused
+        # while the received row count stays the same; a workspace laid out
+        # for another count is zeroed first (its counters sit elsewhere)
+        self._ws = {}
+
+    def _buf(self, name: str, n: int, dtype, device, rows: int):
+        """The first n elements of a reusable device buffer, zero unless it
+        served a call with the same received row count before."""
+        b, last = self._ws.get(name, (None, None))
+        if b is None or b.numel() < n or b.device != device:
+            b, last = self.torch.zeros(max(n, 1), dtype=dtype,
+                                       device=device), rows
+        elif last != rows:
+            b.zero_()
+        self._ws[name] = (b, rows)
+        return b[:n]
 
     def forward(self, x, out) -> None:
         """x bf16 bits [T x H] (int16 tensor, device); out fp32 [T x H]."""
@@ -136,18 +152,18 @@ class ExpertParallelLayer:
         self.last_rows = n
         y_recv = torch.zeros((n, H), device=x.device)
         if n:
-            El = ep.n_local
+            El, dev = ep.n_local, x.device
+            i32, u8 = torch.int32, torch.uint8
             gws_b = moe.moe_group_workspace_bytes(n, 1, El)
-            gws = torch.zeros(max(256, gws_b), dtype=torch.uint8,
-                              device=x.device)
-            off = torch.empty(El + 1, dtype=torch.int32, device=x.device)
-            prs = torch.empty(n, dtype=torch.int32, device=x.device)
-            act = torch.empty(El, dtype=torch.int32, device=x.device)
-            na = torch.zeros(1, dtype=torch.int32, device=x.device)
+            gws = self._buf("gws", max(256, gws_b), u8, dev, n)
+            off = self._buf("off", El + 1, i32, dev, n)
+            prs = self._buf("prs", n, i32, dev, n)
+            act = self._buf("act", El, i32, dev, n)
+            na = self._buf("na", 1, i32, dev, n)
             moe.moe_group_tokens(lid, n, 1, El, off, prs, act, na, gws,
                                  gws_b)
             fws_b = moe.moe_ffn_workspace_bytes(n, 1, H, shp.F)
-            fws = torch.zeros(fws_b, dtype=torch.uint8, device=x.device)
+            fws = self._buf("fws", fws_b, u8, dev, n)
             moe.moe_expert_ffn_q(self.desc, x_recv, n, 1, off, prs, act, na,
                                  None, y_recv, fws, fws_b)
         y_pairs = ep.combine(y_recv, plan)

@@ -38,13 +38,21 @@ def test_expert_parallel_layer_one_rank_nccl():
         pool = build_pool(shape, 0, 0)
         ep = ExpertParallel(E, k)
         assert ep.n_local == E
-        for T in (3, 40):
+        layer, first = None, {}
+        # one layer object for all calls: its reused workspaces change
+        # layout between the decode and prefill row counts and back
+        for T in (3, 40, 3, 40):
             x, wr, _ = route_inputs(shape, 0, 0, T, step=8)
-            layer = ExpertParallelLayer(ep, shape, pool, dev(wr))
+            if layer is None:
+                layer = ExpertParallelLayer(ep, shape, pool, dev(wr))
             out = torch.full((T, H), float("nan"), device="cuda")
             idx, w = layer.forward(dev(x), out)
             torch.cuda.synchronize()
             assert layer.last_rows == T * k
+            if T in first:
+                assert torch.equal(out, first[T])
+                continue
+            first[T] = out.clone()
             gi = idx.cpu().numpy()
             ref = o.moe_layer(o.bf16_to_f64(x), o.bf16_to_f64(wr), None, k,
                               oracle_experts(shape, 0, 0), topk_idx=gi)
