@@ -90,7 +90,8 @@ WIDE20 = synth.LayerShape(H=512, F=256, E=1024, k=20,
 @pytest.mark.parametrize("shape,T,zipf", [
     (synth.TINY, 8, False), (synth.BIG, 1, False), (synth.BIG, 3, False),
     (synth.BIG, 3, True), (synth.TINY, 16, False),
-    (synth.BIG, 2, False), (synth.BIG, 5, False), (synth.BIG, 8, True),
+    (synth.BIG, 2, False), (synth.BIG, 4, False), (synth.BIG, 5, False),
+    (synth.BIG, 8, True),
     (WIDE, 3, False), (WIDE, 7, True), (WIDE20, 8, False),
 ])
 def test_layer_forward_vs_oracle(shape, T, zipf):
