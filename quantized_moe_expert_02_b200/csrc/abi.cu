@@ -3,6 +3,7 @@
 #include <mutex>
 
 #include "moe_internal.cuh"
+#include "trace.h"
 
 namespace moe {
 
@@ -303,6 +304,7 @@ extern "C" moe_status moe_route_topk(const uint16_t* x, int T, int H,
                                      const float* bias, int k,
                                      int32_t* topk_idx, float* topk_w,
                                      float* logits_out, void* stream) {
+  MOE_TRACE();
   if (!x || !w_router || !topk_idx || !topk_w || !logits_out)
     return logits_out ? MOE_ERR_INVALID : MOE_ERR_WORKSPACE;
   if (T <= 0 || H <= 0 || H % 8 || E <= 0 || E > EMAX || k < 1 || k > 32 ||
@@ -323,6 +325,7 @@ extern "C" moe_status moe_group_tokens(const int32_t* topk_idx, int T, int k,
                                        int32_t* pair_ids, int32_t* active,
                                        int32_t* n_active, void* ws,
                                        size_t ws_bytes, void* stream) {
+  MOE_TRACE();
   if (!topk_idx || !expert_offsets || !pair_ids || !active || !n_active)
     return MOE_ERR_INVALID;
   if (T <= 0 || k <= 0 || E <= 0 || E > EMAX) return MOE_ERR_SHAPE;
@@ -347,6 +350,7 @@ extern "C" size_t moe_layer_workspace_bytes(int T, int k, int E, int H,
 
 extern "C" moe_status moe_workspace_init(void* ws, size_t ws_bytes,
                                          void* stream) {
+  MOE_TRACE();
   if (!ws) return MOE_ERR_WORKSPACE;
   MOE_CUDA_TRY(cudaMemsetAsync(ws, 0, ws_bytes, (cudaStream_t)stream));
   return MOE_OK;
@@ -357,6 +361,7 @@ extern "C" moe_status moe_expert_up_q(
     const int32_t* expert_offsets, const int32_t* pair_ids,
     const int32_t* active, const int32_t* n_active,
     const int32_t* blob_index, void* ws, size_t ws_bytes, void* stream) {
+  MOE_TRACE();
   if (!x || ((uintptr_t)x & 15)) return MOE_ERR_INVALID;
   moe_status st = check_ffn_args(desc, T, k, expert_offsets, pair_ids, active,
                                  n_active, ws, ws_bytes);
@@ -370,6 +375,7 @@ extern "C" moe_status moe_expert_up_gemm_q(
     const moe_layer_desc* desc, int T, int k, const int32_t* expert_offsets,
     const int32_t* pair_ids, const int32_t* active, const int32_t* n_active,
     const int32_t* blob_index, void* ws, size_t ws_bytes, void* stream) {
+  MOE_TRACE();
   moe_status st = check_ffn_args(desc, T, k, expert_offsets, pair_ids, active,
                                  n_active, ws, ws_bytes);
   if (st != MOE_OK) return st;
@@ -386,6 +392,7 @@ extern "C" moe_status moe_expert_down_q(
     const int32_t* blob_index, float* y_pairs, const float* topk_w,
     const float* residual, float* out, uint16_t* out_bf16, void* ws,
     size_t ws_bytes, void* stream) {
+  MOE_TRACE();
   if (!y_pairs && !out) return MOE_ERR_INVALID;
   if (out && !topk_w) return MOE_ERR_INVALID;
   moe_status st = check_ffn_args(desc, T, k, expert_offsets, pair_ids, active,
@@ -403,6 +410,7 @@ extern "C" moe_status moe_expert_ffn_q(
     const int32_t* active, const int32_t* n_active,
     const int32_t* blob_index, float* y_pairs, void* ws, size_t ws_bytes,
     void* stream) {
+  MOE_TRACE();
   if (!y_pairs || !x || ((uintptr_t)x & 15)) return MOE_ERR_INVALID;
   moe_status st = check_ffn_args(desc, T, k, expert_offsets, pair_ids, active,
                                  n_active, ws, ws_bytes);
@@ -424,6 +432,7 @@ extern "C" moe_status moe_expert_ffn_combine_q(
     const int32_t* blob_index, const float* topk_w, const float* residual,
     float* out, uint16_t* out_bf16, void* ws, size_t ws_bytes,
     void* stream) {
+  MOE_TRACE();
   if (!out || !topk_w || !x || ((uintptr_t)x & 15)) return MOE_ERR_INVALID;
   moe_status st = check_ffn_args(desc, T, k, expert_offsets, pair_ids, active,
                                  n_active, ws, ws_bytes);
@@ -444,6 +453,7 @@ extern "C" moe_status moe_layer_forward(
     const float* residual, float* out, uint16_t* out_bf16, int32_t* topk_idx,
     float* topk_w, float* logits_out, void* ws, size_t ws_bytes,
     void* stream) {
+  MOE_TRACE();
   moe_status st = check_desc(desc);
   if (st != MOE_OK) return st;
   if (!x || !w_router || !out || !topk_idx || !topk_w) return MOE_ERR_INVALID;
@@ -497,6 +507,7 @@ extern "C" moe_status moe_layer_forward_residual(
     const uint16_t* w_router, const float* bias, const int32_t* blob_index,
     float* r_out, uint16_t* out_bf16, int32_t* topk_idx, float* topk_w,
     float* logits_out, void* ws, size_t ws_bytes, void* stream) {
+  MOE_TRACE();
   LayerWs w;
   moe_status st = check_residual_args(desc, r, T, k, ws, ws_bytes, &w);
   if (st != MOE_OK) return st;
@@ -529,6 +540,7 @@ extern "C" moe_status moe_layer_route_residual(
     const uint16_t* w_router, const float* bias, int32_t* topk_idx,
     float* topk_w, float* logits_out, void* ws, size_t ws_bytes,
     void* stream) {
+  MOE_TRACE();
   LayerWs w;
   moe_status st = check_residual_args(desc, r, T, k, ws, ws_bytes, &w);
   if (st != MOE_OK) return st;
@@ -552,6 +564,7 @@ extern "C" moe_status moe_layer_ffn_residual(
     const int32_t* topk_idx, const float* topk_w, const int32_t* blob_index,
     float* r_out, uint16_t* out_bf16, void* ws, size_t ws_bytes,
     void* stream) {
+  MOE_TRACE();
   LayerWs w;
   moe_status st = check_residual_args(desc, r, T, k, ws, ws_bytes, &w);
   if (st != MOE_OK) return st;
@@ -594,6 +607,7 @@ extern "C" moe_status moe_layer_ffn_residual_staged(
     const int32_t* miss_expert, const int32_t* miss_slot, int layer, int L,
     const uint64_t* table, int slot_base, int n_slots, int64_t pool_slots,
     void* ws, size_t ws_bytes, void* stream) {
+  MOE_TRACE();
   LayerWs w;
   moe_status st = check_residual_args(desc, r, T, k, ws, ws_bytes, &w);
   if (st != MOE_OK) return st;
@@ -629,6 +643,7 @@ extern "C" moe_status moe_layer_ffn_residual_staged(
 
 extern "C" moe_status moe_get_device_status(void* ws, int32_t* host_err,
                                             void* stream) {
+  MOE_TRACE();
   if (!ws) return MOE_ERR_WORKSPACE;
   cudaStream_t s = (cudaStream_t)stream;
   int32_t v = 0;

@@ -1,6 +1,7 @@
 // Weighted combine of the k expert outputs of each token, and the
 // row-wise RMS normalisation used between the layers of a stack.
 #include "moe_internal.cuh"
+#include "trace.h"
 
 namespace moe {
 
@@ -128,6 +129,7 @@ extern "C" moe_status moe_combine(const float* y_pairs, const float* topk_w,
                                   int T, int k, int H, const float* residual,
                                   float* out, uint16_t* out_bf16,
                                   void* stream) {
+  MOE_TRACE();
   if (!y_pairs || !topk_w || !out) return MOE_ERR_INVALID;
   if (T <= 0 || k <= 0 || H <= 0) return MOE_ERR_SHAPE;
   return launch_combine(y_pairs, topk_w, T, k, H, residual, out, out_bf16,
@@ -136,6 +138,7 @@ extern "C" moe_status moe_combine(const float* y_pairs, const float* topk_w,
 
 extern "C" moe_status moe_rmsnorm_bf16(const float* r, int T, int H,
                                        uint16_t* x_out, void* stream) {
+  MOE_TRACE();
   if (!r || !x_out) return MOE_ERR_INVALID;
   if (T <= 0 || H <= 0) return MOE_ERR_SHAPE;
   return launch_rmsnorm_bf16(r, T, H, x_out, (cudaStream_t)stream);

@@ -13,6 +13,7 @@
 //  prefill : the fp16 A-operand tiles that the dequant warps of the
 //            grouped GEMM write to shared memory (prefill.cu), un-swizzled.
 #include "decode_pieces.cuh"
+#include "trace.h"
 
 namespace moe {
 
@@ -97,6 +98,7 @@ using namespace moe;
 extern "C" moe_status moe_dequant_path(int fmt, int path,
                                        const uint8_t* packed, int rows,
                                        int cols, void* out, void* stream) {
+  MOE_TRACE();
   if (!packed || !out) return MOE_ERR_INVALID;
   if (!fmt_valid(fmt)) return MOE_ERR_INVALID;
   if (path != MOE_DQ_DECODE && path != MOE_DQ_PREFILL) return MOE_ERR_INVALID;

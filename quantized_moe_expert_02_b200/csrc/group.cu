@@ -2,6 +2,7 @@
 // expert, stable in p -- the per-expert token lists that the expert GEMMs
 // of the "llama-halo-hybrid" post's MoE path consume.
 #include "moe_internal.cuh"
+#include "trace.h"
 
 namespace moe {
 
@@ -291,6 +292,7 @@ extern "C" moe_status moe_group_subset(
     const int32_t* expert_offsets, const int32_t* pair_ids, int E,
     const int32_t* experts, int n, int32_t* sub_offsets, int32_t* sub_pairs,
     int32_t* sub_active, int32_t* sub_n_active, int32_t* err, void* stream) {
+  MOE_TRACE();
   if (!expert_offsets || !pair_ids || !experts || !sub_offsets ||
       !sub_pairs || !sub_active || !sub_n_active || !err)
     return MOE_ERR_INVALID;

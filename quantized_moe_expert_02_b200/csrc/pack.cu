@@ -4,6 +4,7 @@
 // sub-scales per 32), the 4-bit non-uniform-codebook type, and this
 // library's 3-bit non-uniform-codebook super-block (NL3).
 #include "moe_internal.cuh"
+#include "trace.h"
 
 namespace moe {
 
@@ -223,6 +224,7 @@ extern "C" size_t moe_blob_bytes(int fmt_up_gate, int fmt_down, int H,
 extern "C" moe_status moe_pack_tensor(int fmt, const uint8_t* natural,
                                       int rows, int cols, uint8_t* packed,
                                       void* stream) {
+  MOE_TRACE();
   if (!natural || !packed) return MOE_ERR_INVALID;
   if (!fmt_valid(fmt)) return MOE_ERR_INVALID;
   if (!packed_shape_ok(fmt, rows, cols)) return MOE_ERR_SHAPE;
@@ -247,6 +249,7 @@ extern "C" moe_status moe_pack_tensor(int fmt, const uint8_t* natural,
 
 extern "C" moe_status moe_dequant(int fmt, const uint8_t* packed, int rows,
                                   int cols, float* out, void* stream) {
+  MOE_TRACE();
   if (!packed || !out) return MOE_ERR_INVALID;
   if (!fmt_valid(fmt)) return MOE_ERR_INVALID;
   if (!packed_shape_ok(fmt, rows, cols)) return MOE_ERR_SHAPE;

@@ -2,6 +2,7 @@
 // expert slots with non-uniform per-layer capacity; an in-stream kernel
 // resolves hits and reports only the misses).  One block per call.
 #include "moe_internal.cuh"
+#include "trace.h"
 
 namespace moe {
 
@@ -151,6 +152,7 @@ extern "C" moe_status moe_slot_resolve(const int32_t* topk_idx, int T, int k,
                                        int32_t* miss_expert,
                                        int32_t* miss_slot, int32_t* n_miss,
                                        int32_t* err, void* stream) {
+  MOE_TRACE();
   return slot_resolve(topk_idx, T, k, E, slot_table, slot_owner, last_use,
                       n_slots, slot_base, stamp, nullptr, blob_index,
                       miss_expert, miss_slot, n_miss, err, stream);
@@ -161,6 +163,7 @@ extern "C" moe_status moe_slot_resolve_dev(
     int32_t* slot_owner, uint32_t* last_use, int n_slots, int slot_base,
     uint32_t* stamp, int32_t* blob_index, int32_t* miss_expert,
     int32_t* miss_slot, int32_t* n_miss, int32_t* err, void* stream) {
+  MOE_TRACE();
   if (!stamp) return MOE_ERR_INVALID;
   return slot_resolve(topk_idx, T, k, E, slot_table, slot_owner, last_use,
                       n_slots, slot_base, 0u, stamp, blob_index, miss_expert,

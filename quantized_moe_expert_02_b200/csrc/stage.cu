@@ -13,6 +13,7 @@
 #include <vector>
 
 #include "moe_internal.cuh"
+#include "trace.h"
 
 namespace moe {
 namespace {
@@ -71,6 +72,7 @@ __global__ void __launch_bounds__(STAGE_THREADS)
 
 extern "C" moe_status moe_stage_table(const void* const* host_blob, int n,
                                       uint64_t* table, void* stream) {
+  MOE_TRACE();
   if (!host_blob || !table || n < 1) return MOE_ERR_INVALID;
   std::vector<uint64_t> t((size_t)n, 0ull);
   for (int i = 0; i < n; ++i) {
@@ -111,6 +113,7 @@ extern "C" moe_status moe_stage_misses(const int32_t* n_miss,
                                        int64_t blob_stride,
                                        int64_t blob_bytes, int32_t* err,
                                        void* stream) {
+  MOE_TRACE();
   if (!n_miss || !miss_expert || !miss_slot || !table || !pool)
     return MOE_ERR_INVALID;
   if (P < 1 || layer < 0 || layer >= L || E < 1 || slot_base < 0 ||
