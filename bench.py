@@ -38,6 +38,7 @@ DOWN_BYTES = synth.BIG.down_bytes
 BLOB = synth.BIG.blob_bytes
 WR_BYTES = synth.BIG.E * synth.BIG.H * 2   # bf16 router of one layer
 LAUNCHES_PER_STEP = 1                      # the one-kernel decode layer
+SEED = 0                                   # input seed (--seed)
 
 
 KERNEL_SOURCES = ["quantized_moe_expert_02_b200/csrc/decode_layer.cu",
@@ -161,10 +162,10 @@ def oracle_step(layer: int, step: int, T: int, tokens, n_experts=None):
     (fractional when a token is sampled)."""
     import oracle as o
     shp = synth.BIG
-    x = o.bf16_to_f64(synth.gen_x(0, T, shp.H, step))
-    wr = o.bf16_to_f64(synth.gen_router(0, layer, shp.E, shp.H))
+    x = o.bf16_to_f64(synth.gen_x(SEED, T, shp.H, step))
+    wr = o.bf16_to_f64(synth.gen_router(SEED, layer, shp.E, shp.H))
     src = o.ExpertSource(shp.H, shp.F, shp.fmt_up_gate, shp.fmt_down,
-                         lambda e: synth.gen_expert_blob(shp, 0, layer, e))
+                         lambda e: synth.gen_expert_blob(shp, SEED, layer, e))
     logits = o.router_logits(x, wr, None)
     idx, w = o.route(logits, shp.k)
     done = 0.0
@@ -186,11 +187,11 @@ def cpu_baseline_prefill(n_tokens: int = 4) -> dict:
     import oracle as o
     shp = synth.BIG
     t0 = time.perf_counter()
-    x = o.bf16_to_f64(synth.gen_x(0, PF_T, shp.H, 0)[:n_tokens])
-    wr = o.bf16_to_f64(synth.gen_router(0, 0, shp.E, shp.H))
-    bias = synth.gen_zipf_bias(0, 0, shp.E)[0]
+    x = o.bf16_to_f64(synth.gen_x(SEED, PF_T, shp.H, 0)[:n_tokens])
+    wr = o.bf16_to_f64(synth.gen_router(SEED, 0, shp.E, shp.H))
+    bias = synth.gen_zipf_bias(SEED, 0, shp.E)[0]
     src = o.ExpertSource(shp.H, shp.F, shp.fmt_up_gate, shp.fmt_down,
-                         lambda e: synth.gen_expert_blob(shp, 0, 0, e))
+                         lambda e: synth.gen_expert_blob(shp, SEED, 0, e))
     o.moe_layer(x, wr, bias, shp.k, src)
     dt = time.perf_counter() - t0
     return {"value": n_tokens / dt, "unit": "tokens/s",
@@ -282,7 +283,7 @@ def workload_config(args) -> dict:
             "l2": (f"inputs larger than L2: steps rotate over {args.layers} "
                    f"resident layers x {synth.BIG.E * synth.BIG.blob_stride / 1e9:.2f}"
                    f" GB of experts"),
-            "parallelism": f"replicas x{args.gpus}"}
+            "parallelism": f"replicas x{args.gpus}", "seed": SEED}
 
 
 # ---------------------------------------------------------------- GPU ----
@@ -297,9 +298,10 @@ class Layers:
         self.moe, self.torch, self.dev = moe, torch, dev
         shp = self.shape = synth.BIG if shape is None else shape
         self.L, self.n_x = L, n_x
-        self.pools = [build_pool(shp, 0, l) for l in range(L)]
+        self.pools = [build_pool(shp, SEED, l) for l in range(L)]
         self.descs = [layer_desc(shp, p) for p in self.pools]
-        self.wr = [dev(synth.gen_router(0, l, shp.E, shp.H)) for l in range(L)]
+        self.wr = [dev(synth.gen_router(SEED, l, shp.E, shp.H))
+                   for l in range(L)]
         self.bufs = {}
 
     def buffers(self, T: int):
@@ -307,7 +309,8 @@ class Layers:
             return self.bufs[T]
         torch, moe, shp = self.torch, self.moe, self.shape
         b = {}
-        b["xs"] = [self.dev(synth.gen_x(0, T, shp.H, s)) for s in range(self.n_x)]
+        b["xs"] = [self.dev(synth.gen_x(SEED, T, shp.H, s))
+                   for s in range(self.n_x)]
         b["ws_bytes"] = moe.moe_layer_workspace_bytes(T, shp.k, shp.E, shp.H,
                                                       shp.F)
         b["ws"] = torch.zeros(b["ws_bytes"], dtype=torch.uint8, device="cuda")
@@ -391,7 +394,7 @@ def prefill_e2e_time(pf, steps: int, warmup: int) -> float:
     the output of step i comes back while step i+1 computes)."""
     import torch
     H = synth.BIG.H
-    xh = [torch.from_numpy(synth.gen_x(0, pf.T, H, s).view(np.int16))
+    xh = [torch.from_numpy(synth.gen_x(SEED, pf.T, H, s).view(np.int16))
           .pin_memory() for s in range(2)]
     oh = [torch.empty((pf.T, H), dtype=torch.float32).pin_memory()
           for _ in range(2)]
@@ -449,7 +452,7 @@ def e2e_time(lay, T: int, steps: int, warmup: int) -> float:
     import torch
     H = synth.BIG.H
     nh = lay.L * 4
-    xh = [torch.from_numpy(synth.gen_x(0, T, H, s).view(np.int16))
+    xh = [torch.from_numpy(synth.gen_x(SEED, T, H, s).view(np.int16))
           .pin_memory() for s in range(nh)]
     oh = [torch.empty((T, H), dtype=torch.float32).pin_memory()
           for _ in range(nh)]
@@ -610,7 +613,7 @@ def prefill_slots_measure(pool, cap: int = 92, borrow: int = 8,
     from synth.prefill_slots import Partition, PrefillSlots
     import quantized_moe_expert_02_b200 as moe
     shp, T = synth.BIG, PF_T
-    _, rank = synth.gen_zipf_bias(0, l, shp.E)
+    _, rank = synth.gen_zipf_bias(SEED, l, shp.E)
     part = Partition(shp, pool, synth.hottest_experts(rank, cap), cap)
     store = torch.empty((shp.E, shp.blob_bytes), dtype=torch.uint8)
     store = store.pin_memory()
@@ -670,9 +673,9 @@ class Prefill:
         shp = synth.BIG
         self.moe, self.torch, self.T = moe, torch, T
         self.desc = desc
-        self.x = dev(synth.gen_x(0, T, shp.H, 0))
-        self.wr = dev(synth.gen_router(0, l, shp.E, shp.H))
-        self.bias = dev(synth.gen_zipf_bias(0, l, shp.E)[0])
+        self.x = dev(synth.gen_x(SEED, T, shp.H, 0))
+        self.wr = dev(synth.gen_router(SEED, l, shp.E, shp.H))
+        self.bias = dev(synth.gen_zipf_bias(SEED, l, shp.E)[0])
         k, E, H, F = shp.k, shp.E, shp.H, shp.F
         self.ws_bytes = moe.moe_layer_workspace_bytes(T, k, E, H, F)
         self.ws = torch.zeros(self.ws_bytes, dtype=torch.uint8, device="cuda")
@@ -783,7 +786,7 @@ def run_profile(args) -> None:
     import torch
     if args.workload == "prefill":
         from synth.pools import build_pool, layer_desc
-        pool = build_pool(synth.BIG, 0, 0)
+        pool = build_pool(synth.BIG, SEED, 0)
         pf = Prefill(pool, layer_desc(synth.BIG, pool))
         for i in range(args.warmup + args.steps):
             pf.step()
@@ -954,7 +957,7 @@ def stack_measure(S: int, W: int, reps: int, store_gb: float,
     L, T = 48, 3
     shp = synth.BIG
     t0 = time.perf_counter()
-    st = Stack(L, shp, seed=0, T=T)
+    st = Stack(L, shp, seed=SEED, T=T)
     setup_s = time.perf_counter() - t0
     xs = [st.x0(s) for s in range(S)]
     r = torch.empty_like(xs[0])
@@ -1156,7 +1159,7 @@ def run_stack(args) -> None:
                                 "48 x 512 experts resident"),
                    "T": T, "layers": L, "H": 3072, "F": 1024, "E": 512,
                    "k": 10, "l2": "inputs larger than L2: 105 GB of experts",
-                   "parallelism": "replicas x1"},
+                   "parallelism": "replicas x1", "seed": SEED},
         "layer_gbs": res["gbs"], "layer_frac_of_hbm": res["frac"],
         "roofline": {"bound": "hbm", "kernel": "decode_layer_kernel x 48",
                      "achieved": res["gbs"], "peak": res["peak"],
@@ -1193,7 +1196,7 @@ def run_prefill(args) -> None:
         import datetime
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
-    pool = build_pool(synth.BIG, 0, 0)
+    pool = build_pool(synth.BIG, SEED, 0)
     pf = Prefill(pool, layer_desc(synth.BIG, pool))
     K, W = args.steps, args.warmup
     for _ in range(W):
@@ -1227,7 +1230,7 @@ def run_prefill(args) -> None:
                        "F": 1024, "E": 512, "k": 10,
                        "l2": "inputs larger than L2: 2.19 GB of experts, "
                              "1.17 GB y_pairs per step",
-                       "parallelism": f"replicas x{world}"},
+                       "parallelism": f"replicas x{world}", "seed": SEED},
             "tflops": fl["total"] / (ms / K * 1e-3) / 1e12,
             "roofline": {
                 "bound": "tensor",
@@ -1262,6 +1265,10 @@ def run_prefill(args) -> None:
         print(json.dumps(line), flush=True)
 
 
+# Named workloads (the tiny 8-token shape is a parity case, not a bench line)
+CONFIGS = {"c1": "decode", "c2": "stack", "c3": "prefill", "c4": "stack"}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -1286,7 +1293,19 @@ def main():
                     help="steps of the default line's compact stack object")
     ap.add_argument("--no-prefill", action="store_true",
                     help="leave the prefill figures out of the decode line")
+    ap.add_argument("--seed", type=int, default=0,
+                    help="seed of every synthetic input (activations, "
+                         "router, experts, Zipf bias)")
+    ap.add_argument("--config", choices=sorted(CONFIGS),
+                    help="a named workload: c1 one decode layer (--T tokens),"
+                         " c2 / c4 the 48-layer stack, resident and through "
+                         "the slot pool (one line), c3 the 9536-token "
+                         "prefill chunk")
     args = ap.parse_args()
+    if args.config:
+        args.workload = CONFIGS[args.config]
+    global SEED
+    SEED = args.seed
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
