@@ -780,6 +780,27 @@ def prefill_measure(pf: "Prefill", steps: int, warmup: int) -> dict:
     }
 
 
+def prefill_sweep(pool, sizes=(1024, 2048, 4096, 9536, 16384, 32768),
+                  steps: int = 5) -> dict:
+    """The prefill layer at other chunk sizes (same layer, same Zipf-biased
+    routing): per-layer time, tokens/s and the fraction of the measured
+    bf16 peak of its FLOPs (expert GEMMs and router)."""
+    import torch
+    from synth.pools import layer_desc
+    _, tf, _ = peaks()
+    out = {}
+    for T in sizes:
+        pf = Prefill(pool, layer_desc(synth.BIG, pool), T=T)
+        ms = events_time(pf.step, steps, 2)
+        fl = prefill_flops(T)
+        out[str(T)] = {"ms_per_layer": ms, "tokens_per_s": T / (ms / 1e3),
+                       "frac_of_bf16_peak":
+                           fl["total"] / (ms * 1e-3) / 1e12 / tf}
+        del pf
+        torch.cuda.empty_cache()
+    return out
+
+
 def run_profile(args) -> None:
     """Launches for ncu: W warm-up steps then K steps, eager (5 kernels
     each), nothing else on the GPU after the pools are built."""
@@ -1258,6 +1279,10 @@ def run_prefill(args) -> None:
         }
         if not args.no_cpu_baseline and world == 1:
             line["cpu_baseline"] = cpu_baseline_prefill()
+        if world == 1 and not args.no_extras:
+            del pf
+            torch.cuda.empty_cache()
+            line["prefill_sweep"] = prefill_sweep(pool)
     if dist:
         dist.barrier()
         dist.destroy_process_group()
