@@ -12,7 +12,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 def test_reference_arm_json_line():
     out = subprocess.run(
         [sys.executable, os.path.join(ROOT, "bench.py"), "--impl",
-         "reference", "--steps", "1", "--warmup", "3"],
+         "reference", "--config", "c1", "--seed", "1", "--steps", "1",
+         "--warmup", "3"],
         cwd=ROOT, capture_output=True, text=True, timeout=600, check=True)
     lines = [l for l in out.stdout.splitlines() if l.startswith("{")]
     assert len(lines) == 1
@@ -26,6 +27,7 @@ def test_reference_arm_json_line():
     assert d["unit"] == "tokens/s" and d["higher_is_better"] is True
     assert d["value"] > 0 and d["ms_per_step"] > 0
     assert "workload" in d["config"] and d["config"]["T"] == 3
+    assert d["config"]["seed"] == 1
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["sample"]
     assert cb["value"] == d["value"]
